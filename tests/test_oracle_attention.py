@@ -1,0 +1,95 @@
+"""Pins for the oracle's sparse MQA attention (no GPU).
+
+Pinned against torch.nn.functional.scaled_dot_product_attention (float64,
+CPU) on the dense special case (every entry selected, with and without the
+window rows), and closed forms: identical keys, zero query (uniform
+weights), a single key, skipped -1 slots, permutation invariance.
+"""
+
+import numpy as np
+import torch
+
+from oracle import attention, fp4
+
+
+def _rng(s):
+    return np.random.default_rng(s)
+
+
+def _sdpa(q, keys, scale):
+    qt = torch.from_numpy(q)[:, None, :]                           # [64, 1, 512]
+    kt = torch.from_numpy(keys)[None].expand(q.shape[0], -1, -1)   # MQA: one KV head
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, kt, scale=scale)
+    return o[:, 0, :].numpy()
+
+
+def test_dense_case_matches_sdpa():
+    rng = _rng(0)
+    N = 96
+    kv = fp4.quantize_kv_fp4(rng.normal(size=(N, 512)).astype(np.float32))
+    deq = fp4.dequantize_kv_fp4(kv)
+    q = rng.normal(size=(64, 512)) * 0.1
+    o, lse = attention.sparse_mqa(q, deq, np.arange(N), np.zeros((0, 512)))
+    np.testing.assert_allclose(o, _sdpa(q, deq, 1 / np.sqrt(512)), rtol=1e-10, atol=1e-12)
+    logits = torch.from_numpy(q) @ torch.from_numpy(deq).T / np.sqrt(512)
+    np.testing.assert_allclose(lse, torch.logsumexp(logits, dim=1).numpy(), rtol=1e-12)
+
+
+def test_selected_plus_window_matches_sdpa_on_concatenation():
+    rng = _rng(1)
+    N = 300
+    deq = rng.normal(size=(N, 512))
+    idx = rng.choice(N, 40, replace=False)
+    swa = rng.normal(size=(128, 512))
+    q = rng.normal(size=(64, 512)) * 0.05
+    o, _ = attention.sparse_mqa(q, deq, idx, swa, scale=0.3)
+    ref = _sdpa(q, np.concatenate([deq[idx], swa]), 0.3)
+    np.testing.assert_allclose(o, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_identical_keys_return_that_key():
+    rng = _rng(2)
+    k = rng.normal(size=512)
+    deq = np.tile(k, (10, 1))
+    q = rng.normal(size=(64, 512))
+    o, lse = attention.sparse_mqa(q, deq, np.arange(10), np.tile(k, (3, 1)))
+    np.testing.assert_allclose(o, np.tile(k, (64, 1)), rtol=1e-12)
+    np.testing.assert_allclose(lse, np.log(13) + q @ k / np.sqrt(512), rtol=1e-12)
+
+
+def test_zero_query_gives_mean_of_keys():
+    rng = _rng(3)
+    deq = rng.normal(size=(50, 512)); swa = rng.normal(size=(7, 512))
+    idx = np.array([3, 9, 27, 49])
+    o, lse = attention.sparse_mqa(np.zeros((64, 512)), deq, idx, swa)
+    mean = np.concatenate([deq[idx], swa]).mean(axis=0)
+    np.testing.assert_allclose(o, np.tile(mean, (64, 1)), rtol=1e-12)
+    np.testing.assert_allclose(lse, np.log(11.0))
+
+
+def test_single_key_and_empty():
+    rng = _rng(4)
+    deq = rng.normal(size=(5, 512)); q = rng.normal(size=(64, 512))
+    o, _ = attention.sparse_mqa(q, deq, np.array([-1, 2, -1]), np.zeros((0, 512)))
+    np.testing.assert_allclose(o, np.tile(deq[2], (64, 1)), rtol=1e-12)
+    o, lse = attention.sparse_mqa(q, deq, np.array([-1, -1]), np.zeros((0, 512)))
+    assert np.all(o == 0) and np.all(lse == -np.inf)
+
+
+def test_skipped_slots_and_permutation():
+    rng = _rng(5)
+    deq = rng.normal(size=(64, 512)); swa = rng.normal(size=(4, 512))
+    q = rng.normal(size=(64, 512)) * 0.1
+    idx = np.array([5, 17, -1, 33, 60, -1])
+    o1, l1 = attention.sparse_mqa(q, deq, idx, swa)
+    o2, l2 = attention.sparse_mqa(q, deq, idx[::-1][[0, 1, 2, 3, 4, 5]], swa)
+    o3, l3 = attention.sparse_mqa(q, deq, idx[idx >= 0], swa)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-14); np.testing.assert_allclose(l1, l2, rtol=1e-12)
+    np.testing.assert_allclose(o1, o3, rtol=1e-12, atol=1e-14); np.testing.assert_allclose(l1, l3, rtol=1e-12)
+    # softmax weights sum to one: value rows shifted by a constant vector c
+    # shift every output by exactly c when the query is orthogonal to c
+    c = np.zeros(512); c[0] = 3.0
+    qo = q.copy(); qo[:, 0] = 0
+    oa, _ = attention.sparse_mqa(qo, deq, idx, swa)
+    ob, _ = attention.sparse_mqa(qo, deq + c, idx, swa + c)
+    np.testing.assert_allclose(ob - oa, np.tile(c, (64, 1)), atol=1e-12)

@@ -1,0 +1,95 @@
+"""Pins for the oracle's group schedule (no GPU): the mode identities the
+pages imply ([eogee] §3.2/§3.3): Reindex with the Full layer's own index-Q
+selects the same entries; Reuse then equals that Reindex layer; a pool that
+covers every block makes a pool-restricted Reindex equal a full one; new
+entries are quantised into the cache before scoring."""
+
+import numpy as np
+
+from oracle import fp4, group
+
+
+def _setup(seed, N=640, Q=2):
+    rng = np.random.default_rng(seed)
+    kv = fp4.quantize_kv_fp4(rng.normal(size=(N, 512)).astype(np.float32))
+    kI = rng.normal(size=(N, 128))
+    n_vis = np.array([N - 3, N][:Q])
+
+    def layer(mode, qI=None, w=None):
+        return dict(mode=mode,
+                    qI=rng.normal(size=(Q, 32, 128)) if qI is None else qI,
+                    w=rng.uniform(size=(Q, 32)) if w is None else w,
+                    q=rng.normal(size=(Q, 64, 512)) * 0.05,
+                    swa=rng.normal(size=(128, 512)))
+    return kv, kI, n_vis, layer
+
+
+def test_reindex_with_shared_index_q_equals_full_and_reuse_equals_it():
+    kv, kI, n_vis, layer = _setup(0)
+    L0 = layer(group.FULL)
+    L1 = layer(group.REINDEX, qI=L0["qI"], w=L0["w"])
+    L2 = layer(group.REUSE)
+    L2["q"], L2["swa"] = L1["q"], L1["swa"]
+    res = group.group_row(kv, kI, n_vis, [L0, L1, L2], K=64, W=128)
+    np.testing.assert_array_equal(res[0]["idx"], res[1]["idx"])
+    np.testing.assert_array_equal(res[1]["idx"], res[2]["idx"])
+    np.testing.assert_array_equal(res[1]["o"], res[2]["o"])
+    np.testing.assert_array_equal(res[1]["lse"], res[2]["lse"])
+
+
+def test_reuse_takes_the_most_recent_indexing_layer():
+    kv, kI, n_vis, layer = _setup(1)
+    res = group.group_row(kv, kI, n_vis, [layer(group.FULL), layer(group.REINDEX), layer(group.REUSE)], K=32)
+    np.testing.assert_array_equal(res[2]["idx"], res[1]["idx"])
+    assert not np.array_equal(res[0]["idx"], res[1]["idx"])
+
+
+def test_pool_covering_all_blocks_equals_full_reindex():
+    kv, kI, n_vis, layer = _setup(2)
+    L0 = layer(group.FULL)
+    L1 = layer(group.REINDEX_POOL)
+    L1b = dict(L1, mode=group.REINDEX)
+    r_pool = group.group_row(kv.copy(), kI, n_vis, [L0, L1], K=48, hsi_blocks=80, hsi_block=8)
+    r_full = group.group_row(kv.copy(), kI, n_vis, [L0, L1b], K=48)
+    np.testing.assert_array_equal(r_pool[1]["idx"], r_full[1]["idx"])
+    np.testing.assert_allclose(r_pool[1]["o"], r_full[1]["o"], rtol=1e-12)
+    assert r_pool[0]["pool"].shape == (2, 80)
+
+
+def test_new_entries_are_quantised_before_scoring():
+    kv, kI, n_vis, layer = _setup(3)
+    rng = np.random.default_rng(33)
+    new = rng.normal(size=(2, 512)).astype(np.float32) * 50       # large values: attention must see them
+    kv2 = kv.copy()
+    res = group.group_row(kv2, kI, n_vis, [layer(group.FULL)], K=16, kv_new=new, new_rows=[7, 9])
+    np.testing.assert_array_equal(kv2[[7, 9]], fp4.quantize_kv_fp4(new))
+    assert res[0]["o"].shape == (2, 64, 512)
+
+
+def test_topk_indices_valid_and_visible():
+    kv, kI, n_vis, layer = _setup(4, N=300, Q=2)
+    res = group.group_row(kv, kI, n_vis, [layer(group.FULL)], K=512)
+    for i in range(2):
+        idx = res[0]["idx"][i]
+        vis = idx[idx >= 0]
+        assert len(vis) == n_vis[i] and len(set(vis.tolist())) == n_vis[i]
+        assert np.all(idx[n_vis[i]:] == -1)
+        assert vis.max() < n_vis[i]
+
+
+
+def test_window_rows_follow_the_query_position():
+    """Zero query and all-zero main-KV entries: every key gets the same
+    weight, so channel 0 of the output is sum(window row ids) / (K + W).
+    Query i must see window rows [i*step, i*step + W)."""
+    N, Q, K, W, step = 64, 3, 8, 5, 2
+    kv = fp4.quantize_kv_fp4(np.zeros((N, 512), np.float32))
+    kI = np.random.default_rng(0).normal(size=(N, 128))
+    swa = np.zeros((W + (Q - 1) * step, 512))
+    swa[:, 0] = np.arange(swa.shape[0])
+    L = dict(mode=group.FULL, qI=np.ones((Q, 32, 128)), w=np.ones((Q, 32)),
+             q=np.zeros((Q, 64, 512)), swa=swa)
+    res = group.group_row(kv, kI, np.array([N] * Q), [L], K=K, W=W, swa_step=step)
+    for i in range(Q):
+        want = sum(range(i * step, i * step + W)) / (K + W)
+        np.testing.assert_allclose(res[0]["o"][i][:, 0], want, rtol=1e-12)
