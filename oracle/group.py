@@ -42,7 +42,6 @@ def group_row(kv_fp4, kI, n_vis, layers, K=indexer.TOPK, W=attention.WIN,
     """
     if kv_new is not None:
         kv_fp4[np.asarray(new_rows)] = fp4.quantize_kv_fp4(kv_new)
-    kv_deq = fp4.dequantize_kv_fp4(kv_fp4)
     n_vis = np.asarray(n_vis)
     Q = n_vis.shape[0]
     results = []
@@ -80,7 +79,10 @@ def group_row(kv_fp4, kI, n_vis, layers, K=indexer.TOPK, W=attention.WIN,
         swa = np.asarray(L["swa"], dtype=np.float64)
         for i in range(Q):
             rows = swa[i * swa_step: i * swa_step + W]
-            o[i], lse[i] = attention.sparse_mqa(L["q"][i], kv_deq, idx[i], rows, scale)
+            # attention reads only the selected entries: dequantise those
+            sel = idx[i][idx[i] >= 0]
+            deq = fp4.dequantize_kv_fp4(kv_fp4[sel])
+            o[i], lse[i] = attention.sparse_mqa(L["q"][i], deq, np.arange(sel.shape[0]), rows, scale)
         res.update(idx=idx, o=o, lse=lse)
         results.append(res)
     return results
