@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Throughput of one CSA2 decode group step over an FP4 main KV on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
+
+A step is one pass of the whole hot path over one batch: quantise the
+step's new main-KV entries into the FP4 cache, then every layer of the
+group in order (index scan + top-K for Full / Reindex / pool-Reindex
+layers, sparse MQA attention for every layer), through one
+csa2_group_decode call.  Default workload: the decoder group Full,
+Reindex, Reindex, Reuse at 131,072 entries (128K tokens, r=1), batch 4.
+
+Prints one JSON line (rank 0).  value = queries/s over all ranks (a query
+is one (row, position) carried through every layer), measured with CUDA
+events on the launching stream, max over ranks, caches resident in HBM,
+L2 flushed (256 MB memset) between steps outside the timed events.
+Under torchrun each rank runs its own copy of the workload (batch rows
+are independent sequences: no collective on the data path).
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp4_kv_cache_mxfp4_b200 import build as _build  # noqa: E402
+from fp4_kv_cache_mxfp4_b200 import workloads  # noqa: E402
+
+METRIC = "CSA2 decode queries/s and HBM GB/s vs peak at 128K ctx, FP4 main KV"
+UNIT = "queries/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of one index_scan_kernel launch, from the ncu capture
+# summarised in profiles/index_scan_kernel_group4_ctx128k.md, valid only
+# while the kernel sources hash to the recorded value.
+SCAN_TRAFFIC = {"sha": None, "bytes_per_launch": None}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=2)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (barrier and max-reduction only)
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the run
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, line in self.lines:
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1])); smax.append(float(p[2])); power.append(float(p[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------
+# workload on the device
+# ---------------------------------------------------------------------------
+
+def make_device_workload(wl, csa2, seed_shift=0):
+    d = "cuda"
+    B, Q, N, K = wl.B, wl.Q, wl.N, wl.K
+    if seed_shift:
+        wl = workloads.Workload(**{**wl.__dict__, "seed": wl.seed + 7919 * seed_shift, "n_vis": list(wl.n_vis)})
+    kv = torch.empty(B, N, 288, dtype=torch.uint8, device=d)
+    for b in range(B):
+        for r0 in range(0, N - wl.n_new, workloads.KV_CHUNK):
+            n = min(workloads.KV_CHUNK, N - wl.n_new - r0)
+            x = workloads.main_kv_rows(wl, b, r0, n).to(d)
+            csa2.csa2_quantize_kv_fp4(x, kv[b], row_offset=r0)
+    kI = torch.stack([workloads.index_k(wl, b) for b in range(B)]).to(d)
+    new = torch.cat([workloads.main_kv_rows(wl, b, N - wl.n_new, wl.n_new) for b in range(B)]).to(d)
+    new_rows = torch.tensor([b * N + r for b in range(B) for r in wl.new_rows], dtype=torch.int64, device=d)
+    layers = []
+    for l, mode in enumerate(wl.modes):
+        li = workloads.layer_inputs(wl, l)
+        layers.append(dict(mode=mode, qI=li["qI"].to(d), w=li["w"].to(d), q=li["q"].to(d), swa=li["swa"].to(d),
+                           out=torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=d),
+                           lse=torch.empty(B, Q, 64, device=d),
+                           idx=torch.empty(B, Q, K, dtype=torch.int32, device=d) if mode != workloads.REUSE else None))
+    pool = torch.empty(B, Q, wl.hsi_blocks, dtype=torch.int32, device=d) if wl.hsi_blocks else None
+    n_vis = workloads.n_vis_tensor(wl).to(d)
+    g = csa2.group_args(B, Q, K, wl.W, N, n_vis, kI, kv, layers, kv_new=new, new_rows=new_rows,
+                        swa_rows=wl.swa_rows, swa_step=wl.swa_step, hsi_blocks=wl.hsi_blocks,
+                        hsi_block=wl.hsi_block, pool=pool)
+    ws = csa2.workspace(g, csa2.WS_GROUP)
+    torch.cuda.synchronize()
+    return dict(g=g, ws=ws, kv=kv, kI=kI, new=new, new_rows=new_rows, layers=layers, pool=pool, n_vis=n_vis)
+
+
+def scan_algorithmic_bytes(wl):
+    """Bytes one index_scan_kernel launch must move (Full / Reindex scan):
+    index-K rows once, one fp32 score per (query, entry), index-Q and w."""
+    per_row = wl.N * 128 * 2 + wl.Q * wl.N * 4 + wl.Q * (32 * 128 * 2 + 32 * 4)
+    return wl.B * per_row
+
+
+def step_algorithmic_bytes(wl):
+    """Algorithmic HBM bytes of one whole step (same accounting as the
+    per-kernel figures): the scans, the new entries (read bf16, write FP4),
+    and per layer the gathered FP4 entries, the window, q and the output."""
+    n_index = sum(1 for m in wl.modes if m in (workloads.FULL, workloads.REINDEX))
+    total = n_index * scan_algorithmic_bytes(wl)
+    total += wl.B * wl.n_new * (1024 + 288)
+    per_query_attn = wl.K * 288 + wl.W * 1024 + 64 * 512 * 2 * 2
+    total += len(wl.modes) * wl.B * wl.Q * per_query_attn
+    return total
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("common.cuh", "index_scan.cuh"):
+        h.update(open(os.path.join(ROOT, "fp4_kv_cache_mxfp4_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# the oracle as CPU baseline / reference arm
+# ---------------------------------------------------------------------------
+
+def oracle_row_setup(wl, b):
+    """Host inputs of batch row b for the oracle: its FP4 cache built by the
+    oracle's own quantiser (only the rows the oracle's layers will read are
+    filled: attention reads nothing else), index-K and layer inputs."""
+    from oracle import fp4, group, indexer
+    x = workloads.main_kv_rows(wl, b, 0, wl.N).float().numpy()
+    kI = workloads.index_k(wl, b).float().numpy()
+    layers = []
+    for l, mode in enumerate(wl.modes):
+        li = workloads.layer_inputs(wl, l)
+        layers.append(dict(mode=mode, qI=li["qI"][b].float().numpy(), w=li["w"][b].numpy(),
+                           q=li["q"][b].float().numpy(), swa=li["swa"][b].float().numpy()))
+    need = set(wl.new_rows)
+    for L in layers:
+        if L["mode"] in (group.FULL, group.REINDEX):
+            for i in range(wl.Q):
+                s = indexer.index_scores(L["qI"][i], L["w"][i], kI, wl.n_vis[i])
+                need.update(int(p) for p in indexer.topk(s, wl.K)[0] if p >= 0)
+    rows = np.array(sorted(need))
+    kv = np.zeros((wl.N, 288), dtype=np.uint8)
+    kv[rows] = fp4.quantize_kv_fp4(x[rows])
+    new = x[wl.N - wl.n_new:].copy()
+    return dict(kv=kv, kI=kI, layers=layers, new=new)
+
+
+def oracle_row_step(wl, S):
+    from oracle import group
+    kv = S["kv"].copy()
+    return group.group_row(kv, S["kI"], np.array(wl.n_vis), S["layers"], K=wl.K, W=wl.W,
+                           swa_step=wl.swa_step, hsi_blocks=wl.hsi_blocks, hsi_block=wl.hsi_block,
+                           kv_new=S["new"], new_rows=wl.new_rows)
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(wl):
+    S = oracle_row_setup(wl, 0)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_row_step(wl, S)
+        n += 1
+        if time.perf_counter() - t0 > 10.0:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n * wl.Q / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"batch row 0 of {wl.name} through the oracle's full group step "
+                      f"({len(wl.modes)} layers, quantise + scan + top-K + attention), {n} repetition(s), "
+                      f"{dt:.1f} s; host os.cpu_count()={os.cpu_count()}"}
+
+
+def run_reference(args, world, rank):
+    wl = workloads.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    setups = [oracle_row_setup(wl, b) for b in range(wl.B)]
+    for _ in range(args.warmup):
+        oracle_row_step(wl, setups[0])
+    times = []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        for S in setups:
+            oracle_row_step(wl, S)
+        times.append(time.perf_counter() - t0)
+    mean = sum(times) / len(times)
+    value = wl.B * wl.Q / mean
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "N_entries": wl.N,
+                       "layers": ",".join(workloads.MODE_NAMES[m] for m in wl.modes), "K": wl.K, "W": wl.W,
+                       "parallelism": "oracle on host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"every batch row of {wl.name} per step through the oracle group "
+                                       f"schedule (numpy, float64); warm-up steps used row 0 only"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    if rank == 0:
+        _build.build()
+    barrier(world)
+    from fp4_kv_cache_mxfp4_b200 import csa2
+    csa2.load()
+    wl = workloads.WORKLOADS[args.workload]
+    T = make_device_workload(wl, csa2, seed_shift=rank)
+    st = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def step():
+        csa2.csa2_group_decode(T["g"], T["ws"])
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st_code = csa2.csa2_device_status()
+    if st_code != (0, 0):
+        raise RuntimeError(f"device status after warm-up: {st_code}")
+
+    # ---- timed: device-resident inputs
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush.zero_()
+        a.record(st)
+        step()
+        b.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+
+    # ---- traced pass: per-kernel durations with events on the launch stream
+    launches_per_step = None
+    csa2.csa2_trace_begin(64 * args.steps)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for a, b in ev2:
+        flush.zero_()
+        a.record(st)
+        step()
+        b.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    csa2.csa2_trace_stop()
+    recs = csa2.csa2_trace_records()
+    csa2.csa2_trace_end()
+    traced_ms = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
+    launches_per_step = len(recs) / args.steps
+    per_kernel = {}
+    for name, ms in recs:
+        c, t = per_kernel.get(name, (0, 0.0))
+        per_kernel[name] = (c + 1, t + ms)
+
+    # ---- end to end: host inputs -> device -> csa2_group_decode -> host outputs
+    host_in = [(T["new"], torch.empty_like(T["new"], device="cpu").pin_memory())]
+    for L in T["layers"]:
+        for k in ("qI", "w", "q"):
+            host_in.append((L[k], torch.empty_like(L[k], device="cpu").pin_memory()))
+    for dev_t, host_t in host_in:
+        host_t.copy_(dev_t)
+    host_out = [(L["out"], torch.empty_like(L["out"], device="cpu").pin_memory()) for L in T["layers"]]
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+    ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for a, b in ev3:
+        flush.zero_()
+        a.record(st)
+        for dev_t, host_t in host_in:
+            dev_t.copy_(host_t, non_blocking=True)
+        step()
+        for dev_t, host_t in host_out:
+            host_t.copy_(dev_t, non_blocking=True)
+        b.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev3) / args.steps, world)
+    clk = clocks.stop()
+    st_code = csa2.csa2_device_status()
+    if st_code != (0, 0):
+        raise RuntimeError(f"device status after the timed loops: {st_code}")
+
+    if rank != 0:
+        return
+    queries = wl.B * wl.Q * world
+    value = queries / (mean_ms * 1e-3)
+    peak, peak_kind = hbm_peak()
+    n_scan, t_scan = per_kernel.get("index_scan_kernel", (0, 0.0))
+    scan_ms = t_scan / max(n_scan, 1)
+    scan_bytes = scan_algorithmic_bytes(wl)
+    achieved = scan_bytes / (scan_ms * 1e-3) / 1e9 if n_scan else None
+    sha = kernel_source_sha()
+    traffic = SCAN_TRAFFIC["bytes_per_launch"] if SCAN_TRAFFIC["sha"] == sha else None
+    step_bytes = step_algorithmic_bytes(wl)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) caches and inputs)",
+        "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "N_entries": wl.N, "r": wl.r,
+                   "layers": ",".join(workloads.MODE_NAMES[m] for m in wl.modes), "K": wl.K, "W": wl.W,
+                   "kv_cache": "FP4 E2M1 + E4M3/16ch (288 B/entry)", "index_k": "bf16",
+                   "l2": "flushed between steps (256 MB memset outside the timed events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "hbm_gbs_step": step_bytes / (mean_ms * 1e-3) / 1e9,
+        "hbm_frac_step": step_bytes / (mean_ms * 1e-3) / 1e9 / peak,
+        "roofline": {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6.65 TB/s", "unit": "GB/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": scan_bytes, "ms_per_launch": scan_ms,
+                     "launches": n_scan},
+        "kernels": {k: {"launches": c, "ms_mean": t / c} for k, (c, t) in sorted(per_kernel.items())},
+        "ms_per_step_traced": traced_ms,
+        "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": int(round(launches_per_step * args.steps)) if launches_per_step else 0,
+        "clocks": clk,
+    }
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    else:
+        line["cpu_baseline"] = None
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,222 @@
+"""Python binding of libcsa2 (include/csa2.h): argument marshalling only.
+
+Every function takes torch CUDA tensors, passes their device pointers and
+the current CUDA stream to the C ABI and raises ``Csa2Error`` on a non-zero
+status.  All computation happens in the library's CUDA kernels; there is no
+fallback: if libcsa2.so is missing, ``load()`` raises.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa2.so")
+
+FULL, REINDEX, REINDEX_POOL, REUSE = 0, 1, 2, 3
+WS_INDEX, WS_ATTN, WS_GROUP = 1, 2, 3
+ENTRY_BYTES = 288
+
+_c_i32, _c_i64, _c_f32, _c_p = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
+
+
+class Csa2Error(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class IndexArgs(ctypes.Structure):
+    _fields_ = [("mode", _c_i32), ("B", _c_i32), ("Q", _c_i32), ("K", _c_i32), ("N", _c_i64),
+                ("qI", _c_p), ("w", _c_p), ("kI", _c_p), ("n_vis", _c_p), ("idx", _c_p), ("scores", _c_p),
+                ("hsi_blocks", _c_i32), ("hsi_block", _c_i32), ("pool_out", _c_p), ("pool_in", _c_p)]
+
+
+class AttnArgs(ctypes.Structure):
+    _fields_ = [("B", _c_i32), ("Q", _c_i32), ("K", _c_i32), ("W", _c_i32), ("N", _c_i64),
+                ("q", _c_p), ("kv_fp4", _c_p), ("idx", _c_p), ("swa", _c_p),
+                ("swa_rows", _c_i32), ("swa_step", _c_i32), ("scale", _c_f32),
+                ("out", _c_p), ("lse", _c_p)]
+
+
+class Layer(ctypes.Structure):
+    _fields_ = [("mode", _c_i32), ("qI", _c_p), ("w", _c_p), ("q", _c_p), ("swa", _c_p),
+                ("out", _c_p), ("lse", _c_p), ("idx", _c_p), ("scores", _c_p)]
+
+
+class GroupArgs(ctypes.Structure):
+    _fields_ = [("B", _c_i32), ("Q", _c_i32), ("K", _c_i32), ("W", _c_i32), ("N", _c_i64),
+                ("n_vis", _c_p), ("kI", _c_p), ("kv_fp4", _c_p), ("kv_new", _c_p), ("n_new", _c_i64),
+                ("new_rows", _c_p), ("swa_rows", _c_i32), ("swa_step", _c_i32),
+                ("hsi_blocks", _c_i32), ("hsi_block", _c_i32), ("pool", _c_p), ("scale", _c_f32),
+                ("n_layers", _c_i32), ("layers", ctypes.POINTER(Layer))]
+
+
+_lib = None
+
+
+def load(path=LIB_PATH):
+    """Load libcsa2.so (built by ``python -m fp4_kv_cache_mxfp4_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"libcsa2.so not found at {path}; build it with "
+                      f"`python -m fp4_kv_cache_mxfp4_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.csa2_quantize_kv_fp4.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_p]
+    lib.csa2_index_score_topk.argtypes = [ctypes.POINTER(IndexArgs), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_group_decode.argtypes = [ctypes.POINTER(GroupArgs), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_workspace_size.argtypes = [_c_p, _c_i32]
+    lib.csa2_workspace_size.restype = ctypes.c_size_t
+    lib.csa2_device_status.argtypes = [ctypes.POINTER(_c_i32), _c_p]
+    lib.csa2_status_string.argtypes = [_c_i32]
+    lib.csa2_status_string.restype = ctypes.c_char_p
+    lib.csa2_version.restype = _c_i32
+    lib.csa2_trace_begin.argtypes = [_c_i32]
+    lib.csa2_trace_get.argtypes = [_c_i32, ctypes.POINTER(_c_i32), ctypes.POINTER(_c_f32)]
+    lib.csa2_trace_count.restype = _c_i32
+    lib.csa2_kernel_name.argtypes = [_c_i32]
+    lib.csa2_kernel_name.restype = ctypes.c_char_p
+    for name in ("csa2_quantize_kv_fp4", "csa2_index_score_topk", "csa2_sparse_attn",
+                 "csa2_group_decode", "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
+                 "csa2_trace_end", "csa2_trace_get"):
+        getattr(lib, name).restype = _c_i32
+    _lib = lib
+    return lib
+
+
+def status_string(status):
+    return load().csa2_status_string(int(status)).decode()
+
+
+def version():
+    return int(load().csa2_version())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status, what):
+    if status != 0:
+        raise Csa2Error(status, what)
+
+
+# ---------------------------------------------------------------------------
+# The four calls of the C ABI
+# ---------------------------------------------------------------------------
+
+def csa2_quantize_kv_fp4(x, kv_fp4, dst_rows=None, row_offset=0, stream=None):
+    """x bf16 [n, >=512] (row stride = x.stride(0)), kv_fp4 uint8 [rows, 288],
+    dst_rows optional int64 [n]."""
+    n = x.shape[0]
+    _check(load().csa2_quantize_kv_fp4(_ptr(x), n, x.stride(0) if n else 512, _ptr(kv_fp4), _ptr(dst_rows),
+                                       row_offset, _stream(stream)), "csa2_quantize_kv_fp4")
+
+
+def index_args(mode, qI, w, kI, n_vis, idx, scores=None, hsi_blocks=0, hsi_block=8, pool_out=None, pool_in=None):
+    """Build csa2_index_args from tensors: qI [B,Q,32,128], w [B,Q,32],
+    kI [B,N,128], n_vis int32 [B,Q], idx int32 [B,Q,K]."""
+    B, Q = qI.shape[0], qI.shape[1]
+    return IndexArgs(mode=mode, B=B, Q=Q, K=idx.shape[-1], N=kI.shape[1],
+                     qI=_ptr(qI), w=_ptr(w), kI=_ptr(kI), n_vis=_ptr(n_vis), idx=_ptr(idx), scores=_ptr(scores),
+                     hsi_blocks=hsi_blocks, hsi_block=hsi_block, pool_out=_ptr(pool_out), pool_in=_ptr(pool_in))
+
+
+def csa2_index_score_topk(args, ws, stream=None):
+    _check(load().csa2_index_score_topk(ctypes.byref(args), _ptr(ws), ws.numel() * ws.element_size(),
+                                        _stream(stream)), "csa2_index_score_topk")
+
+
+def attn_args(q, kv_fp4, idx, swa, out, lse=None, W=128, swa_step=0, scale=0.0):
+    """q [B,Q,64,512], kv_fp4 uint8 [B,N,288], idx int32 [B,Q,K], swa bf16
+    [B,rows,512], out bf16 [B,Q,64,512], lse f32 [B,Q,64]."""
+    B, Q = q.shape[0], q.shape[1]
+    return AttnArgs(B=B, Q=Q, K=idx.shape[-1] if idx is not None else 0, W=W, N=kv_fp4.shape[1],
+                    q=_ptr(q), kv_fp4=_ptr(kv_fp4), idx=_ptr(idx), swa=_ptr(swa),
+                    swa_rows=swa.shape[1] if swa is not None else 0, swa_step=swa_step, scale=scale,
+                    out=_ptr(out), lse=_ptr(lse))
+
+
+def csa2_sparse_attn(args, ws, stream=None):
+    _check(load().csa2_sparse_attn(ctypes.byref(args), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)), "csa2_sparse_attn")
+
+
+def group_args(B, Q, K, W, N, n_vis, kI, kv_fp4, layers, kv_new=None, new_rows=None, swa_rows=128, swa_step=0,
+               hsi_blocks=0, hsi_block=8, pool=None, scale=0.0):
+    """``layers`` is a list of dicts with keys mode, qI, w, q, swa, out, lse,
+    idx, scores (tensors or None).  The returned struct keeps its layer
+    array alive."""
+    arr = (Layer * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i] = Layer(mode=L["mode"], qI=_ptr(L.get("qI")), w=_ptr(L.get("w")), q=_ptr(L["q"]),
+                       swa=_ptr(L["swa"]), out=_ptr(L["out"]), lse=_ptr(L.get("lse")),
+                       idx=_ptr(L.get("idx")), scores=_ptr(L.get("scores")))
+    g = GroupArgs(B=B, Q=Q, K=K, W=W, N=N, n_vis=_ptr(n_vis), kI=_ptr(kI), kv_fp4=_ptr(kv_fp4),
+                  kv_new=_ptr(kv_new), n_new=0 if kv_new is None else kv_new.shape[0], new_rows=_ptr(new_rows),
+                  swa_rows=swa_rows, swa_step=swa_step, hsi_blocks=hsi_blocks, hsi_block=hsi_block,
+                  pool=_ptr(pool), scale=scale, n_layers=len(layers),
+                  layers=ctypes.cast(arr, ctypes.POINTER(Layer)))
+    g._layer_array = arr
+    return g
+
+
+def csa2_group_decode(args, ws, stream=None):
+    _check(load().csa2_group_decode(ctypes.byref(args), _ptr(ws), ws.numel() * ws.element_size(),
+                                    _stream(stream)), "csa2_group_decode")
+
+
+def csa2_workspace_size(args, which):
+    return int(load().csa2_workspace_size(ctypes.byref(args), which))
+
+
+def csa2_device_status(stream=None):
+    code = _c_i32(0)
+    st = load().csa2_device_status(ctypes.byref(code), _stream(stream))
+    return int(st), int(code.value)
+
+
+def workspace(args, which, device="cuda"):
+    """A workspace tensor of the size the call needs (PyTorch owns the
+    memory; its contents do not matter)."""
+    n = csa2_workspace_size(args, which)
+    if n == 0:
+        raise Csa2Error(2, "csa2_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------
+# Launch tracing
+# ---------------------------------------------------------------------------
+
+def csa2_trace_begin(max_launches):
+    _check(load().csa2_trace_begin(max_launches), "csa2_trace_begin")
+
+
+def csa2_trace_stop():
+    _check(load().csa2_trace_stop(), "csa2_trace_stop")
+
+
+def csa2_trace_end():
+    _check(load().csa2_trace_end(), "csa2_trace_end")
+
+
+def csa2_trace_records():
+    """[(kernel name, ms), ...] of the traced launches (waits for them)."""
+    lib = load()
+    out = []
+    for i in range(lib.csa2_trace_count()):
+        k, ms = _c_i32(0), _c_f32(0.0)
+        _check(lib.csa2_trace_get(i, ctypes.byref(k), ctypes.byref(ms)), "csa2_trace_get")
+        out.append((lib.csa2_kernel_name(k.value).decode(), float(ms.value)))
+    return out

@@ -1,0 +1,525 @@
+// csa2_api.cu -- the C ABI of libcsa2 (declared in include/csa2.h): host-side
+// validation, workspace layout, TMA descriptor set-up and kernel launches.
+// The library is built as this single translation unit.
+#include "../../include/csa2.h"
+
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <algorithm>
+#include <mutex>
+#include <string.h>
+
+#include "common.cuh"
+#include "quantize.cuh"
+#include "index_scan.cuh"
+#include "topk.cuh"
+#include "attention.cuh"
+
+namespace csa2 {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxDynSmem = 227 * 1024;
+constexpr int kTopkChunk = 4096;
+constexpr int kCandCap = 32768;
+
+struct DeviceInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+csa2_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    d.ok = (prop.major == 10);
+    d.sms = prop.multiProcessorCount;
+    d.init = true;
+  }
+  if (!d.ok) return CSA2_ERR_ARCH;
+  if (!d.attrs_set) {
+    if (cudaFuncSetAttribute(index_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(topk_smem_bytes(12))) != cudaSuccess ||
+        cudaFuncSetAttribute(sparse_attn_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return CSA2_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.attrs_set = true;
+  }
+  *out = &d;
+  return CSA2_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// bf16 [rows][128] matrix as a 2-D TMA map with 128-byte swizzle
+bool make_map_bf16_128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- index call
+struct IndexPlan {
+  bool pool, hsi;
+  int BQ, qg, hb, cap, bcap;
+  int64_t n_elems, nblk;
+  // counter region (histograms, candidate counters, tickets): zeroed at the
+  // start of every call; data region (scores, candidates): no precondition
+  size_t off_hist, off_bhist, off_ctr, off_bctr, zero_bytes;
+  size_t off_scores, off_bscores, off_cand, off_bcand, data_bytes;
+  size_t total;
+};
+
+csa2_status validate_index(const csa2_index_args* a) {
+  if (!a) return CSA2_ERR_ARG;
+  if (a->mode != CSA2_FULL && a->mode != CSA2_REINDEX && a->mode != CSA2_REINDEX_POOL) return CSA2_ERR_ARG;
+  if (a->B < 1 || a->Q < 1 || a->Q > CSA2_MAX_Q || a->K < 1 || a->K > CSA2_MAX_K || a->N < 1) return CSA2_ERR_SHAPE;
+  if (static_cast<int64_t>(a->B) * a->N >= (static_cast<int64_t>(1) << 31)) return CSA2_ERR_SHAPE;
+  if (!a->qI || !a->w || !a->kI || !a->n_vis || !a->idx) return CSA2_ERR_ARG;
+  const bool hsi = a->mode == CSA2_FULL && a->hsi_blocks > 0;
+  if (a->hsi_blocks < 0 || a->hsi_blocks > CSA2_MAX_K) return CSA2_ERR_SHAPE;
+  if (hsi || a->mode == CSA2_REINDEX_POOL) {
+    if (a->hsi_block != CSA2_HSI_BLOCK) return CSA2_ERR_SHAPE;
+    if (a->hsi_blocks < 1) return CSA2_ERR_SHAPE;
+  }
+  if (hsi && !a->pool_out) return CSA2_ERR_ARG;
+  if (a->mode == CSA2_REINDEX_POOL && !a->pool_in) return CSA2_ERR_ARG;
+  if (!aligned16(a->qI) || !aligned16(a->w) || !aligned16(a->kI) || !aligned16(a->n_vis) || !aligned16(a->idx) ||
+      (a->scores && !aligned16(a->scores)) || (hsi && !aligned16(a->pool_out)) ||
+      (a->mode == CSA2_REINDEX_POOL && !aligned16(a->pool_in)))
+    return CSA2_ERR_ALIGN;
+  return CSA2_OK;
+}
+
+IndexPlan plan_index(const csa2_index_args* a) {
+  IndexPlan P;
+  P.pool = a->mode == CSA2_REINDEX_POOL;
+  P.hsi = a->mode == CSA2_FULL && a->hsi_blocks > 0;
+  P.BQ = a->B * a->Q;
+  P.qg = P.pool ? 1 : a->Q;
+  P.hb = (P.qg <= 2) ? 12 : 10;
+  P.n_elems = P.pool ? static_cast<int64_t>(a->hsi_blocks) * 8 : a->N;
+  P.nblk = P.hsi ? (a->N + 7) / 8 : 0;
+  P.cap = static_cast<int>(std::min<int64_t>(P.n_elems, kCandCap));
+  P.bcap = static_cast<int>(std::min<int64_t>(P.nblk, kCandCap));
+  const size_t nb = static_cast<size_t>(1) << P.hb;
+  size_t off = 0;
+  P.off_hist = off;    off = up256(off + static_cast<size_t>(P.BQ) * nb * 4);
+  P.off_bhist = off;   off = up256(off + (P.hsi ? static_cast<size_t>(P.BQ) * nb * 4 : 0));
+  P.off_ctr = off;     off = up256(off + static_cast<size_t>(P.BQ) * 16);
+  P.off_bctr = off;    off = up256(off + static_cast<size_t>(P.BQ) * 16);
+  P.zero_bytes = off;
+  off = 0;
+  P.off_scores = off;  off = up256(off + static_cast<size_t>(P.BQ) * P.n_elems * 4);
+  P.off_bscores = off; off = up256(off + static_cast<size_t>(P.BQ) * P.nblk * 4);
+  P.off_cand = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.cap * 8);
+  P.off_bcand = off;   off = up256(off + static_cast<size_t>(P.BQ) * P.bcap * 8);
+  P.data_bytes = off;
+  P.total = P.zero_bytes + P.data_bytes;
+  return P;
+}
+
+// zero: the call's counter region (already zeroed); data: its data region
+csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zero, void* data, cudaStream_t st) {
+  const IndexPlan P = plan_index(a);
+  uint8_t* z = static_cast<uint8_t*>(zero);
+  uint8_t* w = static_cast<uint8_t*>(data);
+
+  ScanParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.pool_mode = P.pool;
+  sp.B = a->B; sp.Q = a->Q; sp.qg = P.qg; sp.N = a->N; sp.n_elems = P.n_elems;
+  sp.n_vis = a->n_vis; sp.w = a->w;
+  sp.pool = P.pool ? a->pool_in : nullptr;
+  sp.pool_blocks = P.pool ? a->hsi_blocks : 0;
+  sp.scores = reinterpret_cast<float*>(w + P.off_scores);
+  sp.bscores = P.hsi ? reinterpret_cast<float*>(w + P.off_bscores) : nullptr;
+  sp.nblk = P.nblk;
+  sp.hist = reinterpret_cast<uint32_t*>(z + P.off_hist);
+  sp.bhist = P.hsi ? reinterpret_cast<uint32_t*>(z + P.off_bhist) : nullptr;
+  sp.hb = P.hb;
+  sp.groups = P.pool ? P.BQ : a->B;
+  sp.tiles_per_group = static_cast<int>((P.n_elems + kTileRows - 1) / kTileRows);
+  sp.ctas_per_group = std::max(1, std::min(sp.tiles_per_group, dev.sms / sp.groups));
+  const uint32_t n_mma = 32u * P.qg;
+  sp.acc_bufs = n_mma <= 64 ? 4 : 2;
+  uint32_t cols = 32;
+  while (cols < sp.acc_bufs * n_mma) cols <<= 1;
+  sp.tmem_cols = cols;
+  const ScanSmem L0 = scan_smem_layout(0, P.qg, P.hb, P.hsi);
+  sp.stages = std::min(8, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / kStageBytes));
+  if (sp.stages < 2) return CSA2_ERR_SHAPE;
+  const ScanSmem L = scan_smem_layout(sp.stages, P.qg, P.hb, P.hsi);
+
+  CUtensorMap tk, tq;
+  if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : kTileRows)) return CSA2_ERR_CUDA;
+  if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, 32u * P.qg)) return CSA2_ERR_CUDA;
+
+  const unsigned grid = static_cast<unsigned>(sp.groups * sp.ctas_per_group);
+  trace_pre(kKIndexScan, st);
+  index_scan_kernel<<<grid, kScanThreads, L.total + 1024, st>>>(tk, tq, sp);
+  trace_post(st);
+  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+
+  TopkParams tp;
+  memset(&tp, 0, sizeof(tp));
+  tp.scores = sp.scores;
+  tp.n_elems = P.n_elems;
+  tp.n_vis = P.pool ? nullptr : a->n_vis;
+  tp.vis_div = 1;
+  tp.pool = sp.pool;
+  tp.pool_blocks = sp.pool_blocks;
+  tp.hist = sp.hist;
+  tp.hb = P.hb;
+  tp.cand = reinterpret_cast<uint64_t*>(w + P.off_cand);
+  tp.cap = P.cap;
+  tp.ctr = reinterpret_cast<uint32_t*>(z + P.off_ctr);
+  tp.K = a->K;
+  tp.chunk = kTopkChunk;
+  tp.out_idx = a->idx;
+  tp.out_scores = a->scores;
+  tp.out_by_pos = 0;
+  const size_t tsm = topk_smem_bytes(P.hb);
+  dim3 tgrid(static_cast<unsigned>((P.n_elems + kTopkChunk - 1) / kTopkChunk), static_cast<unsigned>(P.BQ));
+  trace_pre(kKTopk, st);
+  topk_select_kernel<<<tgrid, kTopkThreads, tsm, st>>>(tp);
+  trace_post(st);
+  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+
+  if (P.hsi) {
+    TopkParams bp = tp;
+    bp.scores = sp.bscores;
+    bp.n_elems = P.nblk;
+    bp.n_vis = a->n_vis;
+    bp.vis_div = 8;
+    bp.pool = nullptr;
+    bp.hist = sp.bhist;
+    bp.cand = reinterpret_cast<uint64_t*>(w + P.off_bcand);
+    bp.cap = P.bcap;
+    bp.ctr = reinterpret_cast<uint32_t*>(z + P.off_bctr);
+    bp.K = a->hsi_blocks;
+    bp.out_idx = a->pool_out;
+    bp.out_scores = nullptr;
+    bp.out_by_pos = 1;
+    dim3 bgrid(static_cast<unsigned>((P.nblk + kTopkChunk - 1) / kTopkChunk), static_cast<unsigned>(P.BQ));
+    trace_pre(kKTopk, st);
+    topk_select_kernel<<<bgrid, kTopkThreads, tsm, st>>>(bp);
+    trace_post(st);
+    if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+  }
+  return CSA2_OK;
+}
+
+// ---------------------------------------------------------------- attention call
+csa2_status validate_attn(const csa2_attn_args* a) {
+  if (!a) return CSA2_ERR_ARG;
+  if (a->B < 1 || a->Q < 1 || a->Q > CSA2_MAX_Q || a->K < 0 || a->K > CSA2_MAX_K || a->W < 0 || a->W > CSA2_MAX_W ||
+      a->K + a->W < 1 || a->N < 1 || a->swa_step < 0)
+    return CSA2_ERR_SHAPE;
+  if (!a->q || !a->out || (a->K > 0 && (!a->kv_fp4 || !a->idx)) || (a->W > 0 && !a->swa)) return CSA2_ERR_ARG;
+  if (a->W > 0 && static_cast<int64_t>(a->Q - 1) * a->swa_step + a->W > a->swa_rows) return CSA2_ERR_SHAPE;
+  if (!aligned16(a->q) || !aligned16(a->out) || (a->kv_fp4 && !aligned16(a->kv_fp4)) || (a->idx && !aligned16(a->idx)) ||
+      (a->swa && !aligned16(a->swa)) || (a->lse && !aligned16(a->lse)))
+    return CSA2_ERR_ALIGN;
+  return CSA2_OK;
+}
+
+inline int attn_slices(const csa2_attn_args* a) { return (a->K + a->W + kAttnKeys - 1) / kAttnKeys; }
+
+size_t attn_ws_bytes(const csa2_attn_args* a) {
+  const size_t bq = static_cast<size_t>(a->B) * a->Q, s = attn_slices(a);
+  return up256(bq * s * 64 * 512 * 4) + up256(bq * s * 64 * 2 * 4);
+}
+
+csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
+  AttnParams p;
+  p.B = a->B; p.Q = a->Q; p.K = a->K; p.W = a->W; p.N = a->N;
+  p.q = static_cast<const __nv_bfloat16*>(a->q);
+  p.kv = static_cast<const uint8_t*>(a->kv_fp4);
+  p.idx = a->idx;
+  p.swa = static_cast<const __nv_bfloat16*>(a->swa);
+  p.swa_rows = a->swa_rows; p.swa_step = a->swa_step;
+  const float scale = a->scale > 0.0f ? a->scale : 1.0f / sqrtf(512.0f);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.slices = attn_slices(a);
+  const size_t bq = static_cast<size_t>(a->B) * a->Q;
+  p.opart = static_cast<float*>(ws);
+  p.ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + up256(bq * p.slices * 64 * 512 * 4));
+  p.out = static_cast<__nv_bfloat16*>(a->out);
+  p.lse = a->lse;
+  trace_pre(kKAttnSlice, st);
+  sparse_attn_slice_kernel<<<dim3(p.slices, static_cast<unsigned>(bq)), kAttnThreads, kAttnSmem, st>>>(p);
+  trace_post(st);
+  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+  trace_pre(kKAttnCombine, st);
+  sparse_attn_combine_kernel<<<static_cast<unsigned>(bq * 64), 128, 0, st>>>(p);
+  trace_post(st);
+  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+  return CSA2_OK;
+}
+
+// ---------------------------------------------------------------- group call
+csa2_index_args layer_index_args(const csa2_group_args* g, const csa2_layer& L) {
+  csa2_index_args a;
+  memset(&a, 0, sizeof(a));
+  a.mode = L.mode; a.B = g->B; a.Q = g->Q; a.K = g->K; a.N = g->N;
+  a.qI = L.qI; a.w = L.w; a.kI = g->kI; a.n_vis = g->n_vis;
+  a.idx = L.idx; a.scores = L.scores;
+  a.hsi_blocks = (L.mode == CSA2_FULL || L.mode == CSA2_REINDEX_POOL) ? g->hsi_blocks : 0;
+  a.hsi_block = g->hsi_block;
+  a.pool_out = (L.mode == CSA2_FULL && g->hsi_blocks > 0) ? g->pool : nullptr;
+  a.pool_in = (L.mode == CSA2_REINDEX_POOL) ? g->pool : nullptr;
+  return a;
+}
+
+csa2_attn_args layer_attn_args(const csa2_group_args* g, const csa2_layer& L, const int32_t* idx) {
+  csa2_attn_args a;
+  memset(&a, 0, sizeof(a));
+  a.B = g->B; a.Q = g->Q; a.K = g->K; a.W = g->W; a.N = g->N;
+  a.q = L.q; a.kv_fp4 = g->kv_fp4; a.idx = idx; a.swa = L.swa;
+  a.swa_rows = g->swa_rows; a.swa_step = g->swa_step; a.scale = g->scale;
+  a.out = L.out; a.lse = L.lse;
+  return a;
+}
+
+csa2_status validate_group(const csa2_group_args* g, size_t* index_zero, size_t* index_ws, size_t* attn_ws) {
+  if (!g || !g->layers || g->n_layers < 1 || g->n_layers > 64) return CSA2_ERR_ARG;
+  if (g->n_new < 0) return CSA2_ERR_SHAPE;
+  if (g->n_new > 0 && (!g->kv_new || !g->new_rows || !g->kv_fp4)) return CSA2_ERR_ARG;
+  if (g->n_new > 0 && (!aligned16(g->kv_new) || !aligned16(g->kv_fp4) || !aligned16(g->new_rows))) return CSA2_ERR_ALIGN;
+  size_t iz = 0, idata = 0;
+  bool have_idx = false, have_pool = false;
+  for (int i = 0; i < g->n_layers; ++i) {
+    const csa2_layer& L = g->layers[i];
+    if (L.mode == CSA2_REUSE) {
+      if (!have_idx) return CSA2_ERR_ARG;
+    } else {
+      if (L.mode == CSA2_REINDEX_POOL && !have_pool) return CSA2_ERR_ARG;
+      const csa2_index_args a = layer_index_args(g, L);
+      const csa2_status s = validate_index(&a);
+      if (s != CSA2_OK) return s;
+      const IndexPlan P = plan_index(&a);
+      iz += P.zero_bytes;
+      idata = std::max(idata, P.data_bytes);
+      have_idx = true;
+      if (L.mode == CSA2_FULL && g->hsi_blocks > 0) have_pool = true;
+    }
+    const csa2_attn_args aa = layer_attn_args(g, L, L.idx ? L.idx : g->layers[0].idx);
+    const csa2_status s = validate_attn(&aa);
+    if (s != CSA2_OK) return s;
+  }
+  const csa2_layer& L0 = g->layers[0];
+  const csa2_attn_args a0 = layer_attn_args(g, L0, L0.idx);
+  *index_zero = iz;
+  *index_ws = iz + up256(idata);
+  *attn_ws = attn_ws_bytes(&a0);
+  return CSA2_OK;
+}
+
+}  // namespace
+}  // namespace csa2
+
+using namespace csa2;
+
+extern "C" {
+
+csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x, void* kv_fp4, const int64_t* dst_rows,
+                                 int64_t row_offset, void* stream) {
+  if (n < 0 || ld_x < 512 || (ld_x & 7) || row_offset < 0) return CSA2_ERR_SHAPE;
+  if (n == 0) return CSA2_OK;
+  if (!x || !kv_fp4) return CSA2_ERR_ARG;
+  if (!aligned16(x) || !aligned16(kv_fp4) || (dst_rows && (reinterpret_cast<uintptr_t>(dst_rows) & 7))) return CSA2_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  const csa2_status s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  return launch_quantize(x, n, ld_x, kv_fp4, dst_rows, row_offset, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
+csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws, size_t ws_bytes, void* stream) {
+  csa2_status s = validate_index(a);
+  if (s != CSA2_OK) return s;
+  const IndexPlan P = plan_index(a);
+  if (!ws || ws_bytes < P.total || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, P.zero_bytes, st) != cudaSuccess) return CSA2_ERR_CUDA;
+  return run_index(a, *dev, ws, static_cast<uint8_t*>(ws) + P.zero_bytes, st);
+}
+
+csa2_status csa2_sparse_attn(const csa2_attn_args* a, void* ws, size_t ws_bytes, void* stream) {
+  csa2_status s = validate_attn(a);
+  if (s != CSA2_OK) return s;
+  if (!ws || ws_bytes < attn_ws_bytes(a) || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  return run_attn(a, ws, static_cast<cudaStream_t>(stream));
+}
+
+csa2_status csa2_group_decode(const csa2_group_args* g, void* ws, size_t ws_bytes, void* stream) {
+  size_t iz = 0, iw = 0, aw = 0;
+  csa2_status s = validate_group(g, &iz, &iw, &aw);
+  if (s != CSA2_OK) return s;
+  if (!ws || ws_bytes < iw + aw || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
+  for (int i = 0; i < g->n_layers; ++i)
+    if (g->layers[i].mode != CSA2_REUSE && !g->layers[i].idx) return CSA2_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* zws = static_cast<uint8_t*>(ws);     // one counter region per indexing layer
+  uint8_t* dws = zws + iz;                         // data region shared by the layers in turn
+  uint8_t* aws = zws + iw;
+  if (cudaMemsetAsync(zws, 0, iz, st) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (g->n_new > 0) {
+    if (launch_quantize(g->kv_new, g->n_new, 512, g->kv_fp4, g->new_rows, 0, st) != cudaSuccess) return CSA2_ERR_CUDA;
+  }
+  const int32_t* last_idx = nullptr;
+  for (int i = 0; i < g->n_layers; ++i) {
+    const csa2_layer& L = g->layers[i];
+    if (L.mode != CSA2_REUSE) {
+      const csa2_index_args a = layer_index_args(g, L);
+      s = run_index(&a, *dev, zws, dws, st);
+      if (s != CSA2_OK) return s;
+      zws += plan_index(&a).zero_bytes;
+      last_idx = L.idx;
+    }
+    const csa2_attn_args aa = layer_attn_args(g, L, last_idx);
+    s = run_attn(&aa, aws, st);
+    if (s != CSA2_OK) return s;
+  }
+  return CSA2_OK;
+}
+
+size_t csa2_workspace_size(const void* args, int32_t which) {
+  if (!args) return 0;
+  if (which == CSA2_WS_INDEX) {
+    const csa2_index_args* a = static_cast<const csa2_index_args*>(args);
+    return validate_index(a) == CSA2_OK ? plan_index(a).total : 0;
+  }
+  if (which == CSA2_WS_ATTN) {
+    const csa2_attn_args* a = static_cast<const csa2_attn_args*>(args);
+    return validate_attn(a) == CSA2_OK ? attn_ws_bytes(a) : 0;
+  }
+  if (which == CSA2_WS_GROUP) {
+    size_t iz = 0, iw = 0, aw = 0;
+    return validate_group(static_cast<const csa2_group_args*>(args), &iz, &iw, &aw) == CSA2_OK ? iw + aw : 0;
+  }
+  return 0;
+}
+
+csa2_status csa2_device_status(int32_t* code, void* stream) {
+  int v = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (code) *code = v;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+    return CSA2_ERR_DEVICE;
+  }
+  return CSA2_OK;
+}
+
+const char* csa2_status_string(int32_t s) {
+  switch (s) {
+    case CSA2_OK: return "ok";
+    case CSA2_ERR_ARG: return "invalid argument";
+    case CSA2_ERR_SHAPE: return "unsupported shape";
+    case CSA2_ERR_ALIGN: return "misaligned pointer or stride";
+    case CSA2_ERR_WORKSPACE: return "workspace missing or too small";
+    case CSA2_ERR_CUDA: return "CUDA error";
+    case CSA2_ERR_DEVICE: return "device-side failure recorded";
+    case CSA2_ERR_ARCH: return "device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+int32_t csa2_version(void) { return 100; }
+
+csa2_status csa2_trace_begin(int32_t max_launches) {
+  if (max_launches < 1 || max_launches > (1 << 20)) return CSA2_ERR_SHAPE;
+  csa2_trace_end();
+  g_trace.ev = new cudaEvent_t[2 * static_cast<size_t>(max_launches)];
+  g_trace.kid = new int[max_launches];
+  for (int i = 0; i < 2 * max_launches; ++i) {
+    if (cudaEventCreate(&g_trace.ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(g_trace.ev[j]);
+      delete[] g_trace.ev; delete[] g_trace.kid;
+      g_trace.ev = nullptr; g_trace.kid = nullptr;
+      return CSA2_ERR_CUDA;
+    }
+  }
+  g_trace.max = max_launches;
+  g_trace.n = 0;
+  g_trace.on = true;
+  return CSA2_OK;
+}
+
+csa2_status csa2_trace_stop(void) {
+  g_trace.on = false;
+  return CSA2_OK;
+}
+
+csa2_status csa2_trace_end(void) {
+  g_trace.on = false;
+  if (g_trace.ev) {
+    for (int i = 0; i < 2 * g_trace.max; ++i) cudaEventDestroy(g_trace.ev[i]);
+    delete[] g_trace.ev;
+    delete[] g_trace.kid;
+  }
+  g_trace = LaunchTrace();
+  return CSA2_OK;
+}
+
+int32_t csa2_trace_count(void) { return g_trace.n; }
+
+csa2_status csa2_trace_get(int32_t i, int32_t* kernel, float* ms) {
+  if (i < 0 || i >= g_trace.n || !kernel || !ms) return CSA2_ERR_ARG;
+  if (cudaEventSynchronize(g_trace.ev[2 * i + 1]) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (cudaEventElapsedTime(ms, g_trace.ev[2 * i], g_trace.ev[2 * i + 1]) != cudaSuccess) return CSA2_ERR_CUDA;
+  *kernel = g_trace.kid[i];
+  return CSA2_OK;
+}
+
+const char* csa2_kernel_name(int32_t kernel) {
+  switch (kernel) {
+    case kKQuantize: return "quantize_kv_fp4_kernel";
+    case kKIndexScan: return "index_scan_kernel";
+    case kKTopk: return "topk_select_kernel";
+    case kKAttnSlice: return "sparse_attn_slice_kernel";
+    case kKAttnCombine: return "sparse_attn_combine_kernel";
+    default: return "unknown";
+  }
+}
+
+}  // extern "C"

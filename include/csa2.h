@@ -1,0 +1,276 @@
+/*
+ * csa2.h -- C ABI of libcsa2: CSA2 sparse attention over an FP4 main-KV
+ * cache, hand-written for NVIDIA B200 (sm_100a).
+ *
+ * The four calls follow the method's statement on the pages:
+ *
+ *   "DeepSeek V4.1-Flash 技术报告深度解析：CED 架构与 KV Cache 极限压缩"
+ *   (eogee.com/article/126)
+ *     §3.2  CSA2 Full / Reindex / Reuse modes, 32 x 128 indexer, top-512,
+ *           64 heads x 512 attention, SWA window 128
+ *     §3.3  Hierarchical Sparse Indexer: 2048 blocks of 8 positions
+ *     §3.4  FP4 main KV: E2M1 values, one E4M3 scale per 16 channels,
+ *           quantised after RoPE, dequantised before attention
+ *   "DeepSeek-V4.1-Flash" README walk-through (m.nxbn.cn/news/186820)
+ *     §3.1 / §3.3 configuration tables (head sizes, candidate pool sizes)
+ *
+ * Conventions for every call
+ *   - All data pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or keeps them.  Structs are read on the host
+ *     during the call only.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Every call is asynchronous on that stream: it validates its
+ *     arguments on the host, enqueues kernels and returns.
+ *   - Multi-dimensional arrays are dense and row-major in the order written,
+ *     e.g. [B][Q][32][128] means element (b,q,h,d) sits at
+ *     ((b*Q + q)*32 + h)*128 + d.
+ *   - bf16 means IEEE bfloat16, f32 IEEE binary32; inputs must be finite.
+ *   - Every pointer must be 16-byte aligned (CSA2_ERR_ALIGN otherwise).
+ *   - Host-side validation failure returns before anything is enqueued and
+ *     leaves every output untouched.  CSA2_ERR_CUDA reports a launch error;
+ *     kernels enqueued before it by the same call may have run.
+ *   - Workspace: calls that need scratch take (ws, ws_bytes); the size comes
+ *     from csa2_workspace_size().  Its contents on entry do not matter (the
+ *     call clears the part it needs with an asynchronous memset on
+ *     `stream`).  Calls that share a workspace must not overlap in time.
+ *   - Batch rows are independent sequences with their own caches.
+ */
+#ifndef CSA2_ABI_H_
+#define CSA2_ABI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Sizes fixed by the method ([eogee] §3.2, [nxbn] §3.1/§3.3). */
+#define CSA2_D            512   /* main-KV entry width = attention head dim   */
+#define CSA2_ENTRY_BYTES  288   /* packed FP4 entry: 256 B nibbles + 32 B E4M3 scales */
+#define CSA2_SCALE_BLOCK  16    /* channels per E4M3 scale                    */
+#define CSA2_H            64    /* attention query heads (one KV head)        */
+#define CSA2_HI           32    /* indexer heads                              */
+#define CSA2_DI           128   /* indexer head dim                           */
+#define CSA2_TOPK         512   /* the method's top-K                         */
+#define CSA2_WIN          128   /* the method's SWA window                    */
+#define CSA2_HSI_BLOCK    8     /* positions per HSI block                    */
+#define CSA2_HSI_BLOCKS   2048  /* HSI blocks kept                            */
+
+/* Limits of this implementation. */
+#define CSA2_MAX_Q        8     /* query positions per batch row per call     */
+#define CSA2_MAX_K        2048  /* largest top-K (and largest pool, in blocks) */
+#define CSA2_MAX_W        1024  /* largest window (rows per query)            */
+
+typedef enum csa2_status {
+    CSA2_OK            = 0,
+    CSA2_ERR_ARG       = 1,  /* NULL where a pointer is required, bad mode   */
+    CSA2_ERR_SHAPE     = 2,  /* a size outside the supported range           */
+    CSA2_ERR_ALIGN     = 3,  /* a pointer or stride breaks 16-byte alignment */
+    CSA2_ERR_WORKSPACE = 4,  /* workspace NULL or smaller than required      */
+    CSA2_ERR_CUDA      = 5,  /* a CUDA runtime or launch error               */
+    CSA2_ERR_DEVICE    = 6,  /* a kernel recorded a device-side failure      */
+    CSA2_ERR_ARCH      = 7   /* current device is not sm_100                 */
+} csa2_status;
+
+/* Static layer modes, [eogee] §3.2 and §3.3. */
+typedef enum csa2_mode {
+    CSA2_FULL         = 0,  /* score every visible entry                       */
+    CSA2_REINDEX      = 1,  /* re-score the shared index-K with own index-Q    */
+    CSA2_REINDEX_POOL = 2,  /* re-score only the HSI candidate pool            */
+    CSA2_REUSE        = 3   /* no scoring: reuse the previous layer's top-K    */
+} csa2_mode;
+
+/* ------------------------------------------------------------------------
+ * csa2_quantize_kv_fp4 -- [eogee] §3.4 FP4 main-KV cache.
+ *
+ * Quantises n main-KV entries (512 channels, already RoPE-rotated) to the
+ * 288-byte FP4 layout: for each block of 16 channels
+ *     sf = fp32(amax / 6);  s = E4M3(sf)  (round to nearest even, saturate 448)
+ *     q_i = E2M1(fp32(x_i / s))           (round to nearest even, saturate 6;
+ *                                          sign kept; s == 0 gives signed 0)
+ * Entry layout: byte i (0..255) holds channel 2i in its low nibble and
+ * channel 2i+1 in its high nibble; byte 256+k holds the scale of channels
+ * 16k..16k+15.  Dequantised value = E2M1(q) * E4M3(s), exact in bf16.
+ *
+ *   x         bf16 [n][ld_x], entry i in x[i*ld_x .. i*ld_x+511]; ld_x >= 512
+ *             and a multiple of 8
+ *   n         entries, >= 0 (0 enqueues nothing)
+ *   kv_fp4    u8 cache rows of CSA2_ENTRY_BYTES bytes
+ *   dst_rows  optional int64 [n]: entry i goes to row dst_rows[i];
+ *             NULL means row row_offset + i
+ *   row_offset  first destination row when dst_rows is NULL, >= 0
+ * Entries map to distinct rows (overlapping destinations race).
+ * Errors: ARG (x or kv_fp4 NULL with n > 0), SHAPE (n < 0, ld_x < 512,
+ * row_offset < 0), ALIGN, CUDA.
+ * ---------------------------------------------------------------------- */
+csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x,
+                                 void* kv_fp4, const int64_t* dst_rows,
+                                 int64_t row_offset, void* stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_index_score_topk -- [eogee] §3.2 lightweight indexer + top-K,
+ * §3.3 Hierarchical Sparse Indexer.
+ *
+ * Score of query (b,q) for entry t (t < n_vis[b][q]):
+ *     s = sum_h w[b][q][h] * ReLU( sum_d qI[b][q][h][d] * kI[b][t][d] )
+ * bf16 products accumulated in fp32 on the tensor cores.  The K best
+ * entries by (higher score, then lower position) are written best first,
+ * padded with -1 when fewer than K entries are visible.
+ *
+ * mode CSA2_FULL / CSA2_REINDEX: scan t in [0, n_vis).  With hsi_blocks > 0
+ *   (FULL only) the call also builds the HSI pool: block score = max of the
+ *   visible scores in positions [8j, 8j+8), the hsi_blocks best blocks (ties
+ *   to the lower block id) are written to pool_out in ascending block order,
+ *   padded with -1.
+ * mode CSA2_REINDEX_POOL: scan only the positions of pool_in (hsi_blocks
+ *   block ids per query, ascending, -1 padding ignored); positions at or
+ *   beyond n_vis do not score.
+ * ---------------------------------------------------------------------- */
+typedef struct csa2_index_args {
+    int32_t        mode;        /* CSA2_FULL, CSA2_REINDEX or CSA2_REINDEX_POOL  */
+    int32_t        B;           /* batch rows, >= 1                              */
+    int32_t        Q;           /* query positions per row, 1..CSA2_MAX_Q        */
+    int32_t        K;           /* top-K, 1..CSA2_MAX_K                          */
+    int64_t        N;           /* index-K rows per batch row, >= 1              */
+    const void*    qI;          /* bf16 [B][Q][32][128]                          */
+    const float*   w;           /* f32  [B][Q][32]                               */
+    const void*    kI;          /* bf16 [B][N][128]                              */
+    const int32_t* n_vis;       /* int32 [B][Q], each in [0, N]                  */
+    int32_t*       idx;         /* out int32 [B][Q][K]                           */
+    float*         scores;      /* optional out f32 [B][Q][K] (-inf padding)     */
+    int32_t        hsi_blocks;  /* 0, or blocks in the pool (1..CSA2_MAX_K)      */
+    int32_t        hsi_block;   /* positions per block (CSA2_HSI_BLOCK)          */
+    int32_t*       pool_out;    /* FULL with hsi_blocks > 0: out int32 [B][Q][hsi_blocks] */
+    const int32_t* pool_in;     /* REINDEX_POOL: in int32 [B][Q][hsi_blocks]     */
+} csa2_index_args;
+
+csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_sparse_attn -- [eogee] §3.2 sparse MQA: each query attends to its
+ * selected FP4 entries plus the layer's SWA window; §3.4 dequantise before
+ * the attention math.
+ *
+ * For query (b,q): keys = { dequant(kv_fp4[b][idx[b][q][j]]) : idx >= 0 }
+ * followed by the window rows swa[b][q*swa_step + r], r in [0, W).  Each key
+ * is also its value (one 512-dim vector per entry).  With logits
+ * z_hj = scale * q[b][q][h] . key_j (scale <= 0 selects 1/sqrt(512)):
+ *     out[b][q][h] = sum_j softmax_j(z_h)_j * key_j      (bf16, fp32 math)
+ *     lse[b][q][h] = ln sum_j exp(z_hj)                  (optional)
+ * A query with no key at all gets out = 0 and lse = -inf.
+ *
+ * idx entries must be -1 or in [0, N); the window rows read must lie inside
+ * [0, swa_rows).
+ * ---------------------------------------------------------------------- */
+typedef struct csa2_attn_args {
+    int32_t        B, Q;        /* batch rows >= 1; queries per row 1..CSA2_MAX_Q */
+    int32_t        K;           /* idx slots per query, 0..CSA2_MAX_K            */
+    int32_t        W;           /* window rows per query, 0..CSA2_MAX_W          */
+    int64_t        N;           /* cache rows per batch row                      */
+    const void*    q;           /* bf16 [B][Q][64][512]                          */
+    const void*    kv_fp4;      /* u8   [B][N][288]                              */
+    const int32_t* idx;         /* int32 [B][Q][K]                               */
+    const void*    swa;         /* bf16 [B][swa_rows][512]                       */
+    int32_t        swa_rows;    /* rows per batch row in swa, >= (Q-1)*swa_step+W */
+    int32_t        swa_step;    /* window of query q starts at row q*swa_step    */
+    float          scale;       /* logit scale; <= 0 means 1/sqrt(512)           */
+    void*          out;         /* out bf16 [B][Q][64][512]                      */
+    float*         lse;         /* optional out f32 [B][Q][64]                   */
+} csa2_attn_args;
+
+csa2_status csa2_sparse_attn(const csa2_attn_args* a, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_group_decode -- one CSA2 sharing group ([eogee] §3.2, §3.3): the
+ * layers share one FP4 main KV and one index-K and run strictly in order.
+ *   1. if n_new > 0: quantise kv_new into kv_fp4 (csa2_quantize_kv_fp4 with
+ *      dst_rows = new_rows, absolute rows of the [B*N] cache);
+ *   2. for each layer: FULL / REINDEX / REINDEX_POOL score and select
+ *      (csa2_index_score_topk; FULL builds the pool when hsi_blocks > 0 and
+ *      REINDEX_POOL uses the pool of the most recent FULL layer), REUSE
+ *      takes the top-K of the most recent indexing layer; then sparse
+ *      attention with the layer's own q and window (csa2_sparse_attn).
+ * ---------------------------------------------------------------------- */
+typedef struct csa2_layer {
+    int32_t        mode;        /* csa2_mode                                     */
+    const void*    qI;          /* indexing modes: bf16 [B][Q][32][128]          */
+    const float*   w;           /* indexing modes: f32 [B][Q][32]                */
+    const void*    q;           /* bf16 [B][Q][64][512]                          */
+    const void*    swa;         /* bf16 [B][swa_rows][512]                       */
+    void*          out;         /* out bf16 [B][Q][64][512]                      */
+    float*         lse;         /* optional out f32 [B][Q][64]                   */
+    int32_t*       idx;         /* indexing modes: out int32 [B][Q][K]           */
+    float*         scores;      /* optional out f32 [B][Q][K]                    */
+} csa2_layer;
+
+typedef struct csa2_group_args {
+    int32_t          B, Q, K, W;
+    int64_t          N;
+    const int32_t*   n_vis;     /* int32 [B][Q]                                  */
+    const void*      kI;        /* bf16 [B][N][128]                              */
+    void*            kv_fp4;    /* u8 [B][N][288]                                */
+    const void*      kv_new;    /* bf16 [n_new][512], or NULL                    */
+    int64_t          n_new;     /* entries to quantise first (may be 0)          */
+    const int64_t*   new_rows;  /* int64 [n_new] absolute rows in [0, B*N)       */
+    int32_t          swa_rows, swa_step;
+    int32_t          hsi_blocks, hsi_block;
+    int32_t*         pool;      /* hsi_blocks > 0: int32 [B][Q][hsi_blocks]      */
+    float            scale;
+    int32_t          n_layers;  /* 1..64                                         */
+    const csa2_layer* layers;   /* HOST array of n_layers descriptors            */
+} csa2_group_args;
+
+csa2_status csa2_group_decode(const csa2_group_args* g, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* Workspace bytes needed by a call.  which = 1: csa2_index_args,
+ * 2: csa2_attn_args, 3: csa2_group_args.  Returns 0 when the arguments are
+ * invalid for that call. */
+#define CSA2_WS_INDEX 1
+#define CSA2_WS_ATTN  2
+#define CSA2_WS_GROUP 3
+size_t csa2_workspace_size(const void* args, int32_t which);
+
+/* Reads and clears the device-side failure word of the current device
+ * (bounded waits that gave up, internal limits exceeded).  Synchronises
+ * `stream`.  Returns CSA2_OK when clear, CSA2_ERR_DEVICE otherwise and
+ * stores the recorded code in *code (may be NULL). */
+csa2_status csa2_device_status(int32_t* code, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* csa2_status_string(int32_t status);
+
+/* Library ABI version: 100 * major + minor. */
+int32_t csa2_version(void);
+
+/* ------------------------------------------------------------------------
+ * Launch tracing, for profiling harnesses (off by default).
+ * csa2_trace_begin(n) creates 2n CUDA events (outside any timed region) and
+ * from then on brackets every kernel the library enqueues with two of them,
+ * recorded on that kernel's stream, until n launches are recorded or
+ * csa2_trace_stop() is called.  csa2_trace_count() tells how many were
+ * recorded; csa2_trace_get(i, &kernel, &ms) waits for launch i and returns
+ * its kernel id and event-measured duration in milliseconds.
+ * csa2_trace_end() destroys the events.  Kernel ids name the library's
+ * kernels (csa2_kernel_name).  Tracing state is process-global and not
+ * synchronised: enable it only while one thread drives the library.
+ * ---------------------------------------------------------------------- */
+#define CSA2_KERNEL_QUANTIZE     0
+#define CSA2_KERNEL_INDEX_SCAN   1
+#define CSA2_KERNEL_TOPK         2
+#define CSA2_KERNEL_ATTN_SLICE   3
+#define CSA2_KERNEL_ATTN_COMBINE 4
+csa2_status csa2_trace_begin(int32_t max_launches);
+csa2_status csa2_trace_stop(void);
+csa2_status csa2_trace_end(void);
+int32_t csa2_trace_count(void);
+csa2_status csa2_trace_get(int32_t i, int32_t* kernel, float* ms);
+const char* csa2_kernel_name(int32_t kernel);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_ABI_H_ */

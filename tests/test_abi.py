@@ -1,0 +1,173 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/csa2.h declares, the binding's struct layouts equal the C
+compiler's, and host-side validation rejects bad arguments before any
+device work.  Only argument combinations that fail validation (or touch no
+device) are used here, so nothing can reach a kernel."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from fp4_kv_cache_mxfp4_b200 import build, csa2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa2.h")
+FAKE = 0x10000          # 16-byte aligned stand-in pointer, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return csa2.load()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(csa2_\w+)\s*\(", text, re.M)))
+
+
+def test_every_declared_function_is_exported(L):
+    names = _declared_functions()
+    assert {"csa2_quantize_kv_fp4", "csa2_index_score_topk", "csa2_sparse_attn", "csa2_group_decode",
+            "csa2_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", csa2.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (csa2_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_version_and_status_strings(L):
+    assert csa2.version() == 100
+    assert csa2.status_string(0) == "ok"
+    assert "workspace" in csa2.status_string(4)
+    assert csa2.status_string(99) == "unknown status"
+
+
+def _c_layout():
+    fields = {
+        "csa2_index_args": [f for f, _ in csa2.IndexArgs._fields_],
+        "csa2_attn_args": [f for f, _ in csa2.AttnArgs._fields_],
+        "csa2_layer": [f for f, _ in csa2.Layer._fields_],
+        "csa2_group_args": [f for f, _ in csa2.GroupArgs._fields_],
+    }
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "csa2.h"', "int main(void) {"]
+    for s, fs in fields.items():
+        lines.append(f'printf("{s} %zu\\n", sizeof({s}));')
+        for f in fs:
+            lines.append(f'printf("{s}.{f} %zu\\n", offsetof({s}, {f}));')
+    lines.append("return 0; }")
+    with tempfile.TemporaryDirectory() as d:
+        src, exe = os.path.join(d, "l.c"), os.path.join(d, "l")
+        open(src, "w").write("\n".join(lines))
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), "-o", exe, src], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    return dict(line.split() for line in out.strip().splitlines())
+
+
+def test_struct_layouts_match_the_header():
+    c = _c_layout()
+    for cname, py in [("csa2_index_args", csa2.IndexArgs), ("csa2_attn_args", csa2.AttnArgs),
+                      ("csa2_layer", csa2.Layer), ("csa2_group_args", csa2.GroupArgs)]:
+        assert int(c[cname]) == ctypes.sizeof(py), cname
+        for f, _ in py._fields_:
+            assert int(c[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
+
+
+def _index(**kw):
+    a = csa2.IndexArgs(mode=0, B=1, Q=1, K=512, N=4096, qI=FAKE, w=FAKE, kI=FAKE, n_vis=FAKE, idx=FAKE,
+                       scores=None, hsi_blocks=0, hsi_block=8, pool_out=None, pool_in=None)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _attn(**kw):
+    a = csa2.AttnArgs(B=1, Q=1, K=512, W=128, N=4096, q=FAKE, kv_fp4=FAKE, idx=FAKE, swa=FAKE,
+                      swa_rows=128, swa_step=0, scale=0.0, out=FAKE, lse=None)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def _call_index(L, a, ws=FAKE, ws_bytes=0):
+    return L.csa2_index_score_topk(ctypes.byref(a), ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def _call_attn(L, a, ws=FAKE, ws_bytes=0):
+    return L.csa2_sparse_attn(ctypes.byref(a), ctypes.c_void_p(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(mode=3), 1), (dict(mode=7), 1), (dict(qI=None), 1), (dict(n_vis=None), 1), (dict(idx=None), 1),
+    (dict(B=0), 2), (dict(Q=0), 2), (dict(Q=9), 2), (dict(K=0), 2), (dict(K=2049), 2), (dict(N=0), 2),
+    (dict(N=2 ** 31), 2), (dict(hsi_blocks=-1), 2), (dict(hsi_blocks=2048, hsi_block=16, pool_out=FAKE), 2),
+    (dict(hsi_blocks=2048, pool_out=None), 1), (dict(mode=2, hsi_blocks=2048, pool_in=None), 1),
+    (dict(qI=FAKE + 8), 3), (dict(kI=FAKE + 4), 3), (dict(scores=FAKE + 2), 3),
+    (dict(), 4),                       # valid arguments, zero-byte workspace
+])
+def test_index_validation(L, kw, status):
+    assert _call_index(L, _index(**kw)) == status
+
+
+def test_index_validation_null_struct(L):
+    assert L.csa2_index_score_topk(None, None, 0, None) == 1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(out=None), 1), (dict(idx=None), 1), (dict(swa=None), 1),
+    (dict(B=0), 2), (dict(Q=9), 2), (dict(K=-1), 2), (dict(K=0, W=0), 2), (dict(W=1025), 2),
+    (dict(swa_rows=100), 2), (dict(Q=2, swa_step=1, swa_rows=128), 2),
+    (dict(out=FAKE + 8), 3), (dict(lse=FAKE + 4), 3),
+    (dict(), 4),
+])
+def test_attn_validation(L, kw, status):
+    assert _call_attn(L, _attn(**kw)) == status
+
+
+def test_quantize_validation(L):
+    q = L.csa2_quantize_kv_fp4
+    assert q(ctypes.c_void_p(FAKE), -1, 512, ctypes.c_void_p(FAKE), None, 0, None) == 2
+    assert q(ctypes.c_void_p(FAKE), 4, 500, ctypes.c_void_p(FAKE), None, 0, None) == 2
+    assert q(ctypes.c_void_p(FAKE), 4, 516, ctypes.c_void_p(FAKE), None, 0, None) == 2
+    assert q(ctypes.c_void_p(FAKE), 4, 512, ctypes.c_void_p(FAKE), None, -3, None) == 2
+    assert q(None, 4, 512, ctypes.c_void_p(FAKE), None, 0, None) == 1
+    assert q(ctypes.c_void_p(FAKE + 2), 4, 512, ctypes.c_void_p(FAKE), None, 0, None) == 3
+    assert q(ctypes.c_void_p(FAKE), 0, 512, None, None, 0, None) == 0      # nothing to do
+
+
+def test_workspace_sizes(L):
+    a = _index(B=4, Q=1, K=512, N=131072)
+    n = L.csa2_workspace_size(ctypes.byref(a), csa2.WS_INDEX)
+    # scores (4 B per entry per query) + one 4096-bin histogram + candidate buffers
+    assert n >= 4 * 131072 * 4 + 4 * 4096 * 4 + 4 * 32768 * 8
+    assert n < 8 * 2 ** 20
+    assert L.csa2_workspace_size(ctypes.byref(_index(Q=0)), csa2.WS_INDEX) == 0
+    at = _attn(B=4, Q=1, K=512, W=128)
+    m = L.csa2_workspace_size(ctypes.byref(at), csa2.WS_ATTN)
+    assert m >= 4 * 10 * 64 * 512 * 4                   # 10 slices of 64 keys, fp32 partials
+    assert L.csa2_workspace_size(ctypes.byref(at), 9) == 0
+    # a workspace one byte short is refused
+    assert _call_index(L, a, FAKE, n - 1) == 4
+    assert _call_attn(L, at, FAKE, m - 1) == 4
+
+
+def test_group_validation(L):
+    layers = (csa2.Layer * 2)()
+    layers[0] = csa2.Layer(mode=3, q=FAKE, swa=FAKE, out=FAKE)          # REUSE first: nothing to reuse
+    layers[1] = csa2.Layer(mode=0, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)
+    g = csa2.GroupArgs(B=1, Q=1, K=512, W=128, N=4096, n_vis=FAKE, kI=FAKE, kv_fp4=FAKE, kv_new=None, n_new=0,
+                       new_rows=None, swa_rows=128, swa_step=0, hsi_blocks=0, hsi_block=8, pool=None, scale=0.0,
+                       n_layers=2, layers=ctypes.cast(layers, ctypes.POINTER(csa2.Layer)))
+    assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), 0, None) == 1
+    layers[0] = csa2.Layer(mode=0, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)
+    layers[1] = csa2.Layer(mode=2, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)   # pool without HSI
+    assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), 0, None) == 1
+    layers[1] = csa2.Layer(mode=3, q=FAKE, swa=FAKE, out=FAKE)
+    n = L.csa2_workspace_size(ctypes.byref(g), csa2.WS_GROUP)
+    assert n > 0
+    assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), n - 1, None) == 4

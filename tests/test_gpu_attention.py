@@ -1,0 +1,85 @@
+"""GPU parity of csa2_sparse_attn against the float64 oracle on the same
+index sets (1e-2 absolute + 1e-2 relative)."""
+
+import numpy as np
+import pytest
+import torch
+
+from fp4_kv_cache_mxfp4_b200 import csa2
+from oracle import attention, fp4
+from parity import check_attention, f32
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(B, Q, N, K, W, swa_step, seed, q_std=512 ** -0.5, minus_one=0.0):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(B, N, 512, generator=g).to(torch.bfloat16)
+    kv = np.stack([fp4.quantize_kv_fp4(f32(x[b])) for b in range(B)])       # oracle-made cache bytes
+    q = (torch.randn(B, Q, 64, 512, generator=g) * q_std).to(torch.bfloat16)
+    rows = W + (Q - 1) * swa_step if W else 1
+    swa = torch.randn(B, rows, 512, generator=g).to(torch.bfloat16)
+    rng = np.random.default_rng(seed)
+    idx = np.stack([[rng.choice(N, K, replace=False) if K else np.zeros(0, int) for _ in range(Q)]
+                    for _ in range(B)]).astype(np.int32).reshape(B, Q, K)
+    if minus_one:
+        idx[rng.random(idx.shape) < minus_one] = -1
+    return kv, q, swa, idx
+
+
+def _run(kv, q, swa, idx, W, swa_step, scale=0.0, want_lse=True):
+    B, Q = q.shape[:2]
+    d = "cuda"
+    kv_d = torch.from_numpy(kv).to(d)
+    q_d, swa_d = q.to(d), swa.to(d)
+    idx_d = torch.from_numpy(idx).to(d)
+    out = torch.full((B, Q, 64, 512), float("nan"), dtype=torch.bfloat16, device=d)
+    lse = torch.full((B, Q, 64), float("nan"), device=d) if want_lse else None
+    a = csa2.attn_args(q_d, kv_d, idx_d, swa_d, out, lse, W=W, swa_step=swa_step, scale=scale)
+    ws = csa2.workspace(a, csa2.WS_ATTN)
+    csa2.csa2_sparse_attn(a, ws)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), (lse.cpu().numpy() if want_lse else None)
+
+
+def _oracle(kv, q, swa, idx, W, swa_step, scale=None):
+    B, Q = q.shape[:2]
+    o = np.zeros((B, Q, 64, 512))
+    lse = np.zeros((B, Q, 64))
+    for b in range(B):
+        deq = fp4.dequantize_kv_fp4(kv[b])
+        for i in range(Q):
+            rows = f32(swa[b])[i * swa_step: i * swa_step + W]
+            o[b, i], lse[b, i] = attention.sparse_mqa(f32(q[b, i]), deq, idx[b, i], rows, scale)
+    return o, lse
+
+
+@pytest.mark.parametrize("B,Q,N,K,W,step,seed,m1", [
+    (1, 4, 2048, 512, 128, 0, 0, 0.0),
+    (2, 3, 700, 512, 128, 0, 1, 0.1),      # some empty slots
+    (1, 2, 300, 100, 37, 1, 2, 0.0),       # ragged slices, causal windows
+    (3, 1, 64, 64, 0, 0, 3, 0.0),          # selected entries only
+    (1, 1, 10, 0, 128, 0, 4, 0.0),         # window only
+])
+def test_attention_parity(B, Q, N, K, W, step, seed, m1):
+    kv, q, swa, idx = _case(B, Q, N, K, W, step, seed, minus_one=m1)
+    out, lse = _run(kv, q, swa, idx, W, step)
+    o_ref, lse_ref = _oracle(kv, q, swa, idx, W, step)
+    check_attention(out, o_ref, what="out")
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-3, atol=1e-3)
+
+
+def test_peaked_softmax_and_explicit_scale():
+    kv, q, swa, idx = _case(2, 1, 1000, 512, 128, 0, 5, q_std=1.0)
+    out, lse = _run(kv, q, swa, idx, 128, 0, scale=0.125)
+    o_ref, lse_ref = _oracle(kv, q, swa, idx, 128, 0, scale=0.125)
+    check_attention(out, o_ref, what="peaked")
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-3, atol=1e-2)
+
+
+def test_no_keys_at_all():
+    kv, q, swa, idx = _case(1, 2, 100, 64, 0, 0, 6)
+    idx[:] = -1
+    out, lse = _run(kv, q, swa, idx, 0, 0)
+    assert np.all(out == 0)
+    assert np.all(np.isneginf(lse))
