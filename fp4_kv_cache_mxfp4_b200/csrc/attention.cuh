@@ -24,6 +24,8 @@
 namespace csa2 {
 
 constexpr int kAttnThreads = 128;
+constexpr int kAttnMaxK = 2048;      // largest K (CSA2_MAX_K)
+constexpr int kAttnMaxW = 1024;      // largest window (CSA2_MAX_W)
 constexpr int kAttnKeys = 64;        // key slots per slice
 constexpr int kAttnSmem = 64 * 1024 * 2 + 1024 + 256 + 1024;   // q, keys, nibble table, flags, align
 
@@ -248,25 +250,38 @@ sparse_attn_slice_kernel(AttnParams p) {
   }
 }
 
-// Merge the slices of one (query, head): 128 threads x 4 dims.
+// Merge the slices of one (query, head): 128 threads x 4 dims.  The slice
+// statistics are loaded once into shared memory; the partial outputs are
+// fetched eight slices at a time so their L2 latencies overlap.
+constexpr int kAttnMaxSlices = (kAttnMaxK + kAttnMaxW + kAttnKeys - 1) / kAttnKeys;
+
 __global__ void __launch_bounds__(128)
 sparse_attn_combine_kernel(AttnParams p) {
+  __shared__ float m_s[kAttnMaxSlices], l_s[kAttnMaxSlices];
   const int bq = blockIdx.x >> 6, h = blockIdx.x & 63;
   const int t = threadIdx.x;
   const float* ml = p.ml + static_cast<int64_t>(bq) * p.slices * 128;
+  if (t < p.slices) { m_s[t] = ml[t * 128 + h * 2]; l_s[t] = ml[t * 128 + h * 2 + 1]; }
+  __syncthreads();
   float M = -INFINITY;
-  for (int s = 0; s < p.slices; ++s) M = fmaxf(M, ml[s * 128 + h * 2]);
+  for (int s = 0; s < p.slices; ++s) M = fmaxf(M, m_s[s]);
   float L = 0.0f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (M != -INFINITY) {
-    for (int s = 0; s < p.slices; ++s) {
-      const float ms = ml[s * 128 + h * 2];
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L += f * ml[s * 128 + h * 2 + 1];
-      const float4 o = __ldcg(reinterpret_cast<const float4*>(
-          p.opart + ((static_cast<int64_t>(bq) * p.slices + s) * 64 + h) * 512) + t);
-      acc.x += f * o.x; acc.y += f * o.y; acc.z += f * o.z; acc.w += f * o.w;
+    const float4* op = reinterpret_cast<const float4*>(p.opart + (static_cast<int64_t>(bq) * p.slices * 64 + h) * 512) + t;
+    const int64_t stride = 64 * 512 / 4;             // float4s between consecutive slices
+    for (int s0 = 0; s0 < p.slices; s0 += 8) {
+      float4 o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (s0 + j < p.slices) o[j] = __ldcg(op + (s0 + j) * stride);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (s0 + j >= p.slices || m_s[s0 + j] == -INFINITY) continue;
+        const float f = exp2f(m_s[s0 + j] - M);
+        L += f * l_s[s0 + j];
+        acc.x += f * o[j].x; acc.y += f * o[j].y; acc.z += f * o[j].z; acc.w += f * o[j].w;
+      }
     }
   }
   const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;

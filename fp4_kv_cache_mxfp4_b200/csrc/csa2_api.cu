@@ -20,8 +20,6 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxDynSmem = 227 * 1024;
-constexpr int kTopkChunk = 4096;
-constexpr int kCandCap = 32768;
 
 struct DeviceInfo {
   bool init = false;
@@ -32,6 +30,40 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// index_scan_kernel instances: queries per MMA group (1, 2, 4, 8) x HSI
+template <int QG, bool HSI>
+cudaError_t set_scan_attr_one() {
+  return cudaFuncSetAttribute(index_scan_kernel<QG, HSI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+}
+cudaError_t set_scan_attrs() {
+  cudaError_t e = cudaSuccess;
+  cudaError_t r[8] = {set_scan_attr_one<1, false>(), set_scan_attr_one<1, true>(), set_scan_attr_one<2, false>(),
+                      set_scan_attr_one<2, true>(), set_scan_attr_one<4, false>(), set_scan_attr_one<4, true>(),
+                      set_scan_attr_one<8, false>(), set_scan_attr_one<8, true>()};
+  for (cudaError_t x : r) if (x != cudaSuccess) e = x;
+  return e;
+}
+inline int scan_qg(int qg) { return qg <= 1 ? 1 : qg <= 2 ? 2 : qg <= 4 ? 4 : 8; }
+
+template <int QG, bool HSI>
+void launch_scan_t(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk, const CUtensorMap& tq,
+                   const ScanParams& sp) {
+  index_scan_kernel<QG, HSI><<<grid, kScanThreads, smem, st>>>(tk, tq, sp);
+}
+void launch_scan(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
+                 const CUtensorMap& tq, const ScanParams& sp) {
+  switch (QG * 2 + (hsi ? 1 : 0)) {
+    case 2: launch_scan_t<1, false>(grid, smem, st, tk, tq, sp); break;
+    case 3: launch_scan_t<1, true>(grid, smem, st, tk, tq, sp); break;
+    case 4: launch_scan_t<2, false>(grid, smem, st, tk, tq, sp); break;
+    case 5: launch_scan_t<2, true>(grid, smem, st, tk, tq, sp); break;
+    case 8: launch_scan_t<4, false>(grid, smem, st, tk, tq, sp); break;
+    case 9: launch_scan_t<4, true>(grid, smem, st, tk, tq, sp); break;
+    case 16: launch_scan_t<8, false>(grid, smem, st, tk, tq, sp); break;
+    default: launch_scan_t<8, true>(grid, smem, st, tk, tq, sp); break;
+  }
+}
 
 csa2_status device_info(DeviceInfo** out) {
   int dev = 0;
@@ -47,9 +79,9 @@ csa2_status device_info(DeviceInfo** out) {
   }
   if (!d.ok) return CSA2_ERR_ARCH;
   if (!d.attrs_set) {
-    if (cudaFuncSetAttribute(index_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) != cudaSuccess ||
+    if (set_scan_attrs() != cudaSuccess ||
         cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(topk_smem_bytes(12))) != cudaSuccess ||
+                             static_cast<int>(topk_smem_bytes())) != cudaSuccess ||
         cudaFuncSetAttribute(sparse_attn_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
       return CSA2_ERR_CUDA;
     if (!g_encode) {
@@ -83,12 +115,12 @@ bool make_map_bf16_128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t
 // ---------------------------------------------------------------- index call
 struct IndexPlan {
   bool pool, hsi;
-  int BQ, qg, hb, cap, bcap;
+  int BQ, qg, hb, nchunks, bchunks;
   int64_t n_elems, nblk;
   // counter region (histograms, candidate counters, tickets): zeroed at the
   // start of every call; data region (scores, candidates): no precondition
-  size_t off_hist, off_bhist, off_ctr, off_bctr, zero_bytes;
-  size_t off_scores, off_bscores, off_cand, off_bcand, data_bytes;
+  size_t off_hist, off_bhist, off_ctr, zero_bytes;
+  size_t off_scores, off_bscores, off_seg, off_bseg, off_cnt, off_bcnt, data_bytes;
   size_t total;
 };
 
@@ -122,20 +154,21 @@ IndexPlan plan_index(const csa2_index_args* a) {
   P.hb = (P.qg <= 2) ? 12 : 10;
   P.n_elems = P.pool ? static_cast<int64_t>(a->hsi_blocks) * 8 : a->N;
   P.nblk = P.hsi ? (a->N + 7) / 8 : 0;
-  P.cap = static_cast<int>(std::min<int64_t>(P.n_elems, kCandCap));
-  P.bcap = static_cast<int>(std::min<int64_t>(P.nblk, kCandCap));
+  P.nchunks = static_cast<int>((P.n_elems + kTopkChunk - 1) / kTopkChunk);
+  P.bchunks = static_cast<int>((P.nblk + kTopkChunk - 1) / kTopkChunk);
   const size_t nb = static_cast<size_t>(1) << P.hb;
   size_t off = 0;
   P.off_hist = off;    off = up256(off + static_cast<size_t>(P.BQ) * nb * 4);
   P.off_bhist = off;   off = up256(off + (P.hsi ? static_cast<size_t>(P.BQ) * nb * 4 : 0));
-  P.off_ctr = off;     off = up256(off + static_cast<size_t>(P.BQ) * 16);
-  P.off_bctr = off;    off = up256(off + static_cast<size_t>(P.BQ) * 16);
+  P.off_ctr = off;     off = up256(off + static_cast<size_t>(P.BQ) * 8 * 4);
   P.zero_bytes = off;
   off = 0;
   P.off_scores = off;  off = up256(off + static_cast<size_t>(P.BQ) * P.n_elems * 4);
   P.off_bscores = off; off = up256(off + static_cast<size_t>(P.BQ) * P.nblk * 4);
-  P.off_cand = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.cap * 8);
-  P.off_bcand = off;   off = up256(off + static_cast<size_t>(P.BQ) * P.bcap * 8);
+  P.off_seg = off;     off = up256(off + static_cast<size_t>(P.BQ) * P.n_elems * 8);
+  P.off_bseg = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.nblk * 8);
+  P.off_cnt = off;     off = up256(off + static_cast<size_t>(P.BQ) * P.nchunks * 4);
+  P.off_bcnt = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.bchunks * 4);
   P.data_bytes = off;
   P.total = P.zero_bytes + P.data_bytes;
   return P;
@@ -159,27 +192,30 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.nblk = P.nblk;
   sp.hist = reinterpret_cast<uint32_t*>(z + P.off_hist);
   sp.bhist = P.hsi ? reinterpret_cast<uint32_t*>(z + P.off_bhist) : nullptr;
+  sp.ctr = reinterpret_cast<uint32_t*>(z + P.off_ctr);
+  sp.K = a->K;
+  sp.bK = P.hsi ? a->hsi_blocks : 0;
   sp.hb = P.hb;
   sp.groups = P.pool ? P.BQ : a->B;
   sp.tiles_per_group = static_cast<int>((P.n_elems + kTileRows - 1) / kTileRows);
   sp.ctas_per_group = std::max(1, std::min(sp.tiles_per_group, dev.sms / sp.groups));
-  const uint32_t n_mma = 32u * P.qg;
-  sp.acc_bufs = n_mma <= 64 ? 4 : 2;
+  const int QG = scan_qg(P.qg);
+  const uint32_t n_mma = 32u * QG;
   uint32_t cols = 32;
-  while (cols < sp.acc_bufs * n_mma) cols <<= 1;
+  while (cols < scan_acc_bufs(QG) * n_mma) cols <<= 1;
   sp.tmem_cols = cols;
-  const ScanSmem L0 = scan_smem_layout(0, P.qg, P.hb, P.hsi);
+  const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi);
   sp.stages = std::min(8, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / kStageBytes));
   if (sp.stages < 2) return CSA2_ERR_SHAPE;
-  const ScanSmem L = scan_smem_layout(sp.stages, P.qg, P.hb, P.hsi);
+  const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi);
 
   CUtensorMap tk, tq;
   if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : kTileRows)) return CSA2_ERR_CUDA;
-  if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, 32u * P.qg)) return CSA2_ERR_CUDA;
+  if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, n_mma)) return CSA2_ERR_CUDA;
 
   const unsigned grid = static_cast<unsigned>(sp.groups * sp.ctas_per_group);
   trace_pre(kKIndexScan, st);
-  index_scan_kernel<<<grid, kScanThreads, L.total + 1024, st>>>(tk, tq, sp);
+  launch_scan(QG, P.hsi, grid, L.total + 1024, st, tk, tq, sp);
   trace_post(st);
   if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
 
@@ -191,20 +227,19 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   tp.vis_div = 1;
   tp.pool = sp.pool;
   tp.pool_blocks = sp.pool_blocks;
-  tp.hist = sp.hist;
   tp.hb = P.hb;
-  tp.cand = reinterpret_cast<uint64_t*>(w + P.off_cand);
-  tp.cap = P.cap;
-  tp.ctr = reinterpret_cast<uint32_t*>(z + P.off_ctr);
+  tp.seg = reinterpret_cast<uint64_t*>(w + P.off_seg);
+  tp.seg_cnt = reinterpret_cast<uint32_t*>(w + P.off_cnt);
+  tp.nchunks = P.nchunks;
+  tp.ctr = sp.ctr;
+  tp.tb_slot = 2;
+  tp.ticket_slot = 1;
   tp.K = a->K;
-  tp.chunk = kTopkChunk;
   tp.out_idx = a->idx;
   tp.out_scores = a->scores;
-  tp.out_by_pos = 0;
-  const size_t tsm = topk_smem_bytes(P.hb);
-  dim3 tgrid(static_cast<unsigned>((P.n_elems + kTopkChunk - 1) / kTopkChunk), static_cast<unsigned>(P.BQ));
+  const size_t tsm = topk_smem_bytes();
   trace_pre(kKTopk, st);
-  topk_select_kernel<<<tgrid, kTopkThreads, tsm, st>>>(tp);
+  topk_select_kernel<<<dim3(static_cast<unsigned>(P.nchunks), static_cast<unsigned>(P.BQ)), kTopkThreads, tsm, st>>>(tp);
   trace_post(st);
   if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
 
@@ -215,17 +250,16 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
     bp.n_vis = a->n_vis;
     bp.vis_div = 8;
     bp.pool = nullptr;
-    bp.hist = sp.bhist;
-    bp.cand = reinterpret_cast<uint64_t*>(w + P.off_bcand);
-    bp.cap = P.bcap;
-    bp.ctr = reinterpret_cast<uint32_t*>(z + P.off_bctr);
+    bp.seg = reinterpret_cast<uint64_t*>(w + P.off_bseg);
+    bp.seg_cnt = reinterpret_cast<uint32_t*>(w + P.off_bcnt);
+    bp.nchunks = P.bchunks;
+    bp.tb_slot = 4;
+    bp.ticket_slot = 6;
     bp.K = a->hsi_blocks;
     bp.out_idx = a->pool_out;
     bp.out_scores = nullptr;
-    bp.out_by_pos = 1;
-    dim3 bgrid(static_cast<unsigned>((P.nblk + kTopkChunk - 1) / kTopkChunk), static_cast<unsigned>(P.BQ));
     trace_pre(kKTopk, st);
-    topk_select_kernel<<<bgrid, kTopkThreads, tsm, st>>>(bp);
+    topk_select_kernel<<<dim3(static_cast<unsigned>(P.bchunks), static_cast<unsigned>(P.BQ)), kTopkThreads, tsm, st>>>(bp);
     trace_post(st);
     if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
   }

@@ -5,17 +5,20 @@
 //
 // The contraction is D[t, (q,h)] = kI_tile[t, :] . qI[(q,h), :]: a
 // 128-entry tile of index-K (128 rows x 128 dims, bf16) is the A operand,
-// the row's index-Q (32*Q heads x 128 dims) is the B operand, the fp32
-// accumulator (128 lanes x 32*Q columns) lives in tensor memory.  Each
-// epilogue thread then owns one entry: it reads its 32*Q head values from
-// TMEM and reduces them to Q scores (ReLU, weight, sum).
+// the row's index-Q (32*QG heads x 128 dims) is the B operand, the fp32
+// accumulator (128 lanes x 32*QG columns) lives in tensor memory.  Each
+// epilogue thread then owns one entry: it reads its 32*QG head values from
+// TMEM and reduces them to QG scores (ReLU, weight, sum).
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: streams index-K tiles into an S-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2..5  epilogue: TMEM -> scores, fused score histogram (for the
-//               top-K threshold) and, with HSI, the block max over 8
-//               positions with its own histogram
+//   warps 2..9  epilogue, two sets of four warps taking alternate tiles
+//               (each set covers the 128 TMEM lanes): TMEM -> scores, the
+//               score histogram used for the top-K threshold and, with HSI,
+//               the block max over 8 positions with its own histogram
+// After the last tile every CTA adds its histograms to the global ones; the
+// last CTA of each group turns them into the threshold bin of each query.
 // Pool mode (Reindex restricted to the HSI pool) gathers the tile as 16
 // blocks of 8 contiguous index-K rows with one 1 KB TMA box per block half.
 //
@@ -26,14 +29,20 @@
 
 namespace csa2 {
 
-constexpr int kScanThreads = 192;
-constexpr int kTileRows = 128;               // entries per MMA tile (M)
+constexpr int kScanEpiWarps = 8;
+constexpr int kScanEpiThreads = kScanEpiWarps * 32;
+constexpr int kScanThreads = 64 + kScanEpiThreads;
+constexpr int kTileRows = 128;                     // entries per MMA tile (M)
 constexpr int kStageBytes = kTileRows * 128 * 2;   // 32 KB: two 128x64 swizzled boxes
+constexpr int kAccBufs = 4;                        // TMEM accumulator slots (barriers)
+
+// accumulators in flight: as many as fit the 512 TMEM columns, at most 4
+__host__ __device__ constexpr int scan_acc_bufs(int QG) { return 32 * QG * 4 <= 512 ? 4 : 2; }
 
 struct ScanParams {
   int pool_mode;          // 0: scan [0, n_vis) of each row; 1: scan the pool of each (b,q)
   int B, Q;               // batch rows, queries per row
-  int qg;                 // queries per MMA group: Q (scan) or 1 (pool)
+  int qg;                 // queries of an MMA group: Q (scan) or 1 (pool); <= the QG template
   int64_t N;              // index-K rows per batch row
   int64_t n_elems;        // score slots per query: N (scan) or pool_blocks*8 (pool)
   const int32_t* n_vis;   // [B*Q]
@@ -43,14 +52,16 @@ struct ScanParams {
   float* scores;          // [B*Q][n_elems]
   float* bscores;         // scan with HSI: [B*Q][nblk]
   int64_t nblk;
-  uint32_t* hist;         // [B*Q][1 << hb]
+  uint32_t* hist;         // [B*Q][1 << hb]       (zero at launch)
   uint32_t* bhist;        // scan with HSI: [B*Q][1 << hb]
+  uint32_t* ctr;          // [B*Q][8]             (zero at launch): [0] group ticket (first query
+                          // of the group), [2..3] tb, need; [4..5] block tb, need
+  int K, bK;              // top-K of positions and (HSI) of blocks
   int hb;                 // histogram bits
   int groups;             // B (scan) or B*Q (pool)
   int tiles_per_group;
   int ctas_per_group;
   int stages;
-  int acc_bufs;
   uint32_t tmem_cols;
 };
 
@@ -59,20 +70,61 @@ struct ScanSmem {
   uint32_t stage0, qi0, w0, hist0, bhist0, bar0, total;
 };
 
-__host__ __device__ inline ScanSmem scan_smem_layout(int stages, int qg, int hb, int hsi) {
+__host__ __device__ inline ScanSmem scan_smem_layout(int stages, int QG, int hb, int hsi) {
   ScanSmem L;
   uint32_t off = 0;
   L.stage0 = off; off += stages * kStageBytes;
-  L.qi0 = off;    off += 2 * (32 * qg) * 128;          // two 64-dim halves of [32*qg x 64] bf16
-  L.w0 = off;     off += qg * 32 * 4;
-  L.hist0 = off;  off += qg * (1u << hb) * 4;
-  L.bhist0 = off; off += hsi ? qg * (1u << hb) * 4 : 0;
+  L.qi0 = off;    off += 2 * (32 * QG) * 128;          // two 64-dim halves of [32*QG x 64] bf16
+  L.w0 = off;     off += QG * 32 * 4;
+  L.hist0 = off;  off += QG * (1u << hb) * 4;
+  L.bhist0 = off; off += hsi ? QG * (1u << hb) * 4 : 0;
   off = (off + 15) & ~15u;
-  L.bar0 = off;   off += (2 * stages + 2 * 4 + 2) * 8 + 16;
+  L.bar0 = off;   off += (2 * stages + 2 * kAccBufs + 2) * 8 + 16 + 64;   // barriers, TMEM slot, flags, scratch
   L.total = off;
   return L;
 }
 
+// Threshold bin for a top-K from a complete global histogram, run by the 256
+// epilogue threads: tb = highest bin whose suffix count reaches
+// need = min(K, total); writes out[0] = tb (nbins when need == 0) and
+// out[1] = need.  stage: nbins words of shared scratch; red: 8 words.
+__device__ void scan_threshold_bin(const uint32_t* hist, int nbins, int K, uint32_t* out, uint32_t* stage,
+                                   uint32_t* red) {
+  const int et = threadIdx.x - 64, lane = threadIdx.x & 31, ew = et >> 5;
+  // coalesced copy into shared memory, all loads in flight together
+#pragma unroll 8
+  for (int i = et; i < nbins; i += kScanEpiThreads) stage[i] = __ldcg(hist + i);
+  named_bar_sync(1, kScanEpiThreads);
+  const int per = nbins / kScanEpiThreads;
+  const int hi = nbins - 1 - et * per;             // this thread owns bins [hi-per+1, hi]
+  uint32_t local = 0;
+  for (int j = 0; j < per; ++j) local += stage[hi - j];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) red[ew] = incl;
+  named_bar_sync(1, kScanEpiThreads);
+  uint32_t wbase = 0, total = 0;
+  for (int w = 0; w < kScanEpiWarps; ++w) { if (w < ew) wbase += red[w]; total += red[w]; }
+  const uint32_t need = total < static_cast<uint32_t>(K) ? total : static_cast<uint32_t>(K);
+  uint32_t above = wbase + incl - local;
+  if (need > 0 && above < need && above + local >= need) {
+    for (int j = 0; j < per; ++j) {
+      above += stage[hi - j];
+      if (above >= need) { out[0] = hi - j; break; }
+    }
+  }
+  if (et == 0) {
+    out[1] = need;
+    if (need == 0) out[0] = nbins;
+  }
+  named_bar_sync(1, kScanEpiThreads);
+}
+
+template <int QG, bool HSI>
 __global__ void __launch_bounds__(kScanThreads, 1)
 index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_q,
@@ -80,15 +132,15 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the swizzle atoms need 1024-byte alignment of every operand tile
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int hsi = (p.bscores != nullptr);
-  const ScanSmem L = scan_smem_layout(p.stages, p.qg, p.hb, hsi);
+  const ScanSmem L = scan_smem_layout(p.stages, QG, p.hb, HSI);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L.bar0);
   uint64_t* empty_bar = full_bar + p.stages;
   uint64_t* tfull_bar = empty_bar + p.stages;
-  uint64_t* tempty_bar = tfull_bar + 4;
-  uint64_t* q_bar = tempty_bar + 4;
+  uint64_t* tempty_bar = tfull_bar + kAccBufs;
+  uint64_t* q_bar = tempty_bar + kAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* red = tmem_slot + 2;                   // 9 words of scratch
   float* w_s = reinterpret_cast<float*>(smem + L.w0);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L.hist0);
   uint32_t* bhist_s = reinterpret_cast<uint32_t*>(smem + L.bhist0);
@@ -105,30 +157,35 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   // this CTA's tile range; in scan mode, tiles past every query's n_vis are skipped
   int tile_lo = static_cast<int>((static_cast<int64_t>(cig) * p.tiles_per_group) / p.ctas_per_group);
   int tile_hi = static_cast<int>((static_cast<int64_t>(cig + 1) * p.tiles_per_group) / p.ctas_per_group);
+  int nv[QG];
+#pragma unroll
+  for (int q = 0; q < QG; ++q) nv[q] = (q < p.qg) ? p.n_vis[bq0 + q] : 0;
   if (!p.pool_mode) {
     int nmax = 0;
-    for (int q = 0; q < p.qg; ++q) nmax = max(nmax, p.n_vis[bq0 + q]);
+#pragma unroll
+    for (int q = 0; q < QG; ++q) nmax = max(nmax, nv[q]);
     tile_hi = min(tile_hi, (nmax + kTileRows - 1) / kTileRows);
   }
   const int ntiles = max(0, tile_hi - tile_lo);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-    for (int a = 0; a < p.acc_bufs; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 128); }
+    for (int a = 0; a < scan_acc_bufs(QG); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 128); }
     mbar_init(q_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmap_k); tma_prefetch_desc(&tmap_q); }
   if (warp == 1) { tmem_alloc(tmem_slot, p.tmem_cols); tmem_relinquish(); }
-  for (int i = threadIdx.x; i < p.qg * nbins; i += blockDim.x) hist_s[i] = 0;
-  if (hsi) for (int i = threadIdx.x; i < p.qg * nbins; i += blockDim.x) bhist_s[i] = 0;
-  for (int i = threadIdx.x; i < p.qg * 32; i += blockDim.x) w_s[i] = p.w[bq0 * 32 + i];
+  for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) hist_s[i] = 0;
+  if (HSI) for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) bhist_s[i] = 0;
+  for (int i = threadIdx.x; i < QG * 32; i += blockDim.x) w_s[i] = (i < p.qg * 32) ? p.w[bq0 * 32 + i] : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t n_mma = 32u * p.qg;
+  constexpr uint32_t n_mma = 32u * QG;
+  constexpr int ACC = scan_acc_bufs(QG);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -136,7 +193,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const uint64_t pol_stream = l2_policy_evict_first();
       const uint64_t pol_keep = l2_policy_evict_last();
       uint8_t* qi = smem + L.qi0;
-      const uint32_t qbox = n_mma * 128;
+      constexpr uint32_t qbox = n_mma * 128;
       mbar_arrive_expect_tx(q_bar, 2 * qbox);
       tma_load_2d(qi, &tmap_q, q_bar, 0, bq0 * 32, pol_keep);
       tma_load_2d(qi + qbox, &tmap_q, q_bar, 64, bq0 * 32, pol_keep);
@@ -168,14 +225,14 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && ntiles > 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(128, n_mma);
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(128, n_mma);
       const uint32_t qi_addr = smem_u32(smem + L.qi0);
-      const uint32_t qbox = n_mma * 128;
+      constexpr uint32_t qbox = n_mma * 128;
       bool ok = mbar_wait(q_bar, 0, kErrWaitOperand, abort_flag);
       for (int i = 0; ok && i < ntiles; ++i) {
         const int s = i % p.stages;
-        const int a = i % p.acc_bufs;
-        if (!mbar_wait(&tempty_bar[a], ((i / p.acc_bufs) & 1) ^ 1, kErrWaitTmemEmpty, abort_flag)) break;
+        const int a = i % ACC;
+        if (!mbar_wait(&tempty_bar[a], ((i / ACC) & 1) ^ 1, kErrWaitTmemEmpty, abort_flag)) break;
         if (!mbar_wait(&full_bar[s], (i / p.stages) & 1, kErrWaitTmaFull, abort_flag)) break;
         tc_fence_after();
         const uint32_t st_addr = smem_u32(smem + L.stage0 + s * kStageBytes);
@@ -195,46 +252,55 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;                 // TMEM lanes this warp may read
+    const int set = (warp - 2) >> 2;              // tiles set, set+2, set+4, ...
     const int row = quarter * 32 + lane;          // entry within the tile
-    int nv[8];
-    for (int q = 0; q < p.qg; ++q) nv[q] = p.n_vis[bq0 + q];
     const int32_t* pool = p.pool_mode ? p.pool + static_cast<int64_t>(bq0) * p.pool_blocks : nullptr;
-    for (int i = 0; i < ntiles; ++i) {
-      const int a = i % p.acc_bufs;
+    // the weights of one or two queries stay in registers
+    constexpr int WREG = (QG <= 2) ? QG * 32 : 1;
+    float wr[WREG];
+#pragma unroll
+    for (int h = 0; h < WREG; ++h) wr[h] = (QG <= 2) ? w_s[h] : 0.0f;
+    for (int i = set; i < ntiles; i += 2) {
+      const int a = i % ACC;
       // tcgen05.ld is warp-collective: leave the loop as a whole warp
-      const bool ok = mbar_wait(&tfull_bar[a], (i / p.acc_bufs) & 1, kErrWaitTmemFull, abort_flag);
+      const bool ok = mbar_wait(&tfull_bar[a], (i / ACC) & 1, kErrWaitTmemFull, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int tile = tile_lo + i;
       const int64_t e = static_cast<int64_t>(tile) * kTileRows + row;   // score slot
-      for (int q = 0; q < p.qg; ++q) {
+      bool pool_valid = true;
+      int64_t pos = e;
+      if (p.pool_mode) {
+        const int64_t slot = e >> 3;
+        const int blk = (slot < p.pool_blocks) ? pool[slot] : -1;
+        pool_valid = blk >= 0;
+        pos = static_cast<int64_t>(blk) * 8 + (e & 7);
+      }
+#pragma unroll
+      for (int q = 0; q < QG; ++q) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * n_mma + 32 * q, r);
         tmem_ld_wait();
-        float s = 0.0f;
-        const float* wq = w_s + 32 * q;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int h = 0; h < 32; ++h) s = fmaf(wq[h], fmaxf(__uint_as_float(r[h]), 0.0f), s);
-        bool valid;
-        if (!p.pool_mode) {
-          valid = e < nv[q];
-        } else {
-          const int64_t slot = e >> 3;
-          const int blk = (slot < p.pool_blocks) ? pool[slot] : -1;
-          valid = blk >= 0 && (static_cast<int64_t>(blk) * 8 + (e & 7)) < nv[q];
+        for (int h = 0; h < 32; ++h) {
+          const float wh = (QG <= 2) ? wr[(QG <= 2 ? q : 0) * 32 + h] : w_s[q * 32 + h];
+          acc[h & 3] = fmaf(wh, fmaxf(__uint_as_float(r[h]), 0.0f), acc[h & 3]);
         }
+        float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const bool valid = pool_valid && pos < nv[q] && q < p.qg;
         if (!valid) s = -INFINITY;
-        if (e < p.n_elems) {
+        if (e < p.n_elems && q < p.qg) {
           p.scores[static_cast<int64_t>(bq0 + q) * p.n_elems + e] = s;
           if (valid) atomicAdd(&hist_s[q * nbins + (okey(s) >> (32 - p.hb))], 1u);
         }
-        if (hsi) {
+        if (HSI) {
           float m = s;
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
           const int64_t jb = e >> 3;
-          if ((lane & 7) == 0 && jb < p.nblk) {
+          if ((lane & 7) == 0 && jb < p.nblk && q < p.qg) {
             p.bscores[static_cast<int64_t>(bq0 + q) * p.nblk + jb] = m;
             if (m != -INFINITY) atomicAdd(&bhist_s[q * nbins + (okey(m) >> (32 - p.hb))], 1u);
           }
@@ -244,14 +310,30 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
       mbar_arrive(&tempty_bar[a]);
     }
     // flush the CTA's histograms into the global ones
-    named_bar_sync(1, 128);
+    named_bar_sync(1, kScanEpiThreads);
     const int et = threadIdx.x - 64;
-    for (int i = et; i < p.qg * nbins; i += 128) {
+    for (int i = et; i < p.qg * nbins; i += kScanEpiThreads) {
       const uint32_t v = hist_s[i];
       if (v) atomicAdd(&p.hist[static_cast<int64_t>(bq0 + i / nbins) * nbins + (i % nbins)], v);
-      if (hsi) {
+      if (HSI) {
         const uint32_t bv = bhist_s[i];
         if (bv) atomicAdd(&p.bhist[static_cast<int64_t>(bq0 + i / nbins) * nbins + (i % nbins)], bv);
+      }
+    }
+    // the last CTA of the group turns the complete histograms into the
+    // threshold bin of each query's top-K (and of its HSI block top-K)
+    __threadfence();
+    named_bar_sync(1, kScanEpiThreads);
+    if (et == 0) red[8] = (atomicAdd(&p.ctr[static_cast<int64_t>(bq0) * 8], 1u) == static_cast<uint32_t>(p.ctas_per_group - 1));
+    named_bar_sync(1, kScanEpiThreads);
+    if (red[8]) {
+      __threadfence();
+      for (int q = 0; q < p.qg; ++q) {
+        scan_threshold_bin(p.hist + static_cast<int64_t>(bq0 + q) * nbins, nbins, p.K,
+                           p.ctr + static_cast<int64_t>(bq0 + q) * 8 + 2, hist_s, red);
+        if (HSI)
+          scan_threshold_bin(p.bhist + static_cast<int64_t>(bq0 + q) * nbins, nbins, p.bK,
+                             p.ctr + static_cast<int64_t>(bq0 + q) * 8 + 4, hist_s, red);
       }
     }
   }

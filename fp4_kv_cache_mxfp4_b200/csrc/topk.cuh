@@ -5,26 +5,30 @@
 // word inverts the position, so every key is distinct and "larger key" means
 // "higher score, then lower position": the top-K set is the K largest keys.
 //
-// One launch per selection problem, grid (chunks, queries):
-//  1. every CTA reads the query's score histogram (built by the scan
-//     epilogue) and finds the threshold bin tb: the highest bin whose
-//     suffix count reaches K;
-//  2. every CTA appends the keys of its chunk whose bin is >= tb to the
-//     query's candidate list (warp-aggregated atomics);
-//  3. the last CTA to finish (ticket counter) radix-selects the K-th key
-//     among the candidates (8-bit digits, from the top), gathers the K keys
-//     at or above it, sorts them (bitonic, descending) and writes positions
-//     and scores.  If the candidate list overflowed, step 3 runs over the scores
-//     themselves (same filter), which is slower but exact.
-// HBM roofline: 4 B per score read (the scores are usually still in L2).
+// The scan kernel has already reduced the score histogram of each query to
+// a threshold bin tb (every top-K key has its top bits >= tb) and the count
+// `need` = min(K, visible).  One launch per selection problem, grid
+// (chunks, queries), 1024 threads:
+//  1. every CTA compacts the keys of its 4096-slot chunk whose bin is >= tb
+//     into the chunk's own segment, in position order (block prefix scan),
+//     and records the segment's length;
+//  2. the last CTA of the query (ticket counter) gathers the segments in
+//     chunk order into shared memory, radix-selects the need-th largest key
+//     (8-bit digits from the top) and writes the keys at or above it by an
+//     ordered compaction: the result comes out in ascending position order,
+//     deterministically, without a sort.
+// If the candidates do not fit in shared memory, step 2 runs over the
+// scores themselves with the same filter (slower, exact).
+// HBM roofline: 4 B per score read (normally still resident in L2).
 #pragma once
 #include "common.cuh"
 
 namespace csa2 {
 
 constexpr int kTopkThreads = 1024;
-constexpr int kTopkSmemKeys = 4096;      // candidates cached in shared memory
-constexpr int kTopkMaxK = 2048;
+constexpr int kTopkChunk = 4096;          // slots per CTA (4 per thread)
+constexpr int kTopkSmemKeys = 6144;       // candidates cached in shared memory
+constexpr int kTopkMaxChunks = 2048;      // chunk offsets kept in shared memory
 
 struct TopkParams {
   const float* scores;
@@ -33,22 +37,23 @@ struct TopkParams {
   int vis_div;
   const int32_t* pool;      // pool mode: position of slot e = pool[e/8]*8 + e%8
   int pool_blocks;
-  uint32_t* hist;           // [BQ][1 << hb]
   int hb;
-  uint64_t* cand;           // [BQ][cap]
-  int cap;
-  uint32_t* ctr;            // [BQ][4]: candidate count, finished CTAs (zero at launch)
+  uint64_t* seg;            // [BQ][n_elems]: chunk c's candidates at c*kTopkChunk
+  uint32_t* seg_cnt;        // [BQ][nchunks]
+  int nchunks;
+  uint32_t* ctr;            // [BQ][8] (zero at the scan's launch)
+  int tb_slot;              // ctr[tb_slot] = tb, ctr[tb_slot+1] = need (from the scan)
+  int ticket_slot;
   int K;
-  int chunk;                // slots per CTA
   int32_t* out_idx;         // [BQ][K]
   float* out_scores;        // optional [BQ][K]
-  int out_by_pos;           // 1: ascending positions (pool output), 0: best first
 };
 
 struct TopkShared {
   uint32_t h256[256];
-  int tb, need, last, d, gt, eq, cnt, total;
-  uint32_t warp_sum[32];
+  uint32_t warp_tot[32];
+  uint32_t chunk_off[kTopkMaxChunks + 1];
+  int last, d, gt, eq, total;
 };
 
 __device__ __forceinline__ int64_t topk_valid_slots(const TopkParams& p, int bq) {
@@ -72,8 +77,38 @@ __device__ __forceinline__ uint64_t topk_slot_key(const TopkParams& p, int bq, i
   return (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(~topk_position(p, bq, e));
 }
 
-// Highest digit d of a 256-bin histogram with suffix(d) >= remaining, run by
-// warp 0; lane l owns bins 255-8l .. 248-8l.
+// Exclusive prefix sum over the block (1024 threads); *total gets the sum.
+// Ends with a barrier so the scratch can be reused.
+__device__ __forceinline__ uint32_t topk_block_scan(uint32_t v, TopkShared& S, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) S.warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t x = S.warp_tot[lane];
+    uint32_t xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += t;
+    }
+    S.warp_tot[lane] = xi - x;                      // exclusive per warp
+    if (lane == 31) S.total = static_cast<int>(xi);
+  }
+  __syncthreads();
+  const uint32_t r = S.warp_tot[warp] + incl - v;
+  *total = static_cast<uint32_t>(S.total);
+  __syncthreads();
+  return r;
+}
+
+// Highest digit d of the 256-bin histogram with suffix(d) >= remaining, run
+// by warp 0; lane l owns bins 255-8l .. 248-8l.
 __device__ __forceinline__ void topk_pick_digit(TopkShared& S, int remaining) {
   const int lane = threadIdx.x & 31;
   uint32_t c[8], local = 0;
@@ -129,81 +164,53 @@ __device__ uint64_t topk_radix_select(TopkShared& S, int64_t n, int need, KeyAt 
   }
 }
 
+__device__ __forceinline__ void topk_emit(const TopkParams& p, int32_t* out_idx, float* out_sc, uint32_t slot,
+                                          uint64_t k) {
+  if (slot >= static_cast<uint32_t>(p.K)) return;
+  out_idx[slot] = static_cast<int32_t>(~static_cast<uint32_t>(k));
+  if (out_sc) out_sc[slot] = okey_to_float(static_cast<uint32_t>(k >> 32));
+}
+
 __global__ void __launch_bounds__(kTopkThreads)
 topk_select_kernel(TopkParams p) {
   extern __shared__ __align__(1024) uint8_t topk_smem_raw[];
   TopkShared& S = *reinterpret_cast<TopkShared*>(topk_smem_raw);
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(topk_smem_raw + sizeof(TopkShared));
-  const int nbins = 1 << p.hb;
-  uint64_t* keys_s = reinterpret_cast<uint64_t*>(hist_s + nbins);        // kTopkSmemKeys
-  uint64_t* sort_s = keys_s + kTopkSmemKeys;                              // kTopkMaxK
+  uint64_t* keys_s = reinterpret_cast<uint64_t*>(topk_smem_raw + ((sizeof(TopkShared) + 15) & ~size_t(15)));
 
   const int bq = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t* hist = p.hist + static_cast<int64_t>(bq) * nbins;
-  uint32_t* ctr = p.ctr + bq * 4;
+  const int tid = threadIdx.x;
+  uint32_t* ctr = p.ctr + static_cast<int64_t>(bq) * 8;
+  const int tb = static_cast<int>(__ldcg(ctr + p.tb_slot));
+  const int need = static_cast<int>(__ldcg(ctr + p.tb_slot + 1));
   const int64_t nvalid = topk_valid_slots(p, bq);
+  uint64_t* seg_q = p.seg + static_cast<int64_t>(bq) * p.n_elems;
+  uint32_t* cnt_q = p.seg_cnt + static_cast<int64_t>(bq) * p.nchunks;
 
-  // -- 1. threshold bin from the histogram --------------------------------
-  for (int i = tid; i < nbins; i += blockDim.x) hist_s[i] = __ldcg(hist + i);
-  __syncthreads();
-  const int per = (nbins + blockDim.x - 1) / blockDim.x;      // bins per thread, from the top
-  const int hi_bin = nbins - 1 - tid * per;                   // this thread: [hi_bin-per+1, hi_bin]
-  uint32_t local = 0;
-  for (int j = 0; j < per; ++j) if (hi_bin - j >= 0) local += hist_s[hi_bin - j];
-  uint32_t incl = local;
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) S.warp_sum[warp] = incl;
-  if (tid == 0) S.tb = nbins;
-  __syncthreads();
-  uint32_t wbase = 0, total = 0;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
-    if (w < warp) wbase += S.warp_sum[w];
-    total += S.warp_sum[w];
-  }
-  const int need = static_cast<int>(total < static_cast<uint32_t>(p.K) ? total : static_cast<uint32_t>(p.K));
-  uint32_t above = wbase + incl - local;                      // count in bins above this thread's range
-  if (need > 0 && above < static_cast<uint32_t>(need) && above + local >= static_cast<uint32_t>(need)) {
-    for (int j = 0; j < per; ++j) {
-      const int bin = hi_bin - j;
-      if (bin < 0) break;
-      above += hist_s[bin];
-      if (above >= static_cast<uint32_t>(need)) { S.tb = bin; break; }
+  // -- 1. this chunk's candidates, in position order ------------------------
+  {
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kTopkChunk;
+    uint64_t k[4];
+    uint32_t n = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t e = base + 4 * tid + i;
+      k[i] = (need > 0 && e < nvalid) ? topk_slot_key(p, bq, e, tb) : 0;
+      n += (k[i] != 0);
     }
-  }
-  if (tid == 0) { S.need = need; S.total = static_cast<int>(total); }
-  __syncthreads();
-  const int tb = S.tb;
-
-  // -- 2. candidates of this chunk -----------------------------------------
-  if (need > 0) {
-    const int64_t lo = static_cast<int64_t>(blockIdx.x) * p.chunk;
-    const int64_t hi = min(lo + p.chunk, nvalid);
-    uint64_t* cand = p.cand + static_cast<int64_t>(bq) * p.cap;
-    for (int64_t base = lo + warp * 32; base < hi; base += blockDim.x) {
-      const int64_t e = base + lane;
-      const uint64_t k = (e < hi) ? topk_slot_key(p, bq, e, tb) : 0;
-      const uint32_t m = __ballot_sync(0xffffffffu, k != 0);
-      if (m == 0) continue;
-      uint32_t off = 0;
-      if (lane == 0) off = atomicAdd(&ctr[0], __popc(m));
-      off = __shfl_sync(0xffffffffu, off, 0);
-      if (k != 0) {
-        const uint32_t slot = off + __popc(m & ((1u << lane) - 1));
-        if (slot < static_cast<uint32_t>(p.cap)) cand[slot] = k;
-      }
-    }
+    uint32_t total;
+    uint32_t off = topk_block_scan(n, S, &total);
+    uint64_t* seg = seg_q + base;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (k[i] != 0) seg[off++] = k[i];
+    if (tid == 0) cnt_q[blockIdx.x] = total;
   }
 
-  // -- 3. the last CTA of this query selects --------------------------------
+  // -- 2. the last CTA of this query selects ---------------------------------
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    const uint32_t t = atomicAdd(&ctr[1], 1u);
-    S.last = (t == gridDim.x - 1);
+    S.last = (atomicAdd(ctr + p.ticket_slot, 1u) == gridDim.x - 1);
   }
   __syncthreads();
   if (!S.last) return;
@@ -211,91 +218,83 @@ topk_select_kernel(TopkParams p) {
 
   int32_t* out_idx = p.out_idx + static_cast<int64_t>(bq) * p.K;
   float* out_sc = p.out_scores ? p.out_scores + static_cast<int64_t>(bq) * p.K : nullptr;
-  int cnt = 0;
+  uint32_t written = 0;
   if (need > 0) {
-    const uint32_t C = __ldcg(&ctr[0]);
-    uint64_t P;
-    if (C <= static_cast<uint32_t>(p.cap)) {
-      const uint64_t* cand = p.cand + static_cast<int64_t>(bq) * p.cap;
-      if (C <= static_cast<uint32_t>(kTopkSmemKeys)) {
-        for (uint32_t i = tid; i < C; i += blockDim.x) keys_s[i] = __ldcg(cand + i);
-        __syncthreads();
-        P = topk_radix_select(S, C, need, [&](int64_t i) { return keys_s[i]; });
-        if (tid == 0) S.cnt = 0;
-        __syncthreads();
-        for (uint32_t i = tid; i < C; i += blockDim.x) {
-          const uint64_t k = keys_s[i];
-          if (k >= P) { const int s = atomicAdd(&S.cnt, 1); if (s < kTopkMaxK) sort_s[s] = k; }
+    // chunk offsets (exclusive scan of the segment lengths)
+    uint32_t C = 0;
+    bool fits = p.nchunks <= kTopkMaxChunks;
+    if (fits) {
+      for (int c0 = 0; c0 < p.nchunks; c0 += kTopkThreads) {
+        const int c = c0 + tid;
+        const uint32_t v = (c < p.nchunks) ? __ldcg(cnt_q + c) : 0;
+        uint32_t tot;
+        const uint32_t o = topk_block_scan(v, S, &tot);
+        if (c < p.nchunks) S.chunk_off[c] = C + o;
+        C += tot;
+      }
+      if (tid == 0) S.chunk_off[p.nchunks] = C;
+      __syncthreads();
+      fits = C <= static_cast<uint32_t>(kTopkSmemKeys);
+    }
+    if (fits) {
+      // gather the segments in chunk order: one warp per chunk
+      const int lane = tid & 31, warp = tid >> 5;
+      for (int c = warp; c < p.nchunks; c += kTopkThreads / 32) {
+        const uint32_t o = S.chunk_off[c], n = S.chunk_off[c + 1] - o;
+        const uint64_t* seg = seg_q + static_cast<int64_t>(c) * kTopkChunk;
+        for (uint32_t i = lane; i < n; i += 32) keys_s[o + i] = __ldcg(seg + i);
+      }
+      __syncthreads();
+      const uint64_t P = topk_radix_select(S, C, need, [&](int64_t i) { return keys_s[i]; });
+      // ordered compaction of the keys >= P (4 consecutive keys per thread)
+      for (uint32_t i0 = 0; i0 < C; i0 += 4 * kTopkThreads) {
+        uint64_t k[4];
+        uint32_t n = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t j = i0 + 4 * tid + i;
+          k[i] = (j < C) ? keys_s[j] : 0;
+          if (k[i] < P) k[i] = 0;
+          n += (k[i] != 0);
         }
-      } else {
-        P = topk_radix_select(S, C, need, [&](int64_t i) { return __ldcg(cand + i); });
-        if (tid == 0) S.cnt = 0;
-        __syncthreads();
-        for (uint32_t i = tid; i < C; i += blockDim.x) {
-          const uint64_t k = __ldcg(cand + i);
-          if (k >= P) { const int s = atomicAdd(&S.cnt, 1); if (s < kTopkMaxK) sort_s[s] = k; }
-        }
+        uint32_t tot;
+        uint32_t o = written + topk_block_scan(n, S, &tot);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (k[i] != 0) topk_emit(p, out_idx, out_sc, o++, k[i]);
+        written += tot;
       }
     } else {
-      // candidate list overflowed: select over the scores themselves
-      P = topk_radix_select(S, nvalid, need, [&](int64_t e) { return topk_slot_key(p, bq, e, tb); });
-      if (tid == 0) S.cnt = 0;
-      __syncthreads();
-      for (int64_t e = tid; e < nvalid; e += blockDim.x) {
-        const uint64_t k = topk_slot_key(p, bq, e, tb);
-        if (k != 0 && k >= P) { const int s = atomicAdd(&S.cnt, 1); if (s < kTopkMaxK) sort_s[s] = k; }
-      }
-    }
-    __syncthreads();
-    cnt = S.cnt;
-    if (cnt != need && tid == 0) record_error(kErrSelectCount);
-    cnt = min(cnt, need);
-    // re-key for ascending-position output
-    if (p.out_by_pos) {
-      for (int i = tid; i < cnt; i += blockDim.x) {
-        const uint64_t k = sort_s[i];
-        const uint32_t pos = ~static_cast<uint32_t>(k);
-        sort_s[i] = (static_cast<uint64_t>(0xFFFFFFFFu - pos) << 32) | (k >> 32);
-      }
-    }
-    int M = 1;
-    while (M < cnt) M <<= 1;
-    for (int i = cnt + tid; i < M; i += blockDim.x) sort_s[i] = 0;
-    __syncthreads();
-    for (int k = 2; k <= M; k <<= 1) {
-      for (int j = k >> 1; j > 0; j >>= 1) {
-        for (int i = tid; i < M; i += blockDim.x) {
-          const int ixj = i ^ j;
-          if (ixj > i) {
-            const uint64_t a = sort_s[i], c = sort_s[ixj];
-            const bool desc = (i & k) == 0;
-            if (desc ? (a < c) : (a > c)) { sort_s[i] = c; sort_s[ixj] = a; }
-          }
+      // candidates do not fit: select and compact over the scores themselves
+      const uint64_t P = topk_radix_select(S, nvalid, need, [&](int64_t e) { return topk_slot_key(p, bq, e, tb); });
+      for (int64_t e0 = 0; e0 < nvalid; e0 += 4 * kTopkThreads) {
+        uint64_t k[4];
+        uint32_t n = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t e = e0 + 4 * tid + i;
+          k[i] = (e < nvalid) ? topk_slot_key(p, bq, e, tb) : 0;
+          if (k[i] < P) k[i] = 0;
+          n += (k[i] != 0);
         }
-        __syncthreads();
+        uint32_t tot;
+        uint32_t o = written + topk_block_scan(n, S, &tot);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (k[i] != 0) topk_emit(p, out_idx, out_sc, o++, k[i]);
+        written += tot;
       }
     }
+    if (written != static_cast<uint32_t>(need) && tid == 0) record_error(kErrSelectCount);
   }
-  for (int i = tid; i < p.K; i += blockDim.x) {
-    int32_t pos = -1;
-    float sc = -INFINITY;
-    if (i < cnt) {
-      const uint64_t k = sort_s[i];
-      if (p.out_by_pos) {
-        pos = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(k >> 32));
-        sc = okey_to_float(static_cast<uint32_t>(k));
-      } else {
-        pos = static_cast<int32_t>(~static_cast<uint32_t>(k));
-        sc = okey_to_float(static_cast<uint32_t>(k >> 32));
-      }
-    }
-    out_idx[i] = pos;
-    if (out_sc) out_sc[i] = sc;
+  for (int i = static_cast<int>(min(written, static_cast<uint32_t>(p.K))) + tid; i < p.K; i += kTopkThreads) {
+    out_idx[i] = -1;
+    if (out_sc) out_sc[i] = -INFINITY;
   }
 }
 
-inline size_t topk_smem_bytes(int hb) {
-  return sizeof(TopkShared) + (static_cast<size_t>(1) << hb) * 4 + (kTopkSmemKeys + kTopkMaxK) * 8;
+inline size_t topk_smem_bytes() {
+  return ((sizeof(TopkShared) + 15) & ~size_t(15)) + static_cast<size_t>(kTopkSmemKeys) * 8;
 }
 
 }  // namespace csa2

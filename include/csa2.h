@@ -115,8 +115,9 @@ csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x,
  * Score of query (b,q) for entry t (t < n_vis[b][q]):
  *     s = sum_h w[b][q][h] * ReLU( sum_d qI[b][q][h][d] * kI[b][t][d] )
  * bf16 products accumulated in fp32 on the tensor cores.  The K best
- * entries by (higher score, then lower position) are written best first,
- * padded with -1 when fewer than K entries are visible.
+ * entries by (higher score, then lower position) are written in ascending
+ * position order, then padded with -1 when fewer than K entries are
+ * visible; `scores` (optional) holds the score of each written entry.
  *
  * mode CSA2_FULL / CSA2_REINDEX: scan t in [0, n_vis).  With hsi_blocks > 0
  *   (FULL only) the call also builds the HSI pool: block score = max of the
@@ -125,7 +126,8 @@ csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x,
  *   padded with -1.
  * mode CSA2_REINDEX_POOL: scan only the positions of pool_in (hsi_blocks
  *   block ids per query, ascending, -1 padding ignored); positions at or
- *   beyond n_vis do not score.
+ *   beyond n_vis do not score.  The selected entries come out in pool order
+ *   (ascending positions for an ascending pool).
  * ---------------------------------------------------------------------- */
 typedef struct csa2_index_args {
     int32_t        mode;        /* CSA2_FULL, CSA2_REINDEX or CSA2_REINDEX_POOL  */

@@ -18,7 +18,8 @@ ATTN_RTOL = 1e-2
 
 
 def check_topk(gpu_idx, scores, K, positions=None, band=TOPK_BAND, exact=False, what=""):
-    """gpu_idx: int array [K] from the CUDA path.  scores: oracle scores of
+    """Set comparison (the order of gpu_idx is not checked here).
+    gpu_idx: int array [K] from the CUDA path.  scores: oracle scores of
     the candidate slots (float64, -inf = not visible).  positions: position
     of each slot (default: slot index).  Returns the GPU's valid indices."""
     gpu_idx = np.asarray(gpu_idx).astype(np.int64)
@@ -38,7 +39,7 @@ def check_topk(gpu_idx, scores, K, positions=None, band=TOPK_BAND, exact=False, 
     order = np.lexsort((p_vis, -s_vis))
     oracle = p_vis[order[:kk]]
     if exact:
-        np.testing.assert_array_equal(sel, oracle, err_msg=f"{what}: exact top-K")
+        np.testing.assert_array_equal(np.sort(sel), np.sort(oracle), err_msg=f"{what}: exact top-K")
         return sel
     sK = s_vis[order[kk - 1]]
     lo, hi = sK - band * abs(sK), sK + band * abs(sK)
