@@ -245,6 +245,16 @@ __device__ __forceinline__ float okey_to_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
+// Shared-memory histogram increment aggregated over the lanes of a warp
+// that hit the same bin (one atomic per distinct bin instead of one per
+// lane); `active` says whether this lane counts.  Warp-collective.
+__device__ __forceinline__ void warp_hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  const uint32_t live = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const uint32_t peers = __match_any_sync(live, bin);
+  if ((threadIdx.x & 31) == static_cast<uint32_t>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

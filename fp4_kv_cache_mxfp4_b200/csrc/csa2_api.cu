@@ -192,9 +192,6 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.nblk = P.nblk;
   sp.hist = reinterpret_cast<uint32_t*>(z + P.off_hist);
   sp.bhist = P.hsi ? reinterpret_cast<uint32_t*>(z + P.off_bhist) : nullptr;
-  sp.ctr = reinterpret_cast<uint32_t*>(z + P.off_ctr);
-  sp.K = a->K;
-  sp.bK = P.hsi ? a->hsi_blocks : 0;
   sp.hb = P.hb;
   sp.groups = P.pool ? P.BQ : a->B;
   sp.tiles_per_group = static_cast<int>((P.n_elems + kTileRows - 1) / kTileRows);
@@ -227,12 +224,12 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   tp.vis_div = 1;
   tp.pool = sp.pool;
   tp.pool_blocks = sp.pool_blocks;
+  tp.hist = sp.hist;
   tp.hb = P.hb;
   tp.seg = reinterpret_cast<uint64_t*>(w + P.off_seg);
   tp.seg_cnt = reinterpret_cast<uint32_t*>(w + P.off_cnt);
   tp.nchunks = P.nchunks;
-  tp.ctr = sp.ctr;
-  tp.tb_slot = 2;
+  tp.ctr = reinterpret_cast<uint32_t*>(z + P.off_ctr);
   tp.ticket_slot = 1;
   tp.K = a->K;
   tp.out_idx = a->idx;
@@ -253,8 +250,8 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
     bp.seg = reinterpret_cast<uint64_t*>(w + P.off_bseg);
     bp.seg_cnt = reinterpret_cast<uint32_t*>(w + P.off_bcnt);
     bp.nchunks = P.bchunks;
-    bp.tb_slot = 4;
-    bp.ticket_slot = 6;
+    bp.hist = sp.bhist;
+    bp.ticket_slot = 2;
     bp.K = a->hsi_blocks;
     bp.out_idx = a->pool_out;
     bp.out_scores = nullptr;

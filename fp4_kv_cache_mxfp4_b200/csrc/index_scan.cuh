@@ -17,8 +17,7 @@
 //               (each set covers the 128 TMEM lanes): TMEM -> scores, the
 //               score histogram used for the top-K threshold and, with HSI,
 //               the block max over 8 positions with its own histogram
-// After the last tile every CTA adds its histograms to the global ones; the
-// last CTA of each group turns them into the threshold bin of each query.
+// After the last tile every CTA adds its histograms to the global ones.
 // Pool mode (Reindex restricted to the HSI pool) gathers the tile as 16
 // blocks of 8 contiguous index-K rows with one 1 KB TMA box per block half.
 //
@@ -54,9 +53,6 @@ struct ScanParams {
   int64_t nblk;
   uint32_t* hist;         // [B*Q][1 << hb]       (zero at launch)
   uint32_t* bhist;        // scan with HSI: [B*Q][1 << hb]
-  uint32_t* ctr;          // [B*Q][8]             (zero at launch): [0] group ticket (first query
-                          // of the group), [2..3] tb, need; [4..5] block tb, need
-  int K, bK;              // top-K of positions and (HSI) of blocks
   int hb;                 // histogram bits
   int groups;             // B (scan) or B*Q (pool)
   int tiles_per_group;
@@ -84,46 +80,6 @@ __host__ __device__ inline ScanSmem scan_smem_layout(int stages, int QG, int hb,
   return L;
 }
 
-// Threshold bin for a top-K from a complete global histogram, run by the 256
-// epilogue threads: tb = highest bin whose suffix count reaches
-// need = min(K, total); writes out[0] = tb (nbins when need == 0) and
-// out[1] = need.  stage: nbins words of shared scratch; red: 8 words.
-__device__ void scan_threshold_bin(const uint32_t* hist, int nbins, int K, uint32_t* out, uint32_t* stage,
-                                   uint32_t* red) {
-  const int et = threadIdx.x - 64, lane = threadIdx.x & 31, ew = et >> 5;
-  // coalesced copy into shared memory, all loads in flight together
-#pragma unroll 8
-  for (int i = et; i < nbins; i += kScanEpiThreads) stage[i] = __ldcg(hist + i);
-  named_bar_sync(1, kScanEpiThreads);
-  const int per = nbins / kScanEpiThreads;
-  const int hi = nbins - 1 - et * per;             // this thread owns bins [hi-per+1, hi]
-  uint32_t local = 0;
-  for (int j = 0; j < per; ++j) local += stage[hi - j];
-  uint32_t incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) red[ew] = incl;
-  named_bar_sync(1, kScanEpiThreads);
-  uint32_t wbase = 0, total = 0;
-  for (int w = 0; w < kScanEpiWarps; ++w) { if (w < ew) wbase += red[w]; total += red[w]; }
-  const uint32_t need = total < static_cast<uint32_t>(K) ? total : static_cast<uint32_t>(K);
-  uint32_t above = wbase + incl - local;
-  if (need > 0 && above < need && above + local >= need) {
-    for (int j = 0; j < per; ++j) {
-      above += stage[hi - j];
-      if (above >= need) { out[0] = hi - j; break; }
-    }
-  }
-  if (et == 0) {
-    out[1] = need;
-    if (need == 0) out[0] = nbins;
-  }
-  named_bar_sync(1, kScanEpiThreads);
-}
-
 template <int QG, bool HSI>
 __global__ void __launch_bounds__(kScanThreads, 1)
 index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -140,7 +96,6 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   uint64_t* q_bar = tempty_bar + kAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* red = tmem_slot + 2;                   // 9 words of scratch
   float* w_s = reinterpret_cast<float*>(smem + L.w0);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L.hist0);
   uint32_t* bhist_s = reinterpret_cast<uint32_t*>(smem + L.bhist0);
@@ -290,20 +245,18 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
         float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         const bool valid = pool_valid && pos < nv[q] && q < p.qg;
         if (!valid) s = -INFINITY;
-        if (e < p.n_elems && q < p.qg) {
-          p.scores[static_cast<int64_t>(bq0 + q) * p.n_elems + e] = s;
-          if (valid) atomicAdd(&hist_s[q * nbins + (okey(s) >> (32 - p.hb))], 1u);
-        }
+        const bool in_range = e < p.n_elems && q < p.qg;
+        if (in_range) p.scores[static_cast<int64_t>(bq0 + q) * p.n_elems + e] = s;
+        warp_hist_add(hist_s + q * nbins, okey(s) >> (32 - p.hb), in_range && valid);
         if (HSI) {
           float m = s;
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
           const int64_t jb = e >> 3;
-          if ((lane & 7) == 0 && jb < p.nblk && q < p.qg) {
-            p.bscores[static_cast<int64_t>(bq0 + q) * p.nblk + jb] = m;
-            if (m != -INFINITY) atomicAdd(&bhist_s[q * nbins + (okey(m) >> (32 - p.hb))], 1u);
-          }
+          const bool writer = (lane & 7) == 0 && jb < p.nblk && q < p.qg;
+          if (writer) p.bscores[static_cast<int64_t>(bq0 + q) * p.nblk + jb] = m;
+          warp_hist_add(bhist_s + q * nbins, okey(m) >> (32 - p.hb), writer && m != -INFINITY);
         }
       }
       tc_fence_before();
@@ -318,22 +271,6 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
       if (HSI) {
         const uint32_t bv = bhist_s[i];
         if (bv) atomicAdd(&p.bhist[static_cast<int64_t>(bq0 + i / nbins) * nbins + (i % nbins)], bv);
-      }
-    }
-    // the last CTA of the group turns the complete histograms into the
-    // threshold bin of each query's top-K (and of its HSI block top-K)
-    __threadfence();
-    named_bar_sync(1, kScanEpiThreads);
-    if (et == 0) red[8] = (atomicAdd(&p.ctr[static_cast<int64_t>(bq0) * 8], 1u) == static_cast<uint32_t>(p.ctas_per_group - 1));
-    named_bar_sync(1, kScanEpiThreads);
-    if (red[8]) {
-      __threadfence();
-      for (int q = 0; q < p.qg; ++q) {
-        scan_threshold_bin(p.hist + static_cast<int64_t>(bq0 + q) * nbins, nbins, p.K,
-                           p.ctr + static_cast<int64_t>(bq0 + q) * 8 + 2, hist_s, red);
-        if (HSI)
-          scan_threshold_bin(p.bhist + static_cast<int64_t>(bq0 + q) * nbins, nbins, p.bK,
-                             p.ctr + static_cast<int64_t>(bq0 + q) * 8 + 4, hist_s, red);
       }
     }
   }

@@ -5,10 +5,11 @@
 // word inverts the position, so every key is distinct and "larger key" means
 // "higher score, then lower position": the top-K set is the K largest keys.
 //
-// The scan kernel has already reduced the score histogram of each query to
-// a threshold bin tb (every top-K key has its top bits >= tb) and the count
-// `need` = min(K, visible).  One launch per selection problem, grid
-// (chunks, queries), 1024 threads:
+// One launch per selection problem, grid (chunks, queries), 1024 threads:
+//  0. every CTA reads the query's score histogram (built by the scan
+//     epilogue, coalesced) and finds the threshold bin tb, the highest bin
+//     whose suffix count reaches need = min(K, visible): every top-K key has
+//     its top bits >= tb;
 //  1. every CTA compacts the keys of its 4096-slot chunk whose bin is >= tb
 //     into the chunk's own segment, in position order (block prefix scan),
 //     and records the segment's length;
@@ -37,13 +38,13 @@ struct TopkParams {
   int vis_div;
   const int32_t* pool;      // pool mode: position of slot e = pool[e/8]*8 + e%8
   int pool_blocks;
+  const uint32_t* hist;     // [BQ][1 << hb] score histogram from the scan
   int hb;
   uint64_t* seg;            // [BQ][n_elems]: chunk c's candidates at c*kTopkChunk
   uint32_t* seg_cnt;        // [BQ][nchunks]
   int nchunks;
-  uint32_t* ctr;            // [BQ][8] (zero at the scan's launch)
-  int tb_slot;              // ctr[tb_slot] = tb, ctr[tb_slot+1] = need (from the scan)
-  int ticket_slot;
+  uint32_t* ctr;            // [BQ][8], zero at the scan's launch
+  int ticket_slot;          // ctr[ticket_slot]: finished CTAs of the query
   int K;
   int32_t* out_idx;         // [BQ][K]
   float* out_scores;        // optional [BQ][K]
@@ -53,7 +54,7 @@ struct TopkShared {
   uint32_t h256[256];
   uint32_t warp_tot[32];
   uint32_t chunk_off[kTopkMaxChunks + 1];
-  int last, d, gt, eq, total;
+  int last, d, gt, eq, total, tb;
 };
 
 __device__ __forceinline__ int64_t topk_valid_slots(const TopkParams& p, int bq) {
@@ -145,11 +146,11 @@ __device__ uint64_t topk_radix_select(TopkShared& S, int64_t n, int need, KeyAt 
     for (int i = threadIdx.x; i < 256; i += blockDim.x) S.h256[i] = 0;
     if (threadIdx.x == 0) S.d = -1;
     __syncthreads();
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint64_t k = key_at(i);
-      if (k == 0) continue;
-      if (bits > 0 && (k >> (64 - bits)) != (prefix >> (64 - bits))) continue;
-      atomicAdd(&S.h256[(k >> shift) & 255], 1u);
+    for (int64_t i0 = 0; i0 < n; i0 += blockDim.x) {
+      const int64_t i = i0 + threadIdx.x;
+      const uint64_t k = (i < n) ? key_at(i) : 0;
+      const bool act = k != 0 && (bits == 0 || (k >> (64 - bits)) == (prefix >> (64 - bits)));
+      warp_hist_add(S.h256, static_cast<uint32_t>((k >> shift) & 255), act);
     }
     __syncthreads();
     if (threadIdx.x < 32) topk_pick_digit(S, remaining);
@@ -180,9 +181,38 @@ topk_select_kernel(TopkParams p) {
   const int bq = blockIdx.y;
   const int tid = threadIdx.x;
   uint32_t* ctr = p.ctr + static_cast<int64_t>(bq) * 8;
-  const int tb = static_cast<int>(__ldcg(ctr + p.tb_slot));
-  const int need = static_cast<int>(__ldcg(ctr + p.tb_slot + 1));
   const int64_t nvalid = topk_valid_slots(p, bq);
+
+  // -- 0. threshold bin: thread t owns the `per` bins just below bin
+  //       nbins - per*t (descending ranges), read with coalesced loads
+  int need;
+  {
+    const int nbins = 1 << p.hb;
+    const int per = nbins / kTopkThreads;             // 4 (12-bit) or 1 (10-bit)
+    const uint32_t* hq = p.hist + static_cast<int64_t>(bq) * nbins;
+    const int lo_bin = nbins - per * (tid + 1);
+    uint32_t c[4] = {0, 0, 0, 0};
+    if (per == 4) {
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin));
+      c[0] = v.x; c[1] = v.y; c[2] = v.z; c[3] = v.w;
+    } else {
+      c[0] = __ldcg(hq + lo_bin);
+    }
+    const uint32_t local = c[0] + c[1] + c[2] + c[3];
+    uint32_t total;
+    uint32_t above = topk_block_scan(local, S, &total);   // bins above this thread's range
+    need = static_cast<int>(total < static_cast<uint32_t>(p.K) ? total : static_cast<uint32_t>(p.K));
+    if (tid == 0) S.tb = nbins;
+    __syncthreads();
+    if (need > 0 && above < static_cast<uint32_t>(need) && above + local >= static_cast<uint32_t>(need)) {
+      for (int j = per - 1; j >= 0; --j) {
+        above += c[j];
+        if (above >= static_cast<uint32_t>(need)) { S.tb = lo_bin + j; break; }
+      }
+    }
+    __syncthreads();
+  }
+  const int tb = S.tb;
   uint64_t* seg_q = p.seg + static_cast<int64_t>(bq) * p.n_elems;
   uint32_t* cnt_q = p.seg_cnt + static_cast<int64_t>(bq) * p.nchunks;
 

@@ -10,7 +10,8 @@ Full layer of the decoder score only the HSI pool), [eogee] §3.4 (new
 entries are quantised after RoPE, before they join the cache).
 
 Readings: Reuse takes the indices of the most recent indexing layer
-([titansim] "核心机制与研究方法": "上一个模式已经筛选完毕的 Top-512");
+([titansim] "核心机制与研究方法" describes Reuse as taking the previous
+layer's already-selected indices);
 REINDEX_POOL uses the pool built by the most recent Full layer.  The layers
 run strictly in order; each layer's inputs are given.
 
