@@ -67,6 +67,7 @@ def load(path=LIB_PATH):
     lib = ctypes.CDLL(path)
     lib.csa2_quantize_kv_fp4.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_p]
     lib.csa2_index_score_topk.argtypes = [ctypes.POINTER(IndexArgs), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexArgs), _c_p]
     lib.csa2_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_group_decode.argtypes = [ctypes.POINTER(GroupArgs), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_workspace_size.argtypes = [_c_p, _c_i32]
@@ -80,7 +81,7 @@ def load(path=LIB_PATH):
     lib.csa2_trace_count.restype = _c_i32
     lib.csa2_kernel_name.argtypes = [_c_i32]
     lib.csa2_kernel_name.restype = ctypes.c_char_p
-    for name in ("csa2_quantize_kv_fp4", "csa2_index_score_topk", "csa2_sparse_attn",
+    for name in ("csa2_quantize_kv_fp4", "csa2_index_score_topk", "csa2_index_score_topk_noalloc", "csa2_sparse_attn",
                  "csa2_group_decode", "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
                  "csa2_trace_end", "csa2_trace_get"):
         getattr(lib, name).restype = _c_i32
@@ -135,6 +136,16 @@ def index_args(mode, qI, w, kI, n_vis, idx, scores=None, hsi_blocks=0, hsi_block
 def csa2_index_score_topk(args, ws, stream=None):
     _check(load().csa2_index_score_topk(ctypes.byref(args), _ptr(ws), ws.numel() * ws.element_size(),
                                         _stream(stream)), "csa2_index_score_topk")
+
+
+def csa2_index_score_topk_noalloc(args, stream=None):
+    """csa2_index_score_topk on the library's fixed scratch array (no
+    workspace argument; for callers that cannot allocate device memory)."""
+    _check(load().csa2_index_score_topk_noalloc(ctypes.byref(args), _stream(stream)),
+           "csa2_index_score_topk_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 def attn_args(q, kv_fp4, idx, swa, out, lse=None, W=128, swa_step=0, scale=0.0):

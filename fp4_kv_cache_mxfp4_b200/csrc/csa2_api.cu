@@ -369,6 +369,31 @@ csa2_status validate_group(const csa2_group_args* g, size_t* index_zero, size_t*
   return CSA2_OK;
 }
 
+// ---------------------------------------------------------------- no-allocation variant
+// Scratch of csa2_index_score_topk_noalloc: one file-scope device array.
+// Every GPU that loads the library holds it until the process exits, and
+// every call of that entry point on a device shares it.  In host code the
+// symbol is only a stand-in: the kernels get the device address that
+// cudaGetSymbolAddress returns for the current device.
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(CSA2_NOALLOC_SCRATCH_BYTES);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_addr[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the first call on each device does it).
+csa2_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CSA2_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return CSA2_OK;
+}
+
 }  // namespace
 }  // namespace csa2
 
@@ -398,6 +423,23 @@ csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws, size_t ws_
   s = device_info(&dev);
   if (s != CSA2_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, P.zero_bytes, st) != cudaSuccess) return CSA2_ERR_CUDA;
+  return run_index(a, *dev, ws, static_cast<uint8_t*>(ws) + P.zero_bytes, st);
+}
+
+csa2_status csa2_index_score_topk_noalloc(const csa2_index_args* a, void* stream) {
+  csa2_status s = validate_index(a);
+  if (s != CSA2_OK) return s;
+  const IndexPlan P = plan_index(a);
+  if (P.total > kNoAllocScratchBytes) return CSA2_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  void* ws = nullptr;
+  s = noalloc_scratch(&ws);
+  if (s != CSA2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: clear the counter region
   if (cudaMemsetAsync(ws, 0, P.zero_bytes, st) != cudaSuccess) return CSA2_ERR_CUDA;
   return run_index(a, *dev, ws, static_cast<uint8_t*>(ws) + P.zero_bytes, st);
 }

@@ -151,6 +151,35 @@ csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws,
                                   size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * csa2_index_score_topk_noalloc -- the same scoring and selection as
+ * csa2_index_score_topk without a caller workspace.  (The pages have no
+ * counterpart: this serves integrations, not the method.)
+ *
+ * For callers that cannot allocate device memory: code that is handed only
+ * its input and output buffers by a host framework and has no allocator of
+ * its own, or a serving process whose memory pool is fully reserved up front
+ * so that a cudaMalloc would fail or stall the device.  The scratch is a
+ * fixed device array of CSA2_NOALLOC_SCRATCH_BYTES inside the library; every
+ * GPU that loads the library holds it until the process exits.  The call
+ * allocates nothing: no cudaMalloc, no cudaFree.
+ *
+ * - The first call on each device looks up the array's device address with
+ *   cudaGetSymbolAddress (with that device current); make that first call
+ *   before any stream capture.
+ * - A request whose scratch would exceed CSA2_NOALLOC_SCRATCH_BYTES
+ *   (csa2_workspace_size(a, CSA2_WS_INDEX) tells the need) returns
+ *   CSA2_ERR_WORKSPACE before anything is enqueued.
+ * - All calls share the one array, which keeps the previous call's data;
+ *   each call clears the part that must start at zero.  Calls that overlap
+ *   on the GPU (different streams, different host threads) race on it and
+ *   give wrong results: serialise them.
+ * Arguments, outputs and the other errors are those of
+ * csa2_index_score_topk.
+ * ---------------------------------------------------------------------- */
+#define CSA2_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+csa2_status csa2_index_score_topk_noalloc(const csa2_index_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
  * csa2_sparse_attn -- [eogee] §3.2 sparse MQA: each query attends to its
  * selected FP4 entries plus the layer's SWA window; §3.4 dequantise before
  * the attention math.
