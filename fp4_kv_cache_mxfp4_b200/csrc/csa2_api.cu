@@ -14,12 +14,14 @@
 #include "index_scan.cuh"
 #include "topk.cuh"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 
 namespace csa2 {
 namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxDynSmem = 227 * 1024;
+constexpr int kScanStages = 3;
 
 struct DeviceInfo {
   bool init = false;
@@ -32,9 +34,18 @@ std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // index_scan_kernel instances: queries per MMA group (1, 2, 4, 8) x HSI
+// Every kernel asks for the full shared-memory carveout, so consecutive
+// kernels of a step never make an SM reconfigure its L1/shared split.
+template <class F>
+cudaError_t set_smem_attrs(F* f, int dyn_bytes) {
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_bytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
 template <int QG, bool HSI>
 cudaError_t set_scan_attr_one() {
-  return cudaFuncSetAttribute(index_scan_kernel<QG, HSI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+  return set_smem_attrs(index_scan_kernel<QG, HSI>, kMaxDynSmem);
 }
 cudaError_t set_scan_attrs() {
   cudaError_t e = cudaSuccess;
@@ -80,9 +91,10 @@ csa2_status device_info(DeviceInfo** out) {
   if (!d.ok) return CSA2_ERR_ARCH;
   if (!d.attrs_set) {
     if (set_scan_attrs() != cudaSuccess ||
-        cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(topk_smem_bytes())) != cudaSuccess ||
-        cudaFuncSetAttribute(sparse_attn_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
+        set_smem_attrs(topk_select_kernel, static_cast<int>(topk_smem_bytes())) != cudaSuccess ||
+        set_smem_attrs(sparse_attn_tc_kernel, static_cast<int>(kTcAttnSmem)) != cudaSuccess ||
+        set_smem_attrs(sparse_attn_combine_kernel, 0) != cudaSuccess ||
+        set_smem_attrs(quantize_kv_fp4_kernel, 0) != cudaSuccess)
       return CSA2_ERR_CUDA;
     if (!g_encode) {
       void* fn = nullptr;
@@ -202,7 +214,9 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   while (cols < scan_acc_bufs(QG) * n_mma) cols <<= 1;
   sp.tmem_cols = cols;
   const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi);
-  sp.stages = std::min(8, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / kStageBytes));
+  // three 32 KB stages per SM measured fastest (fewer bytes in flight per
+  // stream keep DRAM pages open longer; 2, 4 and 6 stages were slower)
+  sp.stages = std::min(kScanStages, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / kStageBytes));
   if (sp.stages < 2) return CSA2_ERR_SHAPE;
   const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi);
 
@@ -277,7 +291,21 @@ csa2_status validate_attn(const csa2_attn_args* a) {
   return CSA2_OK;
 }
 
-inline int attn_slices(const csa2_attn_args* a) { return (a->K + a->W + kAttnKeys - 1) / kAttnKeys; }
+inline int attn_kv_slices(const csa2_attn_args* a) { return (a->K + kTcAttnKeys - 1) / kTcAttnKeys; }
+inline int attn_slices(const csa2_attn_args* a) {
+  return attn_kv_slices(a) + (a->W + kTcAttnKeys - 1) / kTcAttnKeys;
+}
+
+// bf16 [rows][512] matrix as a 2-D TMA map with 128-byte swizzle, box 64 x box_rows
+bool make_map_bf16_512(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {512, rows};
+  const cuuint64_t strides[1] = {1024};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 size_t attn_ws_bytes(const csa2_attn_args* a) {
   const size_t bq = static_cast<size_t>(a->B) * a->Q, s = attn_slices(a);
@@ -285,25 +313,42 @@ size_t attn_ws_bytes(const csa2_attn_args* a) {
 }
 
 csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
-  AttnParams p;
-  p.B = a->B; p.Q = a->Q; p.K = a->K; p.W = a->W; p.N = a->N;
-  p.q = static_cast<const __nv_bfloat16*>(a->q);
-  p.kv = static_cast<const uint8_t*>(a->kv_fp4);
-  p.idx = a->idx;
-  p.swa = static_cast<const __nv_bfloat16*>(a->swa);
-  p.swa_rows = a->swa_rows; p.swa_step = a->swa_step;
   const float scale = a->scale > 0.0f ? a->scale : 1.0f / sqrtf(512.0f);
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.slices = attn_slices(a);
   const size_t bq = static_cast<size_t>(a->B) * a->Q;
-  p.opart = static_cast<float*>(ws);
-  p.ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + up256(bq * p.slices * 64 * 512 * 4));
-  p.out = static_cast<__nv_bfloat16*>(a->out);
-  p.lse = a->lse;
+  const int slices = attn_slices(a);
+  float* opart = static_cast<float*>(ws);
+  float* ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + up256(bq * slices * 64 * 512 * 4));
+
+  TcAttnParams t;
+  t.B = a->B; t.Q = a->Q; t.K = a->K; t.W = a->W; t.N = a->N;
+  t.kv = static_cast<const uint8_t*>(a->kv_fp4);
+  t.idx = a->idx;
+  t.swa_rows = a->swa_rows; t.swa_step = a->swa_step;
+  t.kv_slices = attn_kv_slices(a);
+  t.slices = slices;
+  t.scale_log2 = scale * 1.4426950408889634f;
+  t.opart = opart;
+  t.ml = ml;
+  CUtensorMap tq, tw;
+  if (!make_map_bf16_512(&tq, a->q, bq * 64, 64)) return CSA2_ERR_CUDA;
+  if (a->W > 0) {
+    if (!make_map_bf16_512(&tw, a->swa, static_cast<uint64_t>(a->B) * a->swa_rows, kTcAttnKeys)) return CSA2_ERR_CUDA;
+  } else {
+    tw = tq;                                    // no window slices: never used
+  }
   trace_pre(kKAttnSlice, st);
-  sparse_attn_slice_kernel<<<dim3(p.slices, static_cast<unsigned>(bq)), kAttnThreads, kAttnSmem, st>>>(p);
+  sparse_attn_tc_kernel<<<dim3(slices, static_cast<unsigned>(bq)), kTcAttnThreads, kTcAttnSmem, st>>>(tq, tw, t);
   trace_post(st);
   if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+
+  AttnParams p;
+  memset(&p, 0, sizeof(p));
+  p.B = a->B; p.Q = a->Q; p.K = a->K; p.W = a->W; p.N = a->N;
+  p.slices = slices;
+  p.opart = opart;
+  p.ml = ml;
+  p.out = static_cast<__nv_bfloat16*>(a->out);
+  p.lse = a->lse;
   trace_pre(kKAttnCombine, st);
   sparse_attn_combine_kernel<<<static_cast<unsigned>(bq * 64), 128, 0, st>>>(p);
   trace_post(st);
@@ -589,7 +634,7 @@ const char* csa2_kernel_name(int32_t kernel) {
     case kKQuantize: return "quantize_kv_fp4_kernel";
     case kKIndexScan: return "index_scan_kernel";
     case kKTopk: return "topk_select_kernel";
-    case kKAttnSlice: return "sparse_attn_slice_kernel";
+    case kKAttnSlice: return "sparse_attn_tc_kernel";
     case kKAttnCombine: return "sparse_attn_combine_kernel";
     default: return "unknown";
   }

@@ -5,7 +5,7 @@
 // word inverts the position, so every key is distinct and "larger key" means
 // "higher score, then lower position": the top-K set is the K largest keys.
 //
-// One launch per selection problem, grid (chunks, queries), 1024 threads:
+// One launch per selection problem, grid (chunks, queries), 256 threads:
 //  0. every CTA reads the query's score histogram (built by the scan
 //     epilogue, coalesced) and finds the threshold bin tb, the highest bin
 //     whose suffix count reaches need = min(K, visible): every top-K key has
@@ -26,8 +26,9 @@
 
 namespace csa2 {
 
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkChunk = 4096;          // slots per CTA (4 per thread)
+constexpr int kTopkThreads = 256;
+constexpr int kTopkPer = 16;              // slots per thread
+constexpr int kTopkChunk = kTopkThreads * kTopkPer;   // 4096 slots per CTA
 constexpr int kTopkSmemKeys = 6144;       // candidates cached in shared memory
 constexpr int kTopkMaxChunks = 2048;      // chunk offsets kept in shared memory
 
@@ -69,6 +70,15 @@ __device__ __forceinline__ uint32_t topk_position(const TopkParams& p, int bq, i
   return static_cast<uint32_t>(blk * 8 + static_cast<int>(e & 7));
 }
 
+// key of score s at slot e, or 0 when the slot holds no visible score or
+// sits below tb
+__device__ __forceinline__ uint64_t topk_key_of(const TopkParams& p, int bq, int64_t e, float s, int tb) {
+  if (s == -INFINITY) return 0;
+  const uint32_t k = okey(s);
+  if (static_cast<int>(k >> (32 - p.hb)) < tb) return 0;
+  return (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(~topk_position(p, bq, e));
+}
+
 // key of slot e, or 0 when the slot holds no visible score or sits below tb
 __device__ __forceinline__ uint64_t topk_slot_key(const TopkParams& p, int bq, int64_t e, int tb) {
   const float s = p.scores[static_cast<int64_t>(bq) * p.n_elems + e];
@@ -78,8 +88,8 @@ __device__ __forceinline__ uint64_t topk_slot_key(const TopkParams& p, int bq, i
   return (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(~topk_position(p, bq, e));
 }
 
-// Exclusive prefix sum over the block (1024 threads); *total gets the sum.
-// Ends with a barrier so the scratch can be reused.
+// Exclusive prefix sum over the block; *total gets the sum.  Ends with a
+// barrier so the scratch can be reused.
 __device__ __forceinline__ uint32_t topk_block_scan(uint32_t v, TopkShared& S, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
@@ -91,7 +101,7 @@ __device__ __forceinline__ uint32_t topk_block_scan(uint32_t v, TopkShared& S, u
   if (lane == 31) S.warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t x = S.warp_tot[lane];
+    const uint32_t x = (lane < kTopkThreads / 32) ? S.warp_tot[lane] : 0;
     uint32_t xi = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -183,31 +193,45 @@ topk_select_kernel(TopkParams p) {
   uint32_t* ctr = p.ctr + static_cast<int64_t>(bq) * 8;
   const int64_t nvalid = topk_valid_slots(p, bq);
 
+  // this thread's 16 slots of the chunk, loaded before the histogram so the
+  // two reads overlap
+  const int64_t slot0 = static_cast<int64_t>(blockIdx.x) * kTopkChunk + kTopkPer * tid;
+  float sv[kTopkPer];
+#pragma unroll
+  for (int i = 0; i < kTopkPer; ++i)
+    sv[i] = (slot0 + i < nvalid) ? p.scores[static_cast<int64_t>(bq) * p.n_elems + slot0 + i] : -INFINITY;
+
   // -- 0. threshold bin: thread t owns the `per` bins just below bin
   //       nbins - per*t (descending ranges), read with coalesced loads
   int need;
   {
     const int nbins = 1 << p.hb;
-    const int per = nbins / kTopkThreads;             // 4 (12-bit) or 1 (10-bit)
+    const int per = nbins / kTopkThreads;             // 16 (12-bit) or 4 (10-bit)
     const uint32_t* hq = p.hist + static_cast<int64_t>(bq) * nbins;
     const int lo_bin = nbins - per * (tid + 1);
-    uint32_t c[4] = {0, 0, 0, 0};
-    if (per == 4) {
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin));
-      c[0] = v.x; c[1] = v.y; c[2] = v.z; c[3] = v.w;
-    } else {
-      c[0] = __ldcg(hq + lo_bin);
+    uint32_t c[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (4 * j < per) v = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin) + j);
+      c[4 * j] = v.x; c[4 * j + 1] = v.y; c[4 * j + 2] = v.z; c[4 * j + 3] = v.w;
     }
-    const uint32_t local = c[0] + c[1] + c[2] + c[3];
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) local += c[j];
     uint32_t total;
     uint32_t above = topk_block_scan(local, S, &total);   // bins above this thread's range
     need = static_cast<int>(total < static_cast<uint32_t>(p.K) ? total : static_cast<uint32_t>(p.K));
     if (tid == 0) S.tb = nbins;
     __syncthreads();
     if (need > 0 && above < static_cast<uint32_t>(need) && above + local >= static_cast<uint32_t>(need)) {
-      for (int j = per - 1; j >= 0; --j) {
-        above += c[j];
-        if (above >= static_cast<uint32_t>(need)) { S.tb = lo_bin + j; break; }
+      bool found = false;
+#pragma unroll
+      for (int j = 15; j >= 0; --j) {
+        if (j < per && !found) {
+          above += c[j];
+          if (above >= static_cast<uint32_t>(need)) { S.tb = lo_bin + j; found = true; }
+        }
       }
     }
     __syncthreads();
@@ -218,22 +242,21 @@ topk_select_kernel(TopkParams p) {
 
   // -- 1. this chunk's candidates, in position order ------------------------
   {
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * kTopkChunk;
-    uint64_t k[4];
+    uint64_t k[kTopkPer];
     uint32_t n = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t e = base + 4 * tid + i;
-      k[i] = (need > 0 && e < nvalid) ? topk_slot_key(p, bq, e, tb) : 0;
+    for (int i = 0; i < kTopkPer; ++i) {
+      k[i] = (need > 0) ? topk_key_of(p, bq, slot0 + i, sv[i], tb) : 0;
       n += (k[i] != 0);
     }
     uint32_t total;
     uint32_t off = topk_block_scan(n, S, &total);
-    uint64_t* seg = seg_q + base;
+    uint64_t* seg = seg_q + static_cast<int64_t>(blockIdx.x) * kTopkChunk;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kTopkPer; ++i)
       if (k[i] != 0) seg[off++] = k[i];
     if (tid == 0) cnt_q[blockIdx.x] = total;
+    __threadfence();                                      // publish this thread's writes before the ticket
   }
 
   // -- 2. the last CTA of this query selects ---------------------------------
