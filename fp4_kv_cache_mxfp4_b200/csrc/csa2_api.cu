@@ -342,8 +342,6 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
   if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
 
   AttnParams p;
-  memset(&p, 0, sizeof(p));
-  p.B = a->B; p.Q = a->Q; p.K = a->K; p.W = a->W; p.N = a->N;
   p.slices = slices;
   p.opart = opart;
   p.ml = ml;
