@@ -139,7 +139,9 @@ struct IndexPlan {
 csa2_status validate_index(const csa2_index_args* a) {
   if (!a) return CSA2_ERR_ARG;
   if (a->mode != CSA2_FULL && a->mode != CSA2_REINDEX && a->mode != CSA2_REINDEX_POOL) return CSA2_ERR_ARG;
-  if (a->B < 1 || a->Q < 1 || a->Q > CSA2_MAX_Q || a->K < 1 || a->K > CSA2_MAX_K || a->N < 1) return CSA2_ERR_SHAPE;
+  if (a->B < 1 || a->Q < 1 || static_cast<int64_t>(a->B) * a->Q > CSA2_MAX_BQ || a->K < 1 || a->K > CSA2_MAX_K ||
+      a->N < 1)
+    return CSA2_ERR_SHAPE;
   if (static_cast<int64_t>(a->B) * a->N >= (static_cast<int64_t>(1) << 31)) return CSA2_ERR_SHAPE;
   if (!a->qI || !a->w || !a->kI || !a->n_vis || !a->idx) return CSA2_ERR_ARG;
   const bool hsi = a->mode == CSA2_FULL && a->hsi_blocks > 0;
@@ -162,7 +164,7 @@ IndexPlan plan_index(const csa2_index_args* a) {
   P.pool = a->mode == CSA2_REINDEX_POOL;
   P.hsi = a->mode == CSA2_FULL && a->hsi_blocks > 0;
   P.BQ = a->B * a->Q;
-  P.qg = P.pool ? 1 : a->Q;
+  P.qg = P.pool ? 1 : std::min(a->Q, 8);
   P.hb = (P.qg <= 2) ? 12 : 10;
   P.n_elems = P.pool ? static_cast<int64_t>(a->hsi_blocks) * 8 : a->N;
   P.nblk = P.hsi ? (a->N + 7) / 8 : 0;
@@ -177,8 +179,8 @@ IndexPlan plan_index(const csa2_index_args* a) {
   off = 0;
   P.off_scores = off;  off = up256(off + static_cast<size_t>(P.BQ) * P.n_elems * 4);
   P.off_bscores = off; off = up256(off + static_cast<size_t>(P.BQ) * P.nblk * 4);
-  P.off_seg = off;     off = up256(off + static_cast<size_t>(P.BQ) * P.n_elems * 8);
-  P.off_bseg = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.nblk * 8);
+  P.off_seg = off;     off = up256(off + static_cast<size_t>(P.BQ) * P.nchunks * kTopkSegCap * 8);
+  P.off_bseg = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.bchunks * kTopkSegCap * 8);
   P.off_cnt = off;     off = up256(off + static_cast<size_t>(P.BQ) * P.nchunks * 4);
   P.off_bcnt = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.bchunks * 4);
   P.data_bytes = off;
@@ -205,7 +207,8 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.hist = reinterpret_cast<uint32_t*>(z + P.off_hist);
   sp.bhist = P.hsi ? reinterpret_cast<uint32_t*>(z + P.off_bhist) : nullptr;
   sp.hb = P.hb;
-  sp.groups = P.pool ? P.BQ : a->B;
+  sp.qblocks = P.pool ? 1 : (a->Q + P.qg - 1) / P.qg;
+  sp.groups = P.pool ? P.BQ : a->B * sp.qblocks;
   sp.tiles_per_group = static_cast<int>((P.n_elems + kTileRows - 1) / kTileRows);
   sp.ctas_per_group = std::max(1, std::min(sp.tiles_per_group, dev.sms / sp.groups));
   const int QG = scan_qg(P.qg);
@@ -245,6 +248,7 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   tp.nchunks = P.nchunks;
   tp.ctr = reinterpret_cast<uint32_t*>(z + P.off_ctr);
   tp.ticket_slot = 1;
+  tp.ovf_slot = 3;
   tp.K = a->K;
   tp.out_idx = a->idx;
   tp.out_scores = a->scores;
@@ -266,6 +270,7 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
     bp.nchunks = P.bchunks;
     bp.hist = sp.bhist;
     bp.ticket_slot = 2;
+    bp.ovf_slot = 4;
     bp.K = a->hsi_blocks;
     bp.out_idx = a->pool_out;
     bp.out_scores = nullptr;
@@ -280,7 +285,8 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
 // ---------------------------------------------------------------- attention call
 csa2_status validate_attn(const csa2_attn_args* a) {
   if (!a) return CSA2_ERR_ARG;
-  if (a->B < 1 || a->Q < 1 || a->Q > CSA2_MAX_Q || a->K < 0 || a->K > CSA2_MAX_K || a->W < 0 || a->W > CSA2_MAX_W ||
+  if (a->B < 1 || a->Q < 1 || static_cast<int64_t>(a->B) * a->Q > CSA2_MAX_BQ || a->K < 0 || a->K > CSA2_MAX_K ||
+      a->W < 0 || a->W > CSA2_MAX_W ||
       a->K + a->W < 1 || a->N < 1 || a->swa_step < 0)
     return CSA2_ERR_SHAPE;
   if (!a->q || !a->out || (a->K > 0 && (!a->kv_fp4 || !a->idx)) || (a->W > 0 && !a->swa)) return CSA2_ERR_ARG;

@@ -41,7 +41,8 @@ __host__ __device__ constexpr int scan_acc_bufs(int QG) { return 32 * QG * 4 <= 
 struct ScanParams {
   int pool_mode;          // 0: scan [0, n_vis) of each row; 1: scan the pool of each (b,q)
   int B, Q;               // batch rows, queries per row
-  int qg;                 // queries of an MMA group: Q (scan) or 1 (pool); <= the QG template
+  int qg;                 // queries per MMA group: min(Q, QG) (scan) or 1 (pool)
+  int qblocks;            // scan: query blocks per batch row, ceil(Q / qg)
   int64_t N;              // index-K rows per batch row
   int64_t n_elems;        // score slots per query: N (scan) or pool_blocks*8 (pool)
   const int32_t* n_vis;   // [B*Q]
@@ -54,7 +55,7 @@ struct ScanParams {
   uint32_t* hist;         // [B*Q][1 << hb]       (zero at launch)
   uint32_t* bhist;        // scan with HSI: [B*Q][1 << hb]
   int hb;                 // histogram bits
-  int groups;             // B (scan) or B*Q (pool)
+  int groups;             // B*qblocks (scan) or B*Q (pool)
   int tiles_per_group;
   int ctas_per_group;
   int stages;
@@ -104,9 +105,10 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int group = blockIdx.x / p.ctas_per_group;
   const int cig = blockIdx.x % p.ctas_per_group;
   // batch row and first query of this MMA group
-  const int b = p.pool_mode ? group / p.Q : group;
-  const int q0 = p.pool_mode ? group % p.Q : 0;
+  const int b = p.pool_mode ? group / p.Q : group / p.qblocks;
+  const int q0 = p.pool_mode ? group % p.Q : (group % p.qblocks) * p.qg;
   const int bq0 = b * p.Q + q0;              // first (b,q) of the group
+  const int qn = p.pool_mode ? 1 : min(p.qg, p.Q - q0);   // queries of this group
   const int nbins = 1 << p.hb;
 
   // this CTA's tile range; in scan mode, tiles past every query's n_vis are skipped
@@ -114,7 +116,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   int tile_hi = static_cast<int>((static_cast<int64_t>(cig + 1) * p.tiles_per_group) / p.ctas_per_group);
   int nv[QG];
 #pragma unroll
-  for (int q = 0; q < QG; ++q) nv[q] = (q < p.qg) ? p.n_vis[bq0 + q] : 0;
+  for (int q = 0; q < QG; ++q) nv[q] = (q < qn) ? p.n_vis[bq0 + q] : 0;
   if (!p.pool_mode) {
     int nmax = 0;
 #pragma unroll
@@ -134,7 +136,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   if (warp == 1) { tmem_alloc(tmem_slot, p.tmem_cols); tmem_relinquish(); }
   for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) hist_s[i] = 0;
   if (HSI) for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) bhist_s[i] = 0;
-  for (int i = threadIdx.x; i < QG * 32; i += blockDim.x) w_s[i] = (i < p.qg * 32) ? p.w[bq0 * 32 + i] : 0.0f;
+  for (int i = threadIdx.x; i < QG * 32; i += blockDim.x) w_s[i] = (i < qn * 32) ? p.w[bq0 * 32 + i] : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -243,9 +245,9 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
           acc[h & 3] = fmaf(wh, fmaxf(__uint_as_float(r[h]), 0.0f), acc[h & 3]);
         }
         float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        const bool valid = pool_valid && pos < nv[q] && q < p.qg;
+        const bool valid = pool_valid && pos < nv[q] && q < qn;
         if (!valid) s = -INFINITY;
-        const bool in_range = e < p.n_elems && q < p.qg;
+        const bool in_range = e < p.n_elems && q < qn;
         if (in_range) p.scores[static_cast<int64_t>(bq0 + q) * p.n_elems + e] = s;
         warp_hist_add(hist_s + q * nbins, okey(s) >> (32 - p.hb), in_range && valid);
         if (HSI) {
@@ -254,7 +256,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
           const int64_t jb = e >> 3;
-          const bool writer = (lane & 7) == 0 && jb < p.nblk && q < p.qg;
+          const bool writer = (lane & 7) == 0 && jb < p.nblk && q < qn;
           if (writer) p.bscores[static_cast<int64_t>(bq0 + q) * p.nblk + jb] = m;
           warp_hist_add(bhist_s + q * nbins, okey(m) >> (32 - p.hb), writer && m != -INFINITY);
         }
@@ -265,7 +267,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // flush the CTA's histograms into the global ones
     named_bar_sync(1, kScanEpiThreads);
     const int et = threadIdx.x - 64;
-    for (int i = et; i < p.qg * nbins; i += kScanEpiThreads) {
+    for (int i = et; i < qn * nbins; i += kScanEpiThreads) {
       const uint32_t v = hist_s[i];
       if (v) atomicAdd(&p.hist[static_cast<int64_t>(bq0 + i / nbins) * nbins + (i % nbins)], v);
       if (HSI) {

@@ -29,6 +29,7 @@ namespace csa2 {
 constexpr int kTopkThreads = 256;
 constexpr int kTopkPer = 16;              // slots per thread
 constexpr int kTopkChunk = kTopkThreads * kTopkPer;   // 4096 slots per CTA
+constexpr int kTopkSegCap = 1024;         // candidates kept per chunk (more: exact fallback)
 constexpr int kTopkSmemKeys = 6144;       // candidates cached in shared memory
 constexpr int kTopkMaxChunks = 2048;      // chunk offsets kept in shared memory
 
@@ -41,11 +42,12 @@ struct TopkParams {
   int pool_blocks;
   const uint32_t* hist;     // [BQ][1 << hb] score histogram from the scan
   int hb;
-  uint64_t* seg;            // [BQ][n_elems]: chunk c's candidates at c*kTopkChunk
+  uint64_t* seg;            // [BQ][nchunks][kTopkSegCap]: chunk c's candidates
   uint32_t* seg_cnt;        // [BQ][nchunks]
   int nchunks;
   uint32_t* ctr;            // [BQ][8], zero at the scan's launch
   int ticket_slot;          // ctr[ticket_slot]: finished CTAs of the query
+  int ovf_slot;             // ctr[ovf_slot] != 0: a chunk had more than kTopkSegCap candidates
   int K;
   int32_t* out_idx;         // [BQ][K]
   float* out_scores;        // optional [BQ][K]
@@ -237,7 +239,7 @@ topk_select_kernel(TopkParams p) {
     __syncthreads();
   }
   const int tb = S.tb;
-  uint64_t* seg_q = p.seg + static_cast<int64_t>(bq) * p.n_elems;
+  uint64_t* seg_q = p.seg + static_cast<int64_t>(bq) * p.nchunks * kTopkSegCap;
   uint32_t* cnt_q = p.seg_cnt + static_cast<int64_t>(bq) * p.nchunks;
 
   // -- 1. this chunk's candidates, in position order ------------------------
@@ -251,11 +253,16 @@ topk_select_kernel(TopkParams p) {
     }
     uint32_t total;
     uint32_t off = topk_block_scan(n, S, &total);
-    uint64_t* seg = seg_q + static_cast<int64_t>(blockIdx.x) * kTopkChunk;
+    uint64_t* seg = seg_q + static_cast<int64_t>(blockIdx.x) * kTopkSegCap;
 #pragma unroll
-    for (int i = 0; i < kTopkPer; ++i)
-      if (k[i] != 0) seg[off++] = k[i];
-    if (tid == 0) cnt_q[blockIdx.x] = total;
+    for (int i = 0; i < kTopkPer; ++i) {
+      if (k[i] != 0 && off < static_cast<uint32_t>(kTopkSegCap)) seg[off] = k[i];
+      off += (k[i] != 0);
+    }
+    if (tid == 0) {
+      cnt_q[blockIdx.x] = min(total, static_cast<uint32_t>(kTopkSegCap));
+      if (total > static_cast<uint32_t>(kTopkSegCap)) atomicOr(ctr + p.ovf_slot, 1u);
+    }
     __threadfence();                                      // publish this thread's writes before the ticket
   }
 
@@ -275,7 +282,7 @@ topk_select_kernel(TopkParams p) {
   if (need > 0) {
     // chunk offsets (exclusive scan of the segment lengths)
     uint32_t C = 0;
-    bool fits = p.nchunks <= kTopkMaxChunks;
+    bool fits = p.nchunks <= kTopkMaxChunks && __ldcg(ctr + p.ovf_slot) == 0;
     if (fits) {
       for (int c0 = 0; c0 < p.nchunks; c0 += kTopkThreads) {
         const int c = c0 + tid;
@@ -294,7 +301,7 @@ topk_select_kernel(TopkParams p) {
       const int lane = tid & 31, warp = tid >> 5;
       for (int c = warp; c < p.nchunks; c += kTopkThreads / 32) {
         const uint32_t o = S.chunk_off[c], n = S.chunk_off[c + 1] - o;
-        const uint64_t* seg = seg_q + static_cast<int64_t>(c) * kTopkChunk;
+        const uint64_t* seg = seg_q + static_cast<int64_t>(c) * kTopkSegCap;
         for (uint32_t i = lane; i < n; i += 32) keys_s[o + i] = __ldcg(seg + i);
       }
       __syncthreads();

@@ -58,7 +58,7 @@ extern "C" {
 #define CSA2_HSI_BLOCKS   2048  /* HSI blocks kept                            */
 
 /* Limits of this implementation. */
-#define CSA2_MAX_Q        8     /* query positions per batch row per call     */
+#define CSA2_MAX_BQ       65535 /* batch rows x query positions per call      */
 #define CSA2_MAX_K        2048  /* largest top-K (and largest pool, in blocks) */
 #define CSA2_MAX_W        1024  /* largest window (rows per query)            */
 
@@ -132,7 +132,7 @@ csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x,
 typedef struct csa2_index_args {
     int32_t        mode;        /* CSA2_FULL, CSA2_REINDEX or CSA2_REINDEX_POOL  */
     int32_t        B;           /* batch rows, >= 1                              */
-    int32_t        Q;           /* query positions per row, 1..CSA2_MAX_Q        */
+    int32_t        Q;           /* query positions per row, B*Q <= CSA2_MAX_BQ   */
     int32_t        K;           /* top-K, 1..CSA2_MAX_K                          */
     int64_t        N;           /* index-K rows per batch row, >= 1              */
     const void*    qI;          /* bf16 [B][Q][32][128]                          */
@@ -196,7 +196,7 @@ csa2_status csa2_index_score_topk_noalloc(const csa2_index_args* a, void* stream
  * [0, swa_rows).
  * ---------------------------------------------------------------------- */
 typedef struct csa2_attn_args {
-    int32_t        B, Q;        /* batch rows >= 1; queries per row 1..CSA2_MAX_Q */
+    int32_t        B, Q;        /* batch rows >= 1; queries per row, B*Q <= CSA2_MAX_BQ */
     int32_t        K;           /* idx slots per query, 0..CSA2_MAX_K            */
     int32_t        W;           /* window rows per query, 0..CSA2_MAX_W          */
     int64_t        N;           /* cache rows per batch row                      */

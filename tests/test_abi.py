@@ -104,7 +104,7 @@ def _call_attn(L, a, ws=FAKE, ws_bytes=0):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(mode=3), 1), (dict(mode=7), 1), (dict(qI=None), 1), (dict(n_vis=None), 1), (dict(idx=None), 1),
-    (dict(B=0), 2), (dict(Q=0), 2), (dict(Q=9), 2), (dict(K=0), 2), (dict(K=2049), 2), (dict(N=0), 2),
+    (dict(B=0), 2), (dict(Q=0), 2), (dict(B=2, Q=40000), 2), (dict(K=0), 2), (dict(K=2049), 2), (dict(N=0), 2),
     (dict(N=2 ** 31), 2), (dict(hsi_blocks=-1), 2), (dict(hsi_blocks=2048, hsi_block=16, pool_out=FAKE), 2),
     (dict(hsi_blocks=2048, pool_out=None), 1), (dict(mode=2, hsi_blocks=2048, pool_in=None), 1),
     (dict(qI=FAKE + 8), 3), (dict(kI=FAKE + 4), 3), (dict(scores=FAKE + 2), 3),
@@ -120,7 +120,7 @@ def test_index_validation_null_struct(L):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(q=None), 1), (dict(out=None), 1), (dict(idx=None), 1), (dict(swa=None), 1),
-    (dict(B=0), 2), (dict(Q=9), 2), (dict(K=-1), 2), (dict(K=0, W=0), 2), (dict(W=1025), 2),
+    (dict(B=0), 2), (dict(B=3, Q=30000), 2), (dict(K=-1), 2), (dict(K=0, W=0), 2), (dict(W=1025), 2),
     (dict(swa_rows=100), 2), (dict(Q=2, swa_step=1, swa_rows=128), 2),
     (dict(out=FAKE + 8), 3), (dict(lse=FAKE + 4), 3),
     (dict(), 4),

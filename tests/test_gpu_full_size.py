@@ -1,0 +1,98 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+bench times (one csa2_group_decode call over a workload staged by
+fp4_kv_cache_mxfp4_b200.device_workload), checked on sampled outputs the
+oracle computes one by one:
+
+* FP4 bytes of every new entry and of sampled older entries: bit-exact;
+* per indexing layer and sampled (row, query): the top-K under the band
+  rule (and the HSI block pool, when the schedule has one);
+* per layer and sampled (row, query): the attention output and its
+  log-sum-exp against the float64 oracle on the GPU's (validated) indices.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from fp4_kv_cache_mxfp4_b200 import csa2, workloads
+from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload
+from oracle import attention, fp4, indexer
+from parity import check_attention, check_topk, f32
+
+pytestmark = pytest.mark.gpu
+
+
+def _samples(wl):
+    """(b, q) pairs checked against the oracle."""
+    if wl.Q == 1:
+        return [(b, 0) for b in range(wl.B)]
+    rng = np.random.default_rng(wl.seed)
+    qs = sorted({0, 1, 7, 8, wl.Q // 2 - 1, wl.Q - 2, wl.Q - 1, *rng.integers(0, wl.Q, 3).tolist()})
+    return [(b, q) for b in range(wl.B) for q in qs]
+
+
+def _attn_oracle(kv_host_b, sel, q, win):
+    """Attention over the selected entries without dequantising the whole
+    cache: the selected rows are dequantised into a compact array."""
+    valid = sel[sel >= 0]
+    deq = fp4.dequantize_kv_fp4(kv_host_b[valid])
+    local = np.full(sel.shape, -1, dtype=np.int64)
+    local[sel >= 0] = np.arange(valid.shape[0])
+    return attention.sparse_mqa(q, deq, local, win)
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 4], ids=lambda w: workloads.WORKLOADS[w].name)
+def test_full_size_sampled(w):
+    wl = workloads.WORKLOADS[w]
+    csa2.load()
+    T = make_device_workload(wl, csa2)
+    csa2.csa2_group_decode(T["g"], T["ws"])
+    torch.cuda.synchronize()
+    assert csa2.csa2_device_status() == (0, 0)
+    B, N = wl.B, wl.N
+    rng = np.random.default_rng(100 + w)
+
+    # FP4 bytes: every new entry, and 64 sampled older ones per row
+    for b in range(B):
+        new_host = T["kv"][b, N - wl.n_new:].cpu().numpy()
+        want = fp4.quantize_kv_fp4(f32(workloads.main_kv_rows(wl, b, N - wl.n_new, wl.n_new)))
+        np.testing.assert_array_equal(new_host, want, err_msg=f"new entries of row {b}")
+        for r in rng.integers(0, N - wl.n_new, 64).tolist():
+            got = T["kv"][b, r].cpu().numpy()
+            np.testing.assert_array_equal(got, fp4.quantize_kv_fp4(f32(workloads.main_kv_rows(wl, b, r, 1)))[0],
+                                          err_msg=f"entry {r} of row {b}")
+
+    samples = _samples(wl)
+    kv_host = {b: T["kv"][b].cpu().numpy() for b in range(B)}
+    n_vis = np.asarray(wl.n_vis)
+    pool = T["pool"].cpu().numpy() if T["pool"] is not None else None
+    last_idx = None
+    for l, mode in enumerate(wl.modes):
+        li = workloads.layer_inputs(wl, l)
+        L = T["layers"][l]
+        if mode != workloads.REUSE:
+            last_idx = L["idx"].cpu().numpy()
+        for b in range(B):
+            kI = f32(workloads.index_k(wl, b)) if mode != workloads.REUSE else None
+            for (bb, q) in samples:
+                if bb != b:
+                    continue
+                what = f"{wl.name} layer {l} b{b} q{q}"
+                nv = int(n_vis[q])
+                if mode in (workloads.FULL, workloads.REINDEX):
+                    s = indexer.index_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, nv)
+                    check_topk(last_idx[b, q], s, wl.K, what=what)
+                    if mode == workloads.FULL and wl.hsi_blocks:
+                        bs = indexer.block_scores(s, 8)
+                        gp = pool[b, q]
+                        v = gp[gp >= 0]
+                        assert np.all(np.diff(v) > 0), f"{what}: pool not ascending"
+                        check_topk(np.concatenate([v[np.argsort(-bs[v], kind="stable")], gp[gp < 0]]), bs,
+                                   wl.hsi_blocks, what=what + " pool")
+                elif mode == workloads.REINDEX_POOL:
+                    pos, ps = indexer.pool_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, pool[b, q], nv)
+                    check_topk(last_idx[b, q], ps, wl.K, positions=pos, what=what)
+                win = f32(li["swa"][b])[q * wl.swa_step: q * wl.swa_step + wl.W]
+                o, lse = _attn_oracle(kv_host[b], last_idx[b, q], f32(li["q"][b, q]), win)
+                check_attention(L["out"][b, q], o, what=what)
+                np.testing.assert_allclose(L["lse"][b, q].cpu().numpy(), lse, rtol=1e-3, atol=1e-3)

@@ -102,7 +102,8 @@ def _check(wl, T, Ls, pool):
 def _small(base, **kw):
     wl = workloads.WORKLOADS[base]
     args = dict(name=wl.name + "_small", seed=wl.seed, B=wl.B, Q=wl.Q, N=wl.N, r=wl.r, modes=list(wl.modes),
-                K=wl.K, W=wl.W, hsi_blocks=wl.hsi_blocks, hsi_block=wl.hsi_block, n_new=wl.n_new)
+                K=wl.K, W=wl.W, hsi_blocks=wl.hsi_blocks, hsi_block=wl.hsi_block, n_new=wl.n_new,
+                prefill=wl.prefill, swa_step=wl.swa_step)
     args.update(kw)
     return workloads.Workload(**args)
 
@@ -113,7 +114,9 @@ def _small(base, **kw):
     _small(2, B=2, N=9000),
     _small(3, B=2, N=8 * 2500 + 3, hsi_blocks=512),
     _small(2, B=1, Q=3, N=3001, n_new=3),
-], ids=lambda w: w.name)
+    _small(4, Q=40, N=3000, n_new=20),                 # causal prefill: 5 query blocks of 8
+    _small(4, B=2, Q=19, N=1333, n_new=10),            # two rows, a partial query block
+], ids=lambda w: f"{w.name}_B{w.B}_Q{w.Q}_N{w.N}")
 def test_group_small(wl):
     T = _make(wl)
     Ls, pool = _run_group(wl, T)

@@ -53,7 +53,8 @@ def _oracle_scores(qI, w, kI, b, q, n_vis):
     return indexer.index_scores(f32(qI[b, q]), f32(w[b, q]), f32(kI[b]), n_vis)
 
 
-@pytest.mark.parametrize("B,Q,N,seed", [(1, 4, 2048, 0), (3, 2, 1000, 1), (2, 1, 5000, 2), (1, 8, 777, 3)])
+@pytest.mark.parametrize("B,Q,N,seed", [(1, 4, 2048, 0), (3, 2, 1000, 1), (2, 1, 5000, 2), (1, 8, 777, 3),
+                                         (1, 21, 3000, 4), (2, 13, 1500, 5)])
 def test_full_scan_random(B, Q, N, seed):
     qI, w, kI = _inputs(B, Q, N, seed)
     rng = np.random.default_rng(seed)
@@ -96,6 +97,22 @@ def test_all_equal_scores_take_lowest_positions():
     r = _run(0, qI, w, kI, [[N]], 512)
     np.testing.assert_array_equal(r["idx"][0, 0], np.arange(512))
     assert np.all(r["scores"][0, 0] == 0)
+
+
+def test_one_chunk_with_more_candidates_than_its_segment():
+    """2000 copies of one index-K row in the first 4096-slot chunk all tie
+    for the top score: the chunk's candidate list overflows and the exact
+    path over the scores picks the lowest 512 positions."""
+    B, Q, N = 1, 3, 9000
+    qI, w, kI = _inputs(B, Q, N, 17)
+    kI[0, 100:2100] = kI[0, 5000]
+    qI[0, :, :, :] = kI[0, 5000].float().to(torch.bfloat16)      # the copied row scores highest
+    r = _run(0, qI, w, kI, [[N, N, 2050]], 512)
+    for q in range(Q):
+        s = _oracle_scores(qI, w, kI, 0, q, [N, N, 2050][q])
+        sel = check_topk(r["idx"][0, q], s, 512, exact=True, what=f"q{q}")
+        assert np.all(np.diff(sel) > 0)
+    np.testing.assert_array_equal(r["idx"][0, 0], np.arange(100, 612))
 
 
 def test_reindex_equals_full_with_same_index_q():
