@@ -125,6 +125,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     fence_barrier_init();
   }
   if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  if (tid == 0) { tma_prefetch_desc(&tmap_q); tma_prefetch_desc(&tmap_swa); }
+  pdl_wait();                                           // idx, q and the FP4 rows come from earlier kernels
+  pdl_launch_dependents();
   int v = 0;
   if (tid < kTcAttnKeys) {
     if (tid < nkeys) {

@@ -7,6 +7,7 @@
 #include <cuda_bf16.h>
 #include <cuda.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace csa2 {
 
@@ -23,6 +24,42 @@ struct LaunchTrace {
   int* kid = nullptr;          // max kernel ids
 };
 static LaunchTrace g_trace;
+
+// Launch with programmatic stream serialisation: the kernel's CTAs may be
+// scheduled while the previous kernel in the stream is finishing, run their
+// set-up (barriers, tensor memory, descriptor prefetch) and then wait in
+// pdl_wait() until that kernel has completed and its writes are visible.
+// cluster_x > 0 adds a (cluster_x, 1, 1) thread-block cluster shape.
+// Tracing records events between launches, which serialises them as usual.
+static bool g_pdl = true;
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (g_pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 inline void trace_pre(int kid, cudaStream_t st) {
   if (g_trace.on && g_trace.n < g_trace.max) {
@@ -51,6 +88,12 @@ enum DeviceError : int {
 };
 
 __device__ int g_device_error;
+
+// Programmatic dependent launch: block until the previous kernel in the
+// stream has completed (returns at once when launched without the
+// attribute), and let the next kernel's CTAs be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void record_error(int code) {
   atomicCAS(&g_device_error, 0, code);

@@ -60,7 +60,7 @@ inline int scan_qg(int qg) { return qg <= 1 ? 1 : qg <= 2 ? 2 : qg <= 4 ? 4 : 8;
 template <int QG, bool HSI>
 void launch_scan_t(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk, const CUtensorMap& tq,
                    const ScanParams& sp) {
-  index_scan_kernel<QG, HSI><<<grid, kScanThreads, smem, st>>>(tk, tq, sp);
+  launch_ex(index_scan_kernel<QG, HSI>, dim3(grid), dim3(kScanThreads), smem, st, 0, tk, tq, sp);
 }
 void launch_scan(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
                  const CUtensorMap& tq, const ScanParams& sp) {
@@ -84,6 +84,9 @@ csa2_status device_info(DeviceInfo** out) {
   if (!d.init) {
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    // CSA2_PDL=0 launches every kernel with plain stream order
+    const char* pdl = getenv("CSA2_PDL");
+    if (pdl && pdl[0] == '0') g_pdl = false;
     d.ok = (prop.major == 10);
     d.sms = prop.multiProcessorCount;
     d.init = true;
@@ -127,12 +130,13 @@ bool make_map_bf16_128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t
 // ---------------------------------------------------------------- index call
 struct IndexPlan {
   bool pool, hsi;
-  int BQ, qg, hb, nchunks, bchunks;
+  int BQ, qg, hb;
   int64_t n_elems, nblk;
-  // counter region (histograms, candidate counters, tickets): zeroed at the
-  // start of every call; data region (scores, candidates): no precondition
-  size_t off_hist, off_bhist, off_ctr, zero_bytes;
-  size_t off_scores, off_bscores, off_seg, off_bseg, off_cnt, off_bcnt, data_bytes;
+  int64_t ld, bld;     // score row strides (multiples of 4 for 16-byte loads)
+  // counter region (histograms): zeroed at the start of every call; data
+  // region (scores): no precondition
+  size_t off_hist, off_bhist, zero_bytes;
+  size_t off_scores, off_bscores, data_bytes;
   size_t total;
 };
 
@@ -168,24 +172,29 @@ IndexPlan plan_index(const csa2_index_args* a) {
   P.hb = (P.qg <= 2) ? 12 : 10;
   P.n_elems = P.pool ? static_cast<int64_t>(a->hsi_blocks) * 8 : a->N;
   P.nblk = P.hsi ? (a->N + 7) / 8 : 0;
-  P.nchunks = static_cast<int>((P.n_elems + kTopkChunk - 1) / kTopkChunk);
-  P.bchunks = static_cast<int>((P.nblk + kTopkChunk - 1) / kTopkChunk);
+  P.ld = (P.n_elems + 3) & ~static_cast<int64_t>(3);
+  P.bld = (P.nblk + 3) & ~static_cast<int64_t>(3);
   const size_t nb = static_cast<size_t>(1) << P.hb;
   size_t off = 0;
   P.off_hist = off;    off = up256(off + static_cast<size_t>(P.BQ) * nb * 4);
   P.off_bhist = off;   off = up256(off + (P.hsi ? static_cast<size_t>(P.BQ) * nb * 4 : 0));
-  P.off_ctr = off;     off = up256(off + static_cast<size_t>(P.BQ) * 8 * 4);
   P.zero_bytes = off;
   off = 0;
-  P.off_scores = off;  off = up256(off + static_cast<size_t>(P.BQ) * P.n_elems * 4);
-  P.off_bscores = off; off = up256(off + static_cast<size_t>(P.BQ) * P.nblk * 4);
-  P.off_seg = off;     off = up256(off + static_cast<size_t>(P.BQ) * P.nchunks * kTopkSegCap * 8);
-  P.off_bseg = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.bchunks * kTopkSegCap * 8);
-  P.off_cnt = off;     off = up256(off + static_cast<size_t>(P.BQ) * P.nchunks * 4);
-  P.off_bcnt = off;    off = up256(off + static_cast<size_t>(P.BQ) * P.bchunks * 4);
+  P.off_scores = off;  off = up256(off + static_cast<size_t>(P.BQ) * P.ld * 4);
+  P.off_bscores = off; off = up256(off + static_cast<size_t>(P.BQ) * P.bld * 4);
   P.data_bytes = off;
   P.total = P.zero_bytes + P.data_bytes;
   return P;
+}
+
+// One cluster of topk_cluster_size() CTAs per selection problem.
+cudaError_t launch_topk(const TopkParams& tp, int problems, const DeviceInfo& dev, cudaStream_t st) {
+  const int C = topk_cluster_size(tp.n_elems, problems, dev.sms);
+  trace_pre(kKTopk, st);
+  const cudaError_t e = launch_ex(topk_select_kernel, dim3(static_cast<unsigned>(C), static_cast<unsigned>(problems)),
+                                  dim3(kTopkThreads), topk_smem_bytes(), st, static_cast<unsigned>(C), tp);
+  trace_post(st);
+  return e;
 }
 
 // zero: the call's counter region (already zeroed); data: its data region
@@ -197,7 +206,7 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   ScanParams sp;
   memset(&sp, 0, sizeof(sp));
   sp.pool_mode = P.pool;
-  sp.B = a->B; sp.Q = a->Q; sp.qg = P.qg; sp.N = a->N; sp.n_elems = P.n_elems;
+  sp.B = a->B; sp.Q = a->Q; sp.qg = P.qg; sp.N = a->N; sp.n_elems = P.n_elems; sp.ld = P.ld; sp.bld = P.bld;
   sp.n_vis = a->n_vis; sp.w = a->w;
   sp.pool = P.pool ? a->pool_in : nullptr;
   sp.pool_blocks = P.pool ? a->hsi_blocks : 0;
@@ -236,6 +245,7 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   TopkParams tp;
   memset(&tp, 0, sizeof(tp));
   tp.scores = sp.scores;
+  tp.ld = P.ld;
   tp.n_elems = P.n_elems;
   tp.n_vis = P.pool ? nullptr : a->n_vis;
   tp.vis_div = 1;
@@ -243,41 +253,24 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   tp.pool_blocks = sp.pool_blocks;
   tp.hist = sp.hist;
   tp.hb = P.hb;
-  tp.seg = reinterpret_cast<uint64_t*>(w + P.off_seg);
-  tp.seg_cnt = reinterpret_cast<uint32_t*>(w + P.off_cnt);
-  tp.nchunks = P.nchunks;
-  tp.ctr = reinterpret_cast<uint32_t*>(z + P.off_ctr);
-  tp.ticket_slot = 1;
-  tp.ovf_slot = 3;
   tp.K = a->K;
   tp.out_idx = a->idx;
   tp.out_scores = a->scores;
-  const size_t tsm = topk_smem_bytes();
-  trace_pre(kKTopk, st);
-  topk_select_kernel<<<dim3(static_cast<unsigned>(P.nchunks), static_cast<unsigned>(P.BQ)), kTopkThreads, tsm, st>>>(tp);
-  trace_post(st);
-  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+  if (launch_topk(tp, P.BQ, dev, st) != cudaSuccess) return CSA2_ERR_CUDA;
 
   if (P.hsi) {
     TopkParams bp = tp;
     bp.scores = sp.bscores;
+    bp.ld = P.bld;
     bp.n_elems = P.nblk;
     bp.n_vis = a->n_vis;
     bp.vis_div = 8;
     bp.pool = nullptr;
-    bp.seg = reinterpret_cast<uint64_t*>(w + P.off_bseg);
-    bp.seg_cnt = reinterpret_cast<uint32_t*>(w + P.off_bcnt);
-    bp.nchunks = P.bchunks;
     bp.hist = sp.bhist;
-    bp.ticket_slot = 2;
-    bp.ovf_slot = 4;
     bp.K = a->hsi_blocks;
     bp.out_idx = a->pool_out;
     bp.out_scores = nullptr;
-    trace_pre(kKTopk, st);
-    topk_select_kernel<<<dim3(static_cast<unsigned>(P.bchunks), static_cast<unsigned>(P.BQ)), kTopkThreads, tsm, st>>>(bp);
-    trace_post(st);
-    if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+    if (launch_topk(bp, P.BQ, dev, st) != cudaSuccess) return CSA2_ERR_CUDA;
   }
   return CSA2_OK;
 }
@@ -343,9 +336,10 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
     tw = tq;                                    // no window slices: never used
   }
   trace_pre(kKAttnSlice, st);
-  sparse_attn_tc_kernel<<<dim3(slices, static_cast<unsigned>(bq)), kTcAttnThreads, kTcAttnSmem, st>>>(tq, tw, t);
+  const cudaError_t e1 = launch_ex(sparse_attn_tc_kernel, dim3(slices, static_cast<unsigned>(bq)), dim3(kTcAttnThreads),
+                                   kTcAttnSmem, st, 0, tq, tw, t);
   trace_post(st);
-  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+  if (e1 != cudaSuccess) return CSA2_ERR_CUDA;
 
   AttnParams p;
   p.slices = slices;
@@ -354,9 +348,9 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
   p.out = static_cast<__nv_bfloat16*>(a->out);
   p.lse = a->lse;
   trace_pre(kKAttnCombine, st);
-  sparse_attn_combine_kernel<<<static_cast<unsigned>(bq * 64), 128, 0, st>>>(p);
+  const cudaError_t e2 = launch_ex(sparse_attn_combine_kernel, dim3(static_cast<unsigned>(bq * 64)), dim3(128), 0, st, 0, p);
   trace_post(st);
-  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+  if (e2 != cudaSuccess) return CSA2_ERR_CUDA;
   return CSA2_OK;
 }
 

@@ -45,12 +45,13 @@ struct ScanParams {
   int qblocks;            // scan: query blocks per batch row, ceil(Q / qg)
   int64_t N;              // index-K rows per batch row
   int64_t n_elems;        // score slots per query: N (scan) or pool_blocks*8 (pool)
+  int64_t ld, bld;        // row strides of scores and bscores (multiples of 4)
   const int32_t* n_vis;   // [B*Q]
   const float* w;         // [B*Q*32]
   const int32_t* pool;    // pool mode: [B*Q][pool_blocks]
   int pool_blocks;
-  float* scores;          // [B*Q][n_elems]
-  float* bscores;         // scan with HSI: [B*Q][nblk]
+  float* scores;          // [B*Q][ld]
+  float* bscores;         // scan with HSI: [B*Q][bld]
   int64_t nblk;
   uint32_t* hist;         // [B*Q][1 << hb]       (zero at launch)
   uint32_t* bhist;        // scan with HSI: [B*Q][1 << hb]
@@ -111,6 +112,23 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int qn = p.pool_mode ? 1 : min(p.qg, p.Q - q0);   // queries of this group
   const int nbins = 1 << p.hb;
 
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int a = 0; a < scan_acc_bufs(QG); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 128); }
+    mbar_init(q_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmap_k); tma_prefetch_desc(&tmap_q); }
+  if (warp == 1) { tmem_alloc(tmem_slot, p.tmem_cols); tmem_relinquish(); }
+  for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) hist_s[i] = 0;
+  if (HSI) for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) bhist_s[i] = 0;
+
+  // the inputs below, and the score buffers this kernel overwrites, belong
+  // to earlier kernels in the stream until they have completed
+  pdl_wait();
+  pdl_launch_dependents();
+
   // this CTA's tile range; in scan mode, tiles past every query's n_vis are skipped
   int tile_lo = static_cast<int>((static_cast<int64_t>(cig) * p.tiles_per_group) / p.ctas_per_group);
   int tile_hi = static_cast<int>((static_cast<int64_t>(cig + 1) * p.tiles_per_group) / p.ctas_per_group);
@@ -124,18 +142,6 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     tile_hi = min(tile_hi, (nmax + kTileRows - 1) / kTileRows);
   }
   const int ntiles = max(0, tile_hi - tile_lo);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-    for (int a = 0; a < scan_acc_bufs(QG); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 128); }
-    mbar_init(q_bar, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmap_k); tma_prefetch_desc(&tmap_q); }
-  if (warp == 1) { tmem_alloc(tmem_slot, p.tmem_cols); tmem_relinquish(); }
-  for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) hist_s[i] = 0;
-  if (HSI) for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) bhist_s[i] = 0;
   for (int i = threadIdx.x; i < QG * 32; i += blockDim.x) w_s[i] = (i < qn * 32) ? p.w[bq0 * 32 + i] : 0.0f;
   tc_fence_before();
   __syncthreads();
@@ -233,36 +239,59 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
         pool_valid = blk >= 0;
         pos = static_cast<int64_t>(blk) * 8 + (e & 7);
       }
+      // QB queries' head values per TMEM round trip: the loads of a batch
+      // are in flight together and one wait covers them
+      constexpr int QB = (QG >= 4) ? (HSI ? 2 : 4) : QG;
 #pragma unroll
-      for (int q = 0; q < QG; ++q) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * n_mma + 32 * q, r);
+      for (int qb = 0; qb < QG; qb += QB) {
+        uint32_t r[QB][32];
+#pragma unroll
+        for (int j = 0; j < QB; ++j)
+          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * n_mma + 32 * (qb + j), r[j]);
         tmem_ld_wait();
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          const float wh = (QG <= 2) ? wr[(QG <= 2 ? q : 0) * 32 + h] : w_s[q * 32 + h];
-          acc[h & 3] = fmaf(wh, fmaxf(__uint_as_float(r[h]), 0.0f), acc[h & 3]);
+        if (qb + QB >= QG) {
+          // every head value of the tile is in registers: hand the
+          // accumulator back to the MMA issuer before the reductions
+          tc_fence_before();
+          mbar_arrive(&tempty_bar[a]);
         }
-        float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        const bool valid = pool_valid && pos < nv[q] && q < qn;
-        if (!valid) s = -INFINITY;
-        const bool in_range = e < p.n_elems && q < qn;
-        if (in_range) p.scores[static_cast<int64_t>(bq0 + q) * p.n_elems + e] = s;
-        warp_hist_add(hist_s + q * nbins, okey(s) >> (32 - p.hb), in_range && valid);
-        if (HSI) {
-          float m = s;
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-          const int64_t jb = e >> 3;
-          const bool writer = (lane & 7) == 0 && jb < p.nblk && q < qn;
-          if (writer) p.bscores[static_cast<int64_t>(bq0 + q) * p.nblk + jb] = m;
-          warp_hist_add(bhist_s + q * nbins, okey(m) >> (32 - p.hb), writer && m != -INFINITY);
+#pragma unroll
+        for (int j = 0; j < QB; ++j) {
+          const int q = qb + j;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          if (QG <= 2) {
+#pragma unroll
+            for (int h = 0; h < 32; ++h)
+              acc[h & 3] = fmaf(wr[(QG <= 2 ? q : 0) * 32 + h], fmaxf(__uint_as_float(r[j][h]), 0.0f), acc[h & 3]);
+          } else {
+            const float4* w4 = reinterpret_cast<const float4*>(w_s + q * 32);
+#pragma unroll
+            for (int h4 = 0; h4 < 8; ++h4) {
+              const float4 wv = w4[h4];
+              acc[0] = fmaf(wv.x, fmaxf(__uint_as_float(r[j][4 * h4 + 0]), 0.0f), acc[0]);
+              acc[1] = fmaf(wv.y, fmaxf(__uint_as_float(r[j][4 * h4 + 1]), 0.0f), acc[1]);
+              acc[2] = fmaf(wv.z, fmaxf(__uint_as_float(r[j][4 * h4 + 2]), 0.0f), acc[2]);
+              acc[3] = fmaf(wv.w, fmaxf(__uint_as_float(r[j][4 * h4 + 3]), 0.0f), acc[3]);
+            }
+          }
+          float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          const bool valid = pool_valid && pos < nv[q] && q < qn;
+          if (!valid) s = -INFINITY;
+          const bool in_range = e < p.n_elems && q < qn;
+          if (in_range) p.scores[static_cast<int64_t>(bq0 + q) * p.ld + e] = s;
+          warp_hist_add(hist_s + q * nbins, okey(s) >> (32 - p.hb), in_range && valid);
+          if (HSI) {
+            float m = s;
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            const int64_t jb = e >> 3;
+            const bool writer = (lane & 7) == 0 && jb < p.nblk && q < qn;
+            if (writer) p.bscores[static_cast<int64_t>(bq0 + q) * p.bld + jb] = m;
+            warp_hist_add(bhist_s + q * nbins, okey(m) >> (32 - p.hb), writer && m != -INFINITY);
+          }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&tempty_bar[a]);
     }
     // flush the CTA's histograms into the global ones
     named_bar_sync(1, kScanEpiThreads);

@@ -46,6 +46,8 @@ quantize_kv_fp4_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t l
                        int64_t row_offset) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
   if (row >= n) return;
 
   const uint4* src = reinterpret_cast<const uint4*>(x + row * ld_x + lane * 16);
@@ -94,10 +96,11 @@ inline cudaError_t launch_quantize(const void* x, int64_t n, int64_t ld_x, void*
   const int warps = 8;
   const int64_t blocks = (n + warps - 1) / warps;
   trace_pre(kKQuantize, st);
-  quantize_kv_fp4_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), n, ld_x, static_cast<uint8_t*>(kv), dst_rows, row_offset);
+  const cudaError_t e = launch_ex(quantize_kv_fp4_kernel, dim3(static_cast<unsigned>(blocks)), dim3(warps * 32), 0, st,
+                                  0, static_cast<const __nv_bfloat16*>(x), n, ld_x, static_cast<uint8_t*>(kv),
+                                  dst_rows, row_offset);
   trace_post(st);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace csa2

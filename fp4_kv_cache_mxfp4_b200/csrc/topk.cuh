@@ -5,49 +5,51 @@
 // word inverts the position, so every key is distinct and "larger key" means
 // "higher score, then lower position": the top-K set is the K largest keys.
 //
-// One launch per selection problem, grid (chunks, queries), 256 threads:
+// One thread-block cluster of C CTAs per selection problem (grid (C,
+// queries), 512 threads per CTA); CTA r of the cluster owns the r-th of C
+// contiguous slices of the query's visible slots.
 //  0. every CTA reads the query's score histogram (built by the scan
 //     epilogue, coalesced) and finds the threshold bin tb, the highest bin
 //     whose suffix count reaches need = min(K, visible): every top-K key has
 //     its top bits >= tb;
-//  1. every CTA compacts the keys of its 4096-slot chunk whose bin is >= tb
-//     into the chunk's own segment, in position order (block prefix scan),
-//     and records the segment's length;
-//  2. the last CTA of the query (ticket counter) gathers the segments in
-//     chunk order into shared memory, radix-selects the need-th largest key
-//     (8-bit digits from the top) and writes the keys at or above it by an
-//     ordered compaction: the result comes out in ascending position order,
-//     deterministically, without a sort.
-// If the candidates do not fit in shared memory, step 2 runs over the
-// scores themselves with the same filter (slower, exact).
+//  1. every CTA streams its slice with 16-byte loads and compacts the keys
+//     whose bin is >= tb into its own shared memory, in position order
+//     (warp prefix sums, one block scan per 8192 slots);
+//  2. the CTAs publish their counts to the cluster's first CTA, which pulls
+//     the other CTAs' candidates over distributed shared memory (in slice
+//     order, so the list stays in position order), radix-selects the
+//     need-th largest key (8-bit digits from the top) and writes the keys at
+//     or above it by an ordered compaction: the result comes out in
+//     ascending position order, deterministically, without a sort.
+// If the candidates do not fit in the first CTA's shared memory (massive
+// ties), step 2 runs over the scores themselves with the same filter
+// (slower, exact).
 // HBM roofline: 4 B per score read (normally still resident in L2).
 #pragma once
+#include <cooperative_groups.h>
 #include "common.cuh"
 
 namespace csa2 {
 
-constexpr int kTopkThreads = 256;
-constexpr int kTopkPer = 16;              // slots per thread
-constexpr int kTopkChunk = kTopkThreads * kTopkPer;   // 4096 slots per CTA
-constexpr int kTopkSegCap = 1024;         // candidates kept per chunk (more: exact fallback)
-constexpr int kTopkSmemKeys = 6144;       // candidates cached in shared memory
-constexpr int kTopkMaxChunks = 2048;      // chunk offsets kept in shared memory
+namespace cg = cooperative_groups;
+
+constexpr int kTopkThreads = 512;
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkWarpSlots = 512;                        // slots per warp per iteration (4 x float4 per lane)
+constexpr int kTopkIterSlots = kTopkWarps * kTopkWarpSlots; // 8192 slots per CTA per iteration
+constexpr int kTopkCap = 12288;                             // candidate keys a CTA holds (the cluster's total)
+constexpr int kTopkMaxCluster = 8;
 
 struct TopkParams {
-  const float* scores;
-  int64_t n_elems;          // score slots per query (row stride)
+  const float* scores;      // [BQ][ld]
+  int64_t ld;               // row stride of scores, a multiple of 4
+  int64_t n_elems;          // score slots per query
   const int32_t* n_vis;     // optional [BQ]: valid slots = ceil(n_vis / vis_div)
   int vis_div;
   const int32_t* pool;      // pool mode: position of slot e = pool[e/8]*8 + e%8
   int pool_blocks;
   const uint32_t* hist;     // [BQ][1 << hb] score histogram from the scan
   int hb;
-  uint64_t* seg;            // [BQ][nchunks][kTopkSegCap]: chunk c's candidates
-  uint32_t* seg_cnt;        // [BQ][nchunks]
-  int nchunks;
-  uint32_t* ctr;            // [BQ][8], zero at the scan's launch
-  int ticket_slot;          // ctr[ticket_slot]: finished CTAs of the query
-  int ovf_slot;             // ctr[ovf_slot] != 0: a chunk had more than kTopkSegCap candidates
   int K;
   int32_t* out_idx;         // [BQ][K]
   float* out_scores;        // optional [BQ][K]
@@ -55,9 +57,9 @@ struct TopkParams {
 
 struct TopkShared {
   uint32_t h256[256];
-  uint32_t warp_tot[32];
-  uint32_t chunk_off[kTopkMaxChunks + 1];
-  int last, d, gt, eq, total, tb;
+  uint32_t warp_tot[kTopkWarps];
+  uint32_t cnt[kTopkMaxCluster];   // first CTA: candidates found by each CTA of the cluster
+  int d, gt, eq, total, tb;
 };
 
 __device__ __forceinline__ int64_t topk_valid_slots(const TopkParams& p, int bq) {
@@ -72,22 +74,19 @@ __device__ __forceinline__ uint32_t topk_position(const TopkParams& p, int bq, i
   return static_cast<uint32_t>(blk * 8 + static_cast<int>(e & 7));
 }
 
-// key of score s at slot e, or 0 when the slot holds no visible score or
-// sits below tb
-__device__ __forceinline__ uint64_t topk_key_of(const TopkParams& p, int bq, int64_t e, float s, int tb) {
-  if (s == -INFINITY) return 0;
-  const uint32_t k = okey(s);
-  if (static_cast<int>(k >> (32 - p.hb)) < tb) return 0;
-  return (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(~topk_position(p, bq, e));
+// is score s a candidate: visible (not -inf) and in bin tb or above
+__device__ __forceinline__ bool topk_is_cand(float s, int tb, int hb) {
+  return s != -INFINITY && static_cast<int>(okey(s) >> (32 - hb)) >= tb;
+}
+
+__device__ __forceinline__ uint64_t topk_make_key(const TopkParams& p, int bq, int64_t e, float s) {
+  return (static_cast<uint64_t>(okey(s)) << 32) | static_cast<uint32_t>(~topk_position(p, bq, e));
 }
 
 // key of slot e, or 0 when the slot holds no visible score or sits below tb
 __device__ __forceinline__ uint64_t topk_slot_key(const TopkParams& p, int bq, int64_t e, int tb) {
-  const float s = p.scores[static_cast<int64_t>(bq) * p.n_elems + e];
-  if (s == -INFINITY) return 0;
-  const uint32_t k = okey(s);
-  if (static_cast<int>(k >> (32 - p.hb)) < tb) return 0;
-  return (static_cast<uint64_t>(k) << 32) | static_cast<uint32_t>(~topk_position(p, bq, e));
+  const float s = p.scores[static_cast<int64_t>(bq) * p.ld + e];
+  return topk_is_cand(s, tb, p.hb) ? topk_make_key(p, bq, e, s) : 0;
 }
 
 // Exclusive prefix sum over the block; *total gets the sum.  Ends with a
@@ -103,14 +102,14 @@ __device__ __forceinline__ uint32_t topk_block_scan(uint32_t v, TopkShared& S, u
   if (lane == 31) S.warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t x = (lane < kTopkThreads / 32) ? S.warp_tot[lane] : 0;
+    const uint32_t x = (lane < kTopkWarps) ? S.warp_tot[lane] : 0;
     uint32_t xi = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t t = __shfl_up_sync(0xffffffffu, xi, o);
       if (lane >= o) xi += t;
     }
-    S.warp_tot[lane] = xi - x;                      // exclusive per warp
+    if (lane < kTopkWarps) S.warp_tot[lane] = xi - x;   // exclusive per warp
     if (lane == 31) S.total = static_cast<int>(xi);
   }
   __syncthreads();
@@ -189,38 +188,43 @@ topk_select_kernel(TopkParams p) {
   extern __shared__ __align__(1024) uint8_t topk_smem_raw[];
   TopkShared& S = *reinterpret_cast<TopkShared*>(topk_smem_raw);
   uint64_t* keys_s = reinterpret_cast<uint64_t*>(topk_smem_raw + ((sizeof(TopkShared) + 15) & ~size_t(15)));
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+
+  // every CTA of the cluster must have started before another one writes
+  // its shared memory: arrive now, wait just before the first remote store
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
   const int bq = blockIdx.y;
-  const int tid = threadIdx.x;
-  uint32_t* ctr = p.ctr + static_cast<int64_t>(bq) * 8;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t nvalid = topk_valid_slots(p, bq);
-
-  // this thread's 16 slots of the chunk, loaded before the histogram so the
-  // two reads overlap
-  const int64_t slot0 = static_cast<int64_t>(blockIdx.x) * kTopkChunk + kTopkPer * tid;
-  float sv[kTopkPer];
-#pragma unroll
-  for (int i = 0; i < kTopkPer; ++i)
-    sv[i] = (slot0 + i < nvalid) ? p.scores[static_cast<int64_t>(bq) * p.n_elems + slot0 + i] : -INFINITY;
+  const float* row = p.scores + static_cast<int64_t>(bq) * p.ld;
 
   // -- 0. threshold bin: thread t owns the `per` bins just below bin
   //       nbins - per*t (descending ranges), read with coalesced loads
   int need;
   {
     const int nbins = 1 << p.hb;
-    const int per = nbins / kTopkThreads;             // 16 (12-bit) or 4 (10-bit)
+    const int per = nbins / kTopkThreads;             // 8 (12-bit) or 2 (10-bit)
     const uint32_t* hq = p.hist + static_cast<int64_t>(bq) * nbins;
     const int lo_bin = nbins - per * (tid + 1);
-    uint32_t c[16];
+    uint32_t c[8];
+    if (per == 8) {
+      const uint4 v0 = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin));
+      const uint4 v1 = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin) + 1);
+      c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w; c[4] = v1.x; c[5] = v1.y; c[6] = v1.z; c[7] = v1.w;
+    } else {
+      const uint2 v0 = __ldcg(reinterpret_cast<const uint2*>(hq + lo_bin));
+      c[0] = v0.x; c[1] = v0.y;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (4 * j < per) v = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin) + j);
-      c[4 * j] = v.x; c[4 * j + 1] = v.y; c[4 * j + 2] = v.z; c[4 * j + 3] = v.w;
+      for (int j = 2; j < 8; ++j) c[j] = 0;
     }
     uint32_t local = 0;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) local += c[j];
+    for (int j = 0; j < 8; ++j) local += c[j];
     uint32_t total;
     uint32_t above = topk_block_scan(local, S, &total);   // bins above this thread's range
     need = static_cast<int>(total < static_cast<uint32_t>(p.K) ? total : static_cast<uint32_t>(p.K));
@@ -229,7 +233,7 @@ topk_select_kernel(TopkParams p) {
     if (need > 0 && above < static_cast<uint32_t>(need) && above + local >= static_cast<uint32_t>(need)) {
       bool found = false;
 #pragma unroll
-      for (int j = 15; j >= 0; --j) {
+      for (int j = 7; j >= 0; --j) {
         if (j < per && !found) {
           above += c[j];
           if (above >= static_cast<uint32_t>(need)) { S.tb = lo_bin + j; found = true; }
@@ -239,86 +243,106 @@ topk_select_kernel(TopkParams p) {
     __syncthreads();
   }
   const int tb = S.tb;
-  uint64_t* seg_q = p.seg + static_cast<int64_t>(bq) * p.nchunks * kTopkSegCap;
-  uint32_t* cnt_q = p.seg_cnt + static_cast<int64_t>(bq) * p.nchunks;
 
-  // -- 1. this chunk's candidates, in position order ------------------------
-  {
-    uint64_t k[kTopkPer];
-    uint32_t n = 0;
+  // -- 1. this CTA's slice: candidates into shared memory, in position order
+  uint32_t n = 0;                                     // candidates so far (uniform over the block)
+  if (need > 0) {
+    const int64_t span = (((nvalid + C - 1) / C) + 3) & ~static_cast<int64_t>(3);
+    const int64_t lo = min(nvalid, static_cast<int64_t>(rank) * span);
+    const int64_t hi = min(nvalid, lo + span);
+    for (int64_t it = lo; it < hi; it += kTopkIterSlots) {
+      const int64_t wbase = it + static_cast<int64_t>(warp) * kTopkWarpSlots;
+      float v[4][4];
 #pragma unroll
-    for (int i = 0; i < kTopkPer; ++i) {
-      k[i] = (need > 0) ? topk_key_of(p, bq, slot0 + i, sv[i], tb) : 0;
-      n += (k[i] != 0);
-    }
-    uint32_t total;
-    uint32_t off = topk_block_scan(n, S, &total);
-    uint64_t* seg = seg_q + static_cast<int64_t>(blockIdx.x) * kTopkSegCap;
+      for (int j = 0; j < 4; ++j) {
+        const int64_t s0 = wbase + 128 * j + 4 * lane;
+        float4 x = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        if (s0 < hi) x = __ldcg(reinterpret_cast<const float4*>(row + s0));
+        v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
+      }
+      // candidate flags and this lane's offset inside the warp's 512 slots
+      uint32_t fl[4], wexcl[4], wtot = 0;
 #pragma unroll
-    for (int i = 0; i < kTopkPer; ++i) {
-      if (k[i] != 0 && off < static_cast<uint32_t>(kTopkSegCap)) seg[off] = k[i];
-      off += (k[i] != 0);
+      for (int j = 0; j < 4; ++j) {
+        const int64_t s0 = wbase + 128 * j + 4 * lane;
+        uint32_t f = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) f |= (s0 + c < hi && topk_is_cand(v[j][c], tb, p.hb)) ? (1u << c) : 0u;
+        fl[j] = f;
+        const uint32_t cnt = __popc(f);
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        wexcl[j] = wtot + incl - cnt;
+        wtot += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      uint32_t btot;
+      const uint32_t wofs = n + topk_block_scan(lane == 0 ? wtot : 0u, S, &btot);
+      const uint32_t wbase_ofs = __shfl_sync(0xffffffffu, wofs, 0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t o = wbase_ofs + wexcl[j];
+        const int64_t s0 = wbase + 128 * j + 4 * lane;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (fl[j] & (1u << c)) {
+            if (o < static_cast<uint32_t>(kTopkCap)) keys_s[o] = topk_make_key(p, bq, s0 + c, v[j][c]);
+            ++o;
+          }
+        }
+      }
+      n += btot;
     }
-    if (tid == 0) {
-      cnt_q[blockIdx.x] = min(total, static_cast<uint32_t>(kTopkSegCap));
-      if (total > static_cast<uint32_t>(kTopkSegCap)) atomicOr(ctr + p.ovf_slot, 1u);
-    }
-    __threadfence();                                      // publish this thread's writes before the ticket
   }
 
-  // -- 2. the last CTA of this query selects ---------------------------------
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    S.last = (atomicAdd(ctr + p.ticket_slot, 1u) == gridDim.x - 1);
+  // -- 2. the cluster's first CTA gathers and selects -------------------------
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (tid == 0) *cluster.map_shared_rank(&S.cnt[rank], 0) = n;
+  cluster.sync();                                     // counts and candidate lists visible cluster-wide
+  bool fits = true;
+  uint32_t n_all = 0;
+  if (rank == 0 && need > 0) {
+    for (int r = 0; r < C; ++r) {
+      const uint32_t c = S.cnt[r];
+      fits = fits && c <= static_cast<uint32_t>(kTopkCap);
+      n_all += c;
+    }
+    fits = fits && n_all <= static_cast<uint32_t>(kTopkCap);
+    if (fits) {
+      uint32_t off = S.cnt[0];
+      for (int r = 1; r < C; ++r) {
+        const uint64_t* remote = cluster.map_shared_rank(keys_s, r);
+        const uint32_t c = S.cnt[r];
+        for (uint32_t i = tid; i < c; i += kTopkThreads) keys_s[off + i] = remote[i];
+        off += c;
+      }
+    }
   }
-  __syncthreads();
-  if (!S.last) return;
-  __threadfence();
+  cluster.sync();                                     // the other CTAs' lists are no longer read
+  if (rank != 0) return;
 
   int32_t* out_idx = p.out_idx + static_cast<int64_t>(bq) * p.K;
   float* out_sc = p.out_scores ? p.out_scores + static_cast<int64_t>(bq) * p.K : nullptr;
   uint32_t written = 0;
   if (need > 0) {
-    // chunk offsets (exclusive scan of the segment lengths)
-    uint32_t C = 0;
-    bool fits = p.nchunks <= kTopkMaxChunks && __ldcg(ctr + p.ovf_slot) == 0;
     if (fits) {
-      for (int c0 = 0; c0 < p.nchunks; c0 += kTopkThreads) {
-        const int c = c0 + tid;
-        const uint32_t v = (c < p.nchunks) ? __ldcg(cnt_q + c) : 0;
-        uint32_t tot;
-        const uint32_t o = topk_block_scan(v, S, &tot);
-        if (c < p.nchunks) S.chunk_off[c] = C + o;
-        C += tot;
-      }
-      if (tid == 0) S.chunk_off[p.nchunks] = C;
-      __syncthreads();
-      fits = C <= static_cast<uint32_t>(kTopkSmemKeys);
-    }
-    if (fits) {
-      // gather the segments in chunk order: one warp per chunk
-      const int lane = tid & 31, warp = tid >> 5;
-      for (int c = warp; c < p.nchunks; c += kTopkThreads / 32) {
-        const uint32_t o = S.chunk_off[c], n = S.chunk_off[c + 1] - o;
-        const uint64_t* seg = seg_q + static_cast<int64_t>(c) * kTopkSegCap;
-        for (uint32_t i = lane; i < n; i += 32) keys_s[o + i] = __ldcg(seg + i);
-      }
-      __syncthreads();
-      const uint64_t P = topk_radix_select(S, C, need, [&](int64_t i) { return keys_s[i]; });
+      const uint64_t P = topk_radix_select(S, n_all, need, [&](int64_t i) { return keys_s[i]; });
       // ordered compaction of the keys >= P (4 consecutive keys per thread)
-      for (uint32_t i0 = 0; i0 < C; i0 += 4 * kTopkThreads) {
+      for (uint32_t i0 = 0; i0 < n_all; i0 += 4 * kTopkThreads) {
         uint64_t k[4];
-        uint32_t n = 0;
+        uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t j = i0 + 4 * tid + i;
-          k[i] = (j < C) ? keys_s[j] : 0;
+          k[i] = (j < n_all) ? keys_s[j] : 0;
           if (k[i] < P) k[i] = 0;
-          n += (k[i] != 0);
+          m += (k[i] != 0);
         }
         uint32_t tot;
-        uint32_t o = written + topk_block_scan(n, S, &tot);
+        uint32_t o = written + topk_block_scan(m, S, &tot);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           if (k[i] != 0) topk_emit(p, out_idx, out_sc, o++, k[i]);
@@ -329,16 +353,16 @@ topk_select_kernel(TopkParams p) {
       const uint64_t P = topk_radix_select(S, nvalid, need, [&](int64_t e) { return topk_slot_key(p, bq, e, tb); });
       for (int64_t e0 = 0; e0 < nvalid; e0 += 4 * kTopkThreads) {
         uint64_t k[4];
-        uint32_t n = 0;
+        uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int64_t e = e0 + 4 * tid + i;
           k[i] = (e < nvalid) ? topk_slot_key(p, bq, e, tb) : 0;
           if (k[i] < P) k[i] = 0;
-          n += (k[i] != 0);
+          m += (k[i] != 0);
         }
         uint32_t tot;
-        uint32_t o = written + topk_block_scan(n, S, &tot);
+        uint32_t o = written + topk_block_scan(m, S, &tot);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           if (k[i] != 0) topk_emit(p, out_idx, out_sc, o++, k[i]);
@@ -354,7 +378,17 @@ topk_select_kernel(TopkParams p) {
 }
 
 inline size_t topk_smem_bytes() {
-  return ((sizeof(TopkShared) + 15) & ~size_t(15)) + static_cast<size_t>(kTopkSmemKeys) * 8;
+  return ((sizeof(TopkShared) + 15) & ~size_t(15)) + static_cast<size_t>(kTopkCap) * 8;
+}
+
+// CTAs per selection problem: enough to spread a long score row over SMs
+// (one CTA per 16K slots, at most a portable cluster of 8), fewer once the
+// problems alone fill the GPU twice over.
+inline int topk_cluster_size(int64_t n_elems, int problems, int sms) {
+  int c = 1;
+  while (c < kTopkMaxCluster && static_cast<int64_t>(c) * 16384 < n_elems) c <<= 1;
+  while (c > 1 && static_cast<int64_t>(problems) * c > 2 * static_cast<int64_t>(sms)) c >>= 1;
+  return c;
 }
 
 }  // namespace csa2

@@ -84,6 +84,10 @@ WORKLOADS = {
     4: Workload("prefill_t4096_prefix256k_r2", 4, B=1, Q=4096, N=131072 + 2048, r=2, modes=[FULL],
                 n_new=2048, prefill=True, swa_step=1,
                 desc="Prefill chunk of 4096 tokens after a 256K-token prefix at r=2, causal"),
+    5: Workload("prefill_t1024_prefix64k_r2", 5, B=1, Q=1024, N=32768 + 512, r=2, modes=[FULL],
+                n_new=512, prefill=True, swa_step=1,
+                desc="Prefill chunk of 1024 tokens after a 64K-token prefix at r=2, causal: the prefill "
+                     "kernels at a size small enough for full profiler captures"),
 }
 
 

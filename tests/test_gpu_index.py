@@ -99,10 +99,9 @@ def test_all_equal_scores_take_lowest_positions():
     assert np.all(r["scores"][0, 0] == 0)
 
 
-def test_one_chunk_with_more_candidates_than_its_segment():
-    """2000 copies of one index-K row in the first 4096-slot chunk all tie
-    for the top score: the chunk's candidate list overflows and the exact
-    path over the scores picks the lowest 512 positions."""
+def test_many_ties_at_the_top():
+    """2000 copies of one index-K row all tie for the top score: the tie
+    break alone decides which 512 are taken (the lowest positions)."""
     B, Q, N = 1, 3, 9000
     qI, w, kI = _inputs(B, Q, N, 17)
     kI[0, 100:2100] = kI[0, 5000]
