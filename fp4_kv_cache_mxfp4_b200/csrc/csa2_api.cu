@@ -28,6 +28,7 @@ struct DeviceInfo {
   bool ok = false;
   int sms = 0;
   bool attrs_set = false;
+  int topk_max_cluster = 8;   // 16 where the GPU can place clusters of 16 top-K CTAs
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -76,6 +77,33 @@ void launch_scan(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, 
   }
 }
 
+// Largest top-K cluster this GPU can place: 16 (non-portable) when at least
+// one such cluster fits, else the portable 8.
+int topk_cluster_limit() {
+  if (cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 8;
+  }
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(16, 1, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.dynamicSmemBytes = topk_smem_bytes();
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 16;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, topk_select_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 8;
+  }
+  return n >= 1 ? 16 : 8;
+}
+
 csa2_status device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
@@ -99,6 +127,7 @@ csa2_status device_info(DeviceInfo** out) {
         set_smem_attrs(sparse_attn_combine_kernel, 0) != cudaSuccess ||
         set_smem_attrs(quantize_kv_fp4_kernel, 0) != cudaSuccess)
       return CSA2_ERR_CUDA;
+    d.topk_max_cluster = topk_cluster_limit();
     if (!g_encode) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -189,7 +218,7 @@ IndexPlan plan_index(const csa2_index_args* a) {
 
 // One cluster of topk_cluster_size() CTAs per selection problem.
 cudaError_t launch_topk(const TopkParams& tp, int problems, const DeviceInfo& dev, cudaStream_t st) {
-  const int C = topk_cluster_size(tp.n_elems, problems, dev.sms);
+  const int C = topk_cluster_size(tp.n_elems, problems, dev.sms, dev.topk_max_cluster);
   trace_pre(kKTopk, st);
   const cudaError_t e = launch_ex(topk_select_kernel, dim3(static_cast<unsigned>(C), static_cast<unsigned>(problems)),
                                   dim3(kTopkThreads), topk_smem_bytes(), st, static_cast<unsigned>(C), tp);

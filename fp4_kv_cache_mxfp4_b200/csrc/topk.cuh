@@ -35,10 +35,11 @@ namespace cg = cooperative_groups;
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkWarpSlots = 512;                        // slots per warp per iteration (4 x float4 per lane)
-constexpr int kTopkIterSlots = kTopkWarps * kTopkWarpSlots; // 8192 slots per CTA per iteration
+constexpr int kTopkVec = 8;                                  // float4 per lane per chunk
+constexpr int kTopkWarpSlots = 32 * 4 * kTopkVec;            // 1024 contiguous slots per warp per chunk
+constexpr int kTopkChunkSlots = kTopkWarps * kTopkWarpSlots; // 16384 slots per CTA per chunk
 constexpr int kTopkCap = 12288;                             // candidate keys a CTA holds (the cluster's total)
-constexpr int kTopkMaxCluster = 8;
+constexpr int kTopkMaxCluster = 16;                         // 16 needs the non-portable cluster attribute
 
 struct TopkParams {
   const float* scores;      // [BQ][ld]
@@ -58,8 +59,8 @@ struct TopkParams {
 struct TopkShared {
   uint32_t h256[256];
   uint32_t warp_tot[kTopkWarps];
-  uint32_t cnt[kTopkMaxCluster];   // first CTA: candidates found by each CTA of the cluster
-  int d, gt, eq, total, tb;
+  uint32_t cnt[kTopkMaxCluster];   // candidates found by each CTA of the cluster
+  int d, gt, eq, total, tb, above;  // above: visible slots in bins higher than tb
 };
 
 __device__ __forceinline__ int64_t topk_valid_slots(const TopkParams& p, int bq) {
@@ -148,12 +149,19 @@ __device__ __forceinline__ void topk_pick_digit(TopkShared& S, int remaining) {
 
 // Radix select over a key source: returns P such that the keys >= P are
 // exactly the `need` largest (keys are distinct; key 0 means "absent").
-template <class KeyAt>
-__device__ uint64_t topk_radix_select(TopkShared& S, int64_t n, int need, KeyAt key_at) {
-  uint64_t prefix = 0;
-  int bits = 0, remaining = need;
+// The caller knows the top `bits0` bits of the need-th key (its histogram
+// bin), `prefix0` holding them, and that `above` keys lie strictly above
+// that bin: the passes only look at keys sharing the prefix.
+// AGG: aggregate equal digits per warp before the shared atomic (for key
+// sources that may hold long runs of equal keys, as the fallback does).
+template <bool AGG, class KeyAt>
+__device__ uint64_t topk_radix_select(TopkShared& S, int64_t n, int need, int bits0, uint64_t prefix0, int above,
+                                      KeyAt key_at) {
+  uint64_t prefix = prefix0;
+  int bits = bits0, remaining = need - above;
   while (true) {
-    const int shift = 56 - bits;
+    const int width = min(8, 64 - bits);
+    const int shift = 64 - bits - width;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) S.h256[i] = 0;
     if (threadIdx.x == 0) S.d = -1;
     __syncthreads();
@@ -161,14 +169,16 @@ __device__ uint64_t topk_radix_select(TopkShared& S, int64_t n, int need, KeyAt 
       const int64_t i = i0 + threadIdx.x;
       const uint64_t k = (i < n) ? key_at(i) : 0;
       const bool act = k != 0 && (bits == 0 || (k >> (64 - bits)) == (prefix >> (64 - bits)));
-      warp_hist_add(S.h256, static_cast<uint32_t>((k >> shift) & 255), act);
+      const uint32_t digit = static_cast<uint32_t>((k >> shift) & ((1u << width) - 1));
+      if (AGG) warp_hist_add(S.h256, digit, act);
+      else if (act) atomicAdd(&S.h256[digit], 1u);       // digits below the threshold bin spread out
     }
     __syncthreads();
     if (threadIdx.x < 32) topk_pick_digit(S, remaining);
     __syncthreads();
     if (S.d < 0) { if (threadIdx.x == 0) record_error(kErrSelectCount); return prefix; }
     prefix |= static_cast<uint64_t>(S.d) << shift;
-    bits += 8;
+    bits += width;
     remaining -= S.gt;
     const bool done = (S.eq == remaining) || bits == 64;
     __syncthreads();
@@ -183,7 +193,7 @@ __device__ __forceinline__ void topk_emit(const TopkParams& p, int32_t* out_idx,
   if (out_sc) out_sc[slot] = okey_to_float(static_cast<uint32_t>(k >> 32));
 }
 
-__global__ void __launch_bounds__(kTopkThreads)
+__global__ void __launch_bounds__(kTopkThreads, 1)
 topk_select_kernel(TopkParams p) {
   extern __shared__ __align__(1024) uint8_t topk_smem_raw[];
   TopkShared& S = *reinterpret_cast<TopkShared*>(topk_smem_raw);
@@ -200,8 +210,38 @@ topk_select_kernel(TopkParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
   pdl_launch_dependents();
-  const int64_t nvalid = topk_valid_slots(p, bq);
   const float* row = p.scores + static_cast<int64_t>(bq) * p.ld;
+
+  // this CTA's slice of the visible slots, streamed kTopkChunkSlots at a
+  // time: warp w owns the chunk's slots [1024w, 1024w + 1024) and its lane l
+  // holds the four slots at 128j + 4l (j < kTopkVec) of them
+  // slices split all n_elems slots, so the first loads go out before the
+  // visible count arrives; slots at or past it are masked afterwards
+  const int64_t span = (((p.n_elems + C - 1) / C) + 3) & ~static_cast<int64_t>(3);
+  const int64_t lo = min(p.n_elems, static_cast<int64_t>(rank) * span);
+  int64_t hi = min(p.n_elems, lo + span);
+  const int lane_slot = warp * kTopkWarpSlots + 4 * lane;   // this lane's first slot in a chunk
+  auto load_chunk = [&](int64_t c0, float4 (&x)[kTopkVec]) {
+    const int64_t left = hi - c0 - lane_slot;          // slots of the slice from this lane's first on
+    const float4* src = reinterpret_cast<const float4*>(row + c0 + lane_slot);
+#pragma unroll
+    for (int j = 0; j < kTopkVec; ++j) {
+      x[j] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (128 * j < left) {
+        x[j] = __ldcg(src + 32 * j);
+        const int64_t rem = left - 128 * j;             // slots of this vector inside the slice
+        if (rem < 4) {
+          x[j].w = -INFINITY;
+          if (rem < 3) x[j].z = -INFINITY;
+          if (rem < 2) x[j].y = -INFINITY;
+        }
+      }
+    }
+  };
+  float4 cur[kTopkVec];
+  load_chunk(lo, cur);                                 // in flight while the histogram is read
+  const int64_t nvalid = topk_valid_slots(p, bq);
+  hi = min(hi, nvalid);
 
   // -- 0. threshold bin: thread t owns the `per` bins just below bin
   //       nbins - per*t (descending ranges), read with coalesced loads
@@ -228,15 +268,17 @@ topk_select_kernel(TopkParams p) {
     uint32_t total;
     uint32_t above = topk_block_scan(local, S, &total);   // bins above this thread's range
     need = static_cast<int>(total < static_cast<uint32_t>(p.K) ? total : static_cast<uint32_t>(p.K));
-    if (tid == 0) S.tb = nbins;
+    if (tid == 0) { S.tb = nbins; S.above = 0; }
     __syncthreads();
     if (need > 0 && above < static_cast<uint32_t>(need) && above + local >= static_cast<uint32_t>(need)) {
       bool found = false;
 #pragma unroll
       for (int j = 7; j >= 0; --j) {
         if (j < per && !found) {
+          if (above + c[j] >= static_cast<uint32_t>(need)) {
+            S.tb = lo_bin + j; S.above = static_cast<int>(above); found = true;
+          }
           above += c[j];
-          if (above >= static_cast<uint32_t>(need)) { S.tb = lo_bin + j; found = true; }
         }
       }
     }
@@ -247,81 +289,81 @@ topk_select_kernel(TopkParams p) {
   // -- 1. this CTA's slice: candidates into shared memory, in position order
   uint32_t n = 0;                                     // candidates so far (uniform over the block)
   if (need > 0) {
-    const int64_t span = (((nvalid + C - 1) / C) + 3) & ~static_cast<int64_t>(3);
-    const int64_t lo = min(nvalid, static_cast<int64_t>(rank) * span);
-    const int64_t hi = min(nvalid, lo + span);
-    for (int64_t it = lo; it < hi; it += kTopkIterSlots) {
-      const int64_t wbase = it + static_cast<int64_t>(warp) * kTopkWarpSlots;
-      float v[4][4];
+    const uint32_t lt = (1u << lane) - 1u;             // lanes below this one
+    for (int64_t c0 = lo; c0 < hi; c0 += kTopkChunkSlots) {
+      float4 nxt[kTopkVec];
+      load_chunk(c0 + kTopkChunkSlots, nxt);           // the next chunk's loads overlap this one's work
+      // position order inside the warp is (j, lane, component): four
+      // ballots per j give each lane its offset without a serial scan
+      if (c0 + kTopkChunkSlots > hi) {
+        // the chunk reaches the end of the visible slots: mask the rest
+        const int64_t left = hi - c0 - lane_slot;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t s0 = wbase + 128 * j + 4 * lane;
-        float4 x = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        if (s0 < hi) x = __ldcg(reinterpret_cast<const float4*>(row + s0));
-        v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
-      }
-      // candidate flags and this lane's offset inside the warp's 512 slots
-      uint32_t fl[4], wexcl[4], wtot = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t s0 = wbase + 128 * j + 4 * lane;
-        uint32_t f = 0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) f |= (s0 + c < hi && topk_is_cand(v[j][c], tb, p.hb)) ? (1u << c) : 0u;
-        fl[j] = f;
-        const uint32_t cnt = __popc(f);
-        uint32_t incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
+        for (int j = 0; j < kTopkVec; ++j) {
+          const int64_t rem = left - 128 * j;
+          if (rem < 4) {
+            cur[j].w = -INFINITY;
+            if (rem < 3) cur[j].z = -INFINITY;
+            if (rem < 2) cur[j].y = -INFINITY;
+            if (rem < 1) cur[j].x = -INFINITY;
+          }
         }
-        wexcl[j] = wtot + incl - cnt;
-        wtot += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      uint32_t fl[kTopkVec], pre[kTopkVec], wtot = 0;
+#pragma unroll
+      for (int j = 0; j < kTopkVec; ++j) {
+        const bool f0 = topk_is_cand(cur[j].x, tb, p.hb), f1 = topk_is_cand(cur[j].y, tb, p.hb);
+        const bool f2 = topk_is_cand(cur[j].z, tb, p.hb), f3 = topk_is_cand(cur[j].w, tb, p.hb);
+        const uint32_t b0 = __ballot_sync(0xffffffffu, f0), b1 = __ballot_sync(0xffffffffu, f1);
+        const uint32_t b2 = __ballot_sync(0xffffffffu, f2), b3 = __ballot_sync(0xffffffffu, f3);
+        fl[j] = (f0 ? 1u : 0u) | (f1 ? 2u : 0u) | (f2 ? 4u : 0u) | (f3 ? 8u : 0u);
+        pre[j] = wtot + __popc(b0 & lt) + __popc(b1 & lt) + __popc(b2 & lt) + __popc(b3 & lt);
+        wtot += __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
       }
       uint32_t btot;
       const uint32_t wofs = n + topk_block_scan(lane == 0 ? wtot : 0u, S, &btot);
       const uint32_t wbase_ofs = __shfl_sync(0xffffffffu, wofs, 0);
+      if (wtot != 0) {
+        const int64_t s_lane = c0 + lane_slot;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t o = wbase_ofs + wexcl[j];
-        const int64_t s0 = wbase + 128 * j + 4 * lane;
+        for (int j = 0; j < kTopkVec; ++j) {
+          if (fl[j] == 0) continue;
+          uint32_t o = wbase_ofs + pre[j];
+          const float v[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (fl[j] & (1u << c)) {
-            if (o < static_cast<uint32_t>(kTopkCap)) keys_s[o] = topk_make_key(p, bq, s0 + c, v[j][c]);
-            ++o;
+          for (int c = 0; c < 4; ++c) {
+            if (fl[j] & (1u << c)) {
+              if (o < static_cast<uint32_t>(kTopkCap)) keys_s[o] = topk_make_key(p, bq, s_lane + 128 * j + c, v[c]);
+              ++o;
+            }
           }
         }
       }
       n += btot;
+#pragma unroll
+      for (int j = 0; j < kTopkVec; ++j) cur[j] = nxt[j];
     }
   }
 
-  // -- 2. the cluster's first CTA gathers and selects -------------------------
+  // -- 2. counts to every CTA; the others push their lists into the first
+  //       CTA's shared memory behind its own, in slice (= position) order
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-  if (tid == 0) *cluster.map_shared_rank(&S.cnt[rank], 0) = n;
-  cluster.sync();                                     // counts and candidate lists visible cluster-wide
+  if (tid < C) *cluster.map_shared_rank(&S.cnt[rank], tid) = n;
+  cluster.sync();                                     // counts visible cluster-wide
   bool fits = true;
-  uint32_t n_all = 0;
-  if (rank == 0 && need > 0) {
-    for (int r = 0; r < C; ++r) {
-      const uint32_t c = S.cnt[r];
-      fits = fits && c <= static_cast<uint32_t>(kTopkCap);
-      n_all += c;
-    }
-    fits = fits && n_all <= static_cast<uint32_t>(kTopkCap);
-    if (fits) {
-      uint32_t off = S.cnt[0];
-      for (int r = 1; r < C; ++r) {
-        const uint64_t* remote = cluster.map_shared_rank(keys_s, r);
-        const uint32_t c = S.cnt[r];
-        for (uint32_t i = tid; i < c; i += kTopkThreads) keys_s[off + i] = remote[i];
-        off += c;
-      }
-    }
+  uint32_t n_all = 0, my_off = 0;
+  for (int r = 0; r < C; ++r) {
+    const uint32_t c = S.cnt[r];
+    fits = fits && c <= static_cast<uint32_t>(kTopkCap);
+    if (r < rank) my_off += c;
+    n_all += c;
   }
-  cluster.sync();                                     // the other CTAs' lists are no longer read
+  fits = fits && n_all <= static_cast<uint32_t>(kTopkCap);
+  if (fits && need > 0 && rank > 0) {
+    uint64_t* dst = cluster.map_shared_rank(keys_s, 0) + my_off;
+    for (uint32_t i = tid; i < n; i += kTopkThreads) dst[i] = keys_s[i];
+  }
+  cluster.sync();                                     // the first CTA holds every list; the rest may exit
   if (rank != 0) return;
 
   int32_t* out_idx = p.out_idx + static_cast<int64_t>(bq) * p.K;
@@ -329,7 +371,8 @@ topk_select_kernel(TopkParams p) {
   uint32_t written = 0;
   if (need > 0) {
     if (fits) {
-      const uint64_t P = topk_radix_select(S, n_all, need, [&](int64_t i) { return keys_s[i]; });
+      const uint64_t P = topk_radix_select<false>(S, n_all, need, p.hb, static_cast<uint64_t>(tb) << (64 - p.hb), S.above,
+                                           [&](int64_t i) { return keys_s[i]; });
       // ordered compaction of the keys >= P (4 consecutive keys per thread)
       for (uint32_t i0 = 0; i0 < n_all; i0 += 4 * kTopkThreads) {
         uint64_t k[4];
@@ -350,7 +393,8 @@ topk_select_kernel(TopkParams p) {
       }
     } else {
       // candidates do not fit: select and compact over the scores themselves
-      const uint64_t P = topk_radix_select(S, nvalid, need, [&](int64_t e) { return topk_slot_key(p, bq, e, tb); });
+      const uint64_t P = topk_radix_select<true>(S, nvalid, need, p.hb, static_cast<uint64_t>(tb) << (64 - p.hb), S.above,
+                                           [&](int64_t e) { return topk_slot_key(p, bq, e, tb); });
       for (int64_t e0 = 0; e0 < nvalid; e0 += 4 * kTopkThreads) {
         uint64_t k[4];
         uint32_t m = 0;
@@ -382,11 +426,11 @@ inline size_t topk_smem_bytes() {
 }
 
 // CTAs per selection problem: enough to spread a long score row over SMs
-// (one CTA per 16K slots, at most a portable cluster of 8), fewer once the
-// problems alone fill the GPU twice over.
-inline int topk_cluster_size(int64_t n_elems, int problems, int sms) {
+// (one CTA per 8K slots, at most max_cluster), fewer once the problems
+// alone fill the GPU twice over.
+inline int topk_cluster_size(int64_t n_elems, int problems, int sms, int max_cluster) {
   int c = 1;
-  while (c < kTopkMaxCluster && static_cast<int64_t>(c) * 16384 < n_elems) c <<= 1;
+  while (c < max_cluster && static_cast<int64_t>(c) * 8192 < n_elems) c <<= 1;
   while (c > 1 && static_cast<int64_t>(problems) * c > 2 * static_cast<int64_t>(sms)) c >>= 1;
   return c;
 }
