@@ -76,6 +76,8 @@ def load(path=LIB_PATH):
     lib.csa2_status_string.argtypes = [_c_i32]
     lib.csa2_status_string.restype = ctypes.c_char_p
     lib.csa2_version.restype = _c_i32
+    lib.csa2_cuda_error_string.argtypes = []
+    lib.csa2_cuda_error_string.restype = ctypes.c_char_p
     lib.csa2_trace_begin.argtypes = [_c_i32]
     lib.csa2_trace_get.argtypes = [_c_i32, ctypes.POINTER(_c_i32), ctypes.POINTER(_c_f32)]
     lib.csa2_trace_count.restype = _c_i32
@@ -109,7 +111,14 @@ def _stream(stream):
 
 def _check(status, what):
     if status != 0:
+        if status == 5:                     # CSA2_ERR_CUDA
+            what = f"{what} ({cuda_error_string()})"
         raise Csa2Error(status, what)
+
+
+def cuda_error_string():
+    """The CUDA runtime's description of the last failure behind a CUDA status."""
+    return load().csa2_cuda_error_string().decode()
 
 
 # ---------------------------------------------------------------------------
@@ -128,9 +137,11 @@ def index_args(mode, qI, w, kI, n_vis, idx, scores=None, hsi_blocks=0, hsi_block
     """Build csa2_index_args from tensors: qI [B,Q,32,128], w [B,Q,32],
     kI [B,N,128], n_vis int32 [B,Q], idx int32 [B,Q,K]."""
     B, Q = qI.shape[0], qI.shape[1]
-    return IndexArgs(mode=mode, B=B, Q=Q, K=idx.shape[-1], N=kI.shape[1],
-                     qI=_ptr(qI), w=_ptr(w), kI=_ptr(kI), n_vis=_ptr(n_vis), idx=_ptr(idx), scores=_ptr(scores),
-                     hsi_blocks=hsi_blocks, hsi_block=hsi_block, pool_out=_ptr(pool_out), pool_in=_ptr(pool_in))
+    a = IndexArgs(mode=mode, B=B, Q=Q, K=idx.shape[-1], N=kI.shape[1],
+                  qI=_ptr(qI), w=_ptr(w), kI=_ptr(kI), n_vis=_ptr(n_vis), idx=_ptr(idx), scores=_ptr(scores),
+                  hsi_blocks=hsi_blocks, hsi_block=hsi_block, pool_out=_ptr(pool_out), pool_in=_ptr(pool_in))
+    a._tensors = (qI, w, kI, n_vis, idx, scores, pool_out, pool_in)     # the struct holds raw pointers
+    return a
 
 
 def csa2_index_score_topk(args, ws, stream=None):
@@ -152,10 +163,12 @@ def attn_args(q, kv_fp4, idx, swa, out, lse=None, W=128, swa_step=0, scale=0.0):
     """q [B,Q,64,512], kv_fp4 uint8 [B,N,288], idx int32 [B,Q,K], swa bf16
     [B,rows,512], out bf16 [B,Q,64,512], lse f32 [B,Q,64]."""
     B, Q = q.shape[0], q.shape[1]
-    return AttnArgs(B=B, Q=Q, K=idx.shape[-1] if idx is not None else 0, W=W, N=kv_fp4.shape[1],
-                    q=_ptr(q), kv_fp4=_ptr(kv_fp4), idx=_ptr(idx), swa=_ptr(swa),
-                    swa_rows=swa.shape[1] if swa is not None else 0, swa_step=swa_step, scale=scale,
-                    out=_ptr(out), lse=_ptr(lse))
+    a = AttnArgs(B=B, Q=Q, K=idx.shape[-1] if idx is not None else 0, W=W, N=kv_fp4.shape[1],
+                 q=_ptr(q), kv_fp4=_ptr(kv_fp4), idx=_ptr(idx), swa=_ptr(swa),
+                 swa_rows=swa.shape[1] if swa is not None else 0, swa_step=swa_step, scale=scale,
+                 out=_ptr(out), lse=_ptr(lse))
+    a._tensors = (q, kv_fp4, idx, swa, out, lse)     # the struct holds raw pointers
+    return a
 
 
 def csa2_sparse_attn(args, ws, stream=None):
@@ -179,6 +192,8 @@ def group_args(B, Q, K, W, N, n_vis, kI, kv_fp4, layers, kv_new=None, new_rows=N
                   pool=_ptr(pool), scale=scale, n_layers=len(layers),
                   layers=ctypes.cast(arr, ctypes.POINTER(Layer)))
     g._layer_array = arr
+    # the structs hold raw pointers: keep every tensor alive with them
+    g._tensors = (n_vis, kI, kv_fp4, kv_new, new_rows, pool, [dict(L) for L in layers])
     return g
 
 

@@ -2,11 +2,11 @@
 // cores ("DeepSeek V4.1-Flash 技术报告深度解析" §3.2 attention, §3.4
 // dequantise before the attention math).
 //
-// One CTA per (128-key slice, query).  The slice's keys (FP4 entries, each
-// 288-byte row fetched by one bulk copy and dequantised by the CTA's
-// threads, or window rows brought by TMA) form a
-// 128 x 512 bf16 tile K in shared memory, stored K-major with the 128-byte
-// swizzle.  The query's 64 heads form Q (64 x 512, TMA).  Then:
+// One CTA (512 threads) per (128-key slice, query).  The slice's keys (FP4
+// entries, each 288-byte row fetched by one bulk copy and dequantised by the
+// CTA's threads, or window rows brought by TMA) form a 128 x 512 bf16 tile
+// K in shared memory, stored K-major with the 128-byte swizzle.  The
+// query's 64 heads form Q (64 x 512, TMA).  Then:
 //   MMA 1   S^T[key, head] = K . Q^T            M = 128 keys, N = 64, K = 512
 //   softmax per head over the slice's keys (fp32, from TMEM via shared
 //           memory), P^T[head, key] = exp2(S^T - max) rounded to bf16 and
@@ -24,12 +24,14 @@
 
 namespace csa2 {
 
-constexpr int kTcAttnThreads = 256;
+constexpr int kTcAttnThreads = 512;
+constexpr int kTcAttnWarps = kTcAttnThreads / 32;
 constexpr int kTcAttnKeys = 128;                       // keys per slice (MMA M)
 constexpr uint32_t kTcKeyTileBytes = 128 * 512 * 2;    // 128 KB: 8 chunks of [128 rows x 64 dims]
 constexpr uint32_t kTcQTileBytes = 64 * 512 * 2;       // 64 KB: 8 chunks of [64 rows x 64 dims]
 constexpr int kTcSPitch = kTcAttnKeys + 4;             // fp32 row pitch of the transposed scores
-constexpr uint32_t kTcAttnSmem = kTcKeyTileBytes + kTcQTileBytes + 2048 + 1024;
+constexpr uint32_t kTcMiscBytes = 2048;
+constexpr uint32_t kTcAttnSmem = kTcKeyTileBytes + kTcQTileBytes + kTcMiscBytes + 1024;
 
 struct TcAttnParams {
   int B, Q, K, W;
@@ -110,7 +112,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                                         // [3] FP4 row gather
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* valid_s = reinterpret_cast<int*>(tmem_slot + 4);   // [128]
+  int* valid_s = reinterpret_cast<int*>(misc + 64);                  // [128]
 
   const int slice = blockIdx.x, bq = blockIdx.y;
   const int b = bq / p.Q, qi = bq % p.Q;
@@ -224,22 +226,21 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     umma_commit(&bars[1]);
   }
 
-  // ---- scores: TMEM -> scaled, masked, transposed into shared memory
-  if (warp < 4) {
+  // ---- scores: TMEM -> scaled, masked, transposed into shared memory.
+  //      Warp w reads TMEM lanes 32(w%4).. (its keys) and heads 16(w/4)..
+  {
     const bool ok = mbar_wait(&bars[1], 0, kErrWaitTmemFull, abort_flag);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
-      const int key = warp * 32 + lane;
+      const int quarter = warp & 3, hg = warp >> 2;
+      const int key = quarter * 32 + lane;
       const bool kv_ok = valid_s[key] != 0;
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 16 * hg, r);
+      tmem_ld_wait();
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 32 * hh, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          st[(32 * hh + j) * kTcSPitch + key] = kv_ok ? __uint_as_float(r[j]) * p.scale_log2 : -INFINITY;
-      }
+      for (int j = 0; j < 16; ++j)
+        st[(16 * hg + j) * kTcSPitch + key] = kv_ok ? __uint_as_float(r[j]) * p.scale_log2 : -INFINITY;
     }
   }
   tc_fence_before();
@@ -247,18 +248,19 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
   // ---- softmax statistics per head; P^T in bf16 as the K-major B operand
   {
-    const int h = tid >> 2, part = tid & 3;               // 4 threads per head, 32 keys each
-    const float* srow = st + h * kTcSPitch + part * 32;
+    const int h = tid >> 3, part = tid & 7;               // 8 threads per head, 16 keys each
+    const float* srow = st + h * kTcSPitch + part * 16;
     float m = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) m = fmaxf(m, srow[j]);
+    for (int j = 0; j < 16; ++j) m = fmaxf(m, srow[j]);
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
     const float mu = (m == -INFINITY) ? 0.0f : m;
     float l = 0.0f;
-    uint32_t pk[16];
+    uint32_t pk[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < 8; ++j) {
       const __nv_bfloat162 v = __floats2bfloat162_rn(exp2f(srow[2 * j] - mu), exp2f(srow[2 * j + 1] - mu));
       const float2 f = __bfloat1622float2(v);
       l += f.x + f.y;
@@ -266,12 +268,13 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     }
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
     __syncthreads();                                      // every thread has read the scores it needs
-    // keys part*32 .. part*32+31 = chunk part/2, units 4(part&1)..4(part&1)+3 of row h
-    uint8_t* chunk = pt + (part >> 1) * 8192;
+    // keys 16part .. 16part+15 = chunk part/4, units 2(part&3), 2(part&3)+1 of row h
+    uint8_t* chunk = pt + (part >> 2) * 8192;
 #pragma unroll
-    for (int t = 0; t < 4; ++t)
-      *reinterpret_cast<uint4*>(chunk + sw128_off(h, 4 * (part & 1) + t)) =
+    for (int t = 0; t < 2; ++t)
+      *reinterpret_cast<uint4*>(chunk + sw128_off(h, 2 * (part & 3) + t)) =
           make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
     if (part == 0) {
       float* ml = p.ml + ((static_cast<int64_t>(bq) * p.slices + slice) * 64 + h) * 2;
@@ -302,42 +305,37 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     umma_commit(&bars[2]);
   }
 
-  // ---- epilogue: O^T tiles -> shared [head][dim] (the key tile is free
-  //      now) -> the 128 KB partial output
+  // ---- epilogue: O^T tile (warp / 4), dims 32(warp % 4).. -> shared
+  //      [head][dim] (the key tile is free now)
   float* obuf = reinterpret_cast<float*>(kt);
   {
     const bool ok = mbar_wait(&bars[2], 0, kErrWaitTmemFull, abort_flag);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
-      const int quarter = warp & 3;
-#pragma unroll 1
-      for (int t = warp >> 2; t < 4; t += 2) {
-        const int d = 128 * t + 32 * quarter + lane;
+      const int quarter = warp & 3, t = warp >> 2;
+      const int d = 128 * t + 32 * quarter + lane;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64 + 64 * t + 32 * hh, r);
-          tmem_ld_wait();
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64 + 64 * t + 32 * hh, r);
+        tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) obuf[(32 * hh + j) * 512 + d] = __uint_as_float(r[j]);
-        }
+        for (int j = 0; j < 32; ++j) obuf[(32 * hh + j) * 512 + d] = __uint_as_float(r[j]);
       }
     }
-    fence_async_smem();
   }
   tc_fence_before();
   __syncthreads();
+  if (warp == 1) {                                      // TMEM is no longer read: free it early
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+
   if (!*abort_flag) {
     float4* op = reinterpret_cast<float4*>(p.opart + (static_cast<int64_t>(bq) * p.slices + slice) * 64 * 512);
     const float4* src = reinterpret_cast<const float4*>(obuf);
-#pragma unroll 8
+#pragma unroll 4
     for (int j = tid; j < 64 * 512 / 4; j += kTcAttnThreads) op[j] = src[j];
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -32,6 +32,8 @@ static LaunchTrace g_trace;
 // cluster_x > 0 adds a (cluster_x, 1, 1) thread-block cluster shape.
 // Tracing records events between launches, which serialises them as usual.
 static bool g_pdl = true;
+// last CUDA failure seen by a launch on this host thread (csa2_cuda_error_string)
+static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                              unsigned cluster_x, Args... args) {
@@ -57,8 +59,10 @@ inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-  return e != cudaSuccess ? e : cudaGetLastError();
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) g_last_cuda_error = e;
+  return e;
 }
 
 inline void trace_pre(int kid, cudaStream_t st) {
@@ -263,6 +267,14 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() {

@@ -59,21 +59,21 @@ cudaError_t set_scan_attrs() {
 inline int scan_qg(int qg) { return qg <= 1 ? 1 : qg <= 2 ? 2 : qg <= 4 ? 4 : 8; }
 
 template <int QG, bool HSI>
-void launch_scan_t(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk, const CUtensorMap& tq,
-                   const ScanParams& sp) {
-  launch_ex(index_scan_kernel<QG, HSI>, dim3(grid), dim3(kScanThreads), smem, st, 0, tk, tq, sp);
+cudaError_t launch_scan_t(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk, const CUtensorMap& tq,
+                          const ScanParams& sp) {
+  return launch_ex(index_scan_kernel<QG, HSI>, dim3(grid), dim3(kScanThreads), smem, st, 0, tk, tq, sp);
 }
-void launch_scan(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
-                 const CUtensorMap& tq, const ScanParams& sp) {
+cudaError_t launch_scan(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
+                        const CUtensorMap& tq, const ScanParams& sp) {
   switch (QG * 2 + (hsi ? 1 : 0)) {
-    case 2: launch_scan_t<1, false>(grid, smem, st, tk, tq, sp); break;
-    case 3: launch_scan_t<1, true>(grid, smem, st, tk, tq, sp); break;
-    case 4: launch_scan_t<2, false>(grid, smem, st, tk, tq, sp); break;
-    case 5: launch_scan_t<2, true>(grid, smem, st, tk, tq, sp); break;
-    case 8: launch_scan_t<4, false>(grid, smem, st, tk, tq, sp); break;
-    case 9: launch_scan_t<4, true>(grid, smem, st, tk, tq, sp); break;
-    case 16: launch_scan_t<8, false>(grid, smem, st, tk, tq, sp); break;
-    default: launch_scan_t<8, true>(grid, smem, st, tk, tq, sp); break;
+    case 2: return launch_scan_t<1, false>(grid, smem, st, tk, tq, sp);
+    case 3: return launch_scan_t<1, true>(grid, smem, st, tk, tq, sp);
+    case 4: return launch_scan_t<2, false>(grid, smem, st, tk, tq, sp);
+    case 5: return launch_scan_t<2, true>(grid, smem, st, tk, tq, sp);
+    case 8: return launch_scan_t<4, false>(grid, smem, st, tk, tq, sp);
+    case 9: return launch_scan_t<4, true>(grid, smem, st, tk, tq, sp);
+    case 16: return launch_scan_t<8, false>(grid, smem, st, tk, tq, sp);
+    default: return launch_scan_t<8, true>(grid, smem, st, tk, tq, sp);
   }
 }
 
@@ -160,6 +160,7 @@ bool make_map_bf16_128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t
 struct IndexPlan {
   bool pool, hsi;
   int BQ, qg, hb;
+  int hist_every;      // 1: exact score histogram; 8: every 8th tile (many queries per MMA group)
   int64_t n_elems, nblk;
   int64_t ld, bld;     // score row strides (multiples of 4 for 16-byte loads)
   // counter region (histograms): zeroed at the start of every call; data
@@ -198,7 +199,12 @@ IndexPlan plan_index(const csa2_index_args* a) {
   P.hsi = a->mode == CSA2_FULL && a->hsi_blocks > 0;
   P.BQ = a->B * a->Q;
   P.qg = P.pool ? 1 : std::min(a->Q, 8);
-  P.hb = (P.qg <= 2) ? 12 : 10;
+  // score histogram bits: 4096 bins per query for 1-2 queries per MMA group,
+  // 2048 for 4-8 (1024 with HSI, whose block histogram needs the room too)
+  P.hb = (P.qg <= 2) ? 12 : (P.hsi ? 10 : 11);
+  // with 4+ queries per group the histogram increments cost a quarter of the
+  // scan: count one tile in 8 and let the top-K verify its threshold
+  P.hist_every = (P.qg >= 4 && !P.hsi) ? 8 : 1;
   P.n_elems = P.pool ? static_cast<int64_t>(a->hsi_blocks) * 8 : a->N;
   P.nblk = P.hsi ? (a->N + 7) / 8 : 0;
   P.ld = (P.n_elems + 3) & ~static_cast<int64_t>(3);
@@ -226,8 +232,26 @@ cudaError_t launch_topk(const TopkParams& tp, int problems, const DeviceInfo& de
   return e;
 }
 
+// CTAs sharing one MMA group's tile range: the split whose waves of one
+// CTA per SM finish first, counting about four tiles of set-up per CTA.
+// Few groups (decode) get one wave over every SM; many groups (prefill) get
+// pieces that keep the last wave nearly full.
+int scan_ctas_per_group(int groups, int tiles, int sms) {
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int c = 1; c <= std::min(tiles, 4096); ++c) {
+    const int64_t waves = (static_cast<int64_t>(groups) * c + sms - 1) / sms;
+    const int64_t cost = waves * ((tiles + c - 1) / c + 4);
+    if (cost < best_cost) { best_cost = cost; best = c; }
+  }
+  return best;
+}
+
 // zero: the call's counter region (already zeroed); data: its data region
-csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zero, void* data, cudaStream_t st) {
+// kv_prefetch: optional FP4 cache whose selected rows are pulled into L2 as
+// the top-K writes their indices (the group call's attention reads them next)
+csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zero, void* data, cudaStream_t st,
+                      const void* kv_prefetch = nullptr) {
   const IndexPlan P = plan_index(a);
   uint8_t* z = static_cast<uint8_t*>(zero);
   uint8_t* w = static_cast<uint8_t*>(data);
@@ -245,10 +269,11 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.hist = reinterpret_cast<uint32_t*>(z + P.off_hist);
   sp.bhist = P.hsi ? reinterpret_cast<uint32_t*>(z + P.off_bhist) : nullptr;
   sp.hb = P.hb;
+  sp.hist_every = P.hist_every;
   sp.qblocks = P.pool ? 1 : (a->Q + P.qg - 1) / P.qg;
   sp.groups = P.pool ? P.BQ : a->B * sp.qblocks;
   sp.tiles_per_group = static_cast<int>((P.n_elems + kTileRows - 1) / kTileRows);
-  sp.ctas_per_group = std::max(1, std::min(sp.tiles_per_group, dev.sms / sp.groups));
+  sp.ctas_per_group = scan_ctas_per_group(sp.groups, sp.tiles_per_group, dev.sms);
   const int QG = scan_qg(P.qg);
   const uint32_t n_mma = 32u * QG;
   uint32_t cols = 32;
@@ -267,9 +292,9 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
 
   const unsigned grid = static_cast<unsigned>(sp.groups * sp.ctas_per_group);
   trace_pre(kKIndexScan, st);
-  launch_scan(QG, P.hsi, grid, L.total + 1024, st, tk, tq, sp);
+  const cudaError_t es = launch_scan(QG, P.hsi, grid, L.total + 1024, st, tk, tq, sp);
   trace_post(st);
-  if (cudaGetLastError() != cudaSuccess) return CSA2_ERR_CUDA;
+  if (es != cudaSuccess) return CSA2_ERR_CUDA;
 
   TopkParams tp;
   memset(&tp, 0, sizeof(tp));
@@ -282,9 +307,13 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   tp.pool_blocks = sp.pool_blocks;
   tp.hist = sp.hist;
   tp.hb = P.hb;
+  tp.hist_sample = P.hist_every;
   tp.K = a->K;
   tp.out_idx = a->idx;
   tp.out_scores = a->scores;
+  tp.prefetch_kv = static_cast<const uint8_t*>(kv_prefetch);
+  tp.prefetch_N = a->N;
+  tp.Q = a->Q;
   if (launch_topk(tp, P.BQ, dev, st) != cudaSuccess) return CSA2_ERR_CUDA;
 
   if (P.hsi) {
@@ -296,9 +325,11 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
     bp.vis_div = 8;
     bp.pool = nullptr;
     bp.hist = sp.bhist;
+    bp.hist_sample = 1;
     bp.K = a->hsi_blocks;
     bp.out_idx = a->pool_out;
     bp.out_scores = nullptr;
+    bp.prefetch_kv = nullptr;
     if (launch_topk(bp, P.BQ, dev, st) != cudaSuccess) return CSA2_ERR_CUDA;
   }
   return CSA2_OK;
@@ -549,7 +580,7 @@ csa2_status csa2_group_decode(const csa2_group_args* g, void* ws, size_t ws_byte
     const csa2_layer& L = g->layers[i];
     if (L.mode != CSA2_REUSE) {
       const csa2_index_args a = layer_index_args(g, L);
-      s = run_index(&a, *dev, zws, dws, st);
+      s = run_index(&a, *dev, zws, dws, st, g->kv_fp4);
       if (s != CSA2_OK) return s;
       zws += plan_index(&a).zero_bytes;
       last_idx = L.idx;
@@ -594,6 +625,8 @@ csa2_status csa2_device_status(int32_t* code, void* stream) {
   }
   return CSA2_OK;
 }
+
+const char* csa2_cuda_error_string(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char* csa2_status_string(int32_t s) {
   switch (s) {

@@ -56,6 +56,7 @@ struct ScanParams {
   uint32_t* hist;         // [B*Q][1 << hb]       (zero at launch)
   uint32_t* bhist;        // scan with HSI: [B*Q][1 << hb]
   int hb;                 // histogram bits
+  int hist_every;         // the score histogram counts tiles with tile % hist_every == 0
   int groups;             // B*qblocks (scan) or B*Q (pool)
   int tiles_per_group;
   int ctas_per_group;
@@ -279,7 +280,8 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
           if (!valid) s = -INFINITY;
           const bool in_range = e < p.n_elems && q < qn;
           if (in_range) p.scores[static_cast<int64_t>(bq0 + q) * p.ld + e] = s;
-          warp_hist_add(hist_s + q * nbins, okey(s) >> (32 - p.hb), in_range && valid);
+          if (tile % p.hist_every == 0)                 // uniform over the warp
+            warp_hist_add(hist_s + q * nbins, okey(s) >> (32 - p.hb), in_range && valid);
           if (HSI) {
             float m = s;
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));

@@ -35,9 +35,10 @@ namespace cg = cooperative_groups;
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkVec = 8;                                  // float4 per lane per chunk
-constexpr int kTopkWarpSlots = 32 * 4 * kTopkVec;            // 1024 contiguous slots per warp per chunk
-constexpr int kTopkChunkSlots = kTopkWarps * kTopkWarpSlots; // 16384 slots per CTA per chunk
+constexpr int kTopkVec = 4;                                  // float4 per lane per chunk
+constexpr int kTopkWarpSlots = 32 * 4 * kTopkVec;            // 512 contiguous slots per warp per chunk
+constexpr int kTopkChunkSlots = kTopkWarps * kTopkWarpSlots; // 8192 slots (32 KB) per chunk
+constexpr int kTopkStages = 3;                               // chunks in flight (bulk copies into shared memory)
 constexpr int kTopkCap = 12288;                             // candidate keys a CTA holds (the cluster's total)
 constexpr int kTopkMaxCluster = 16;                         // 16 needs the non-portable cluster attribute
 
@@ -51,9 +52,15 @@ struct TopkParams {
   int pool_blocks;
   const uint32_t* hist;     // [BQ][1 << hb] score histogram from the scan
   int hb;
+  int hist_sample;          // 1: exact histogram; s > 1: it counts one tile in s, so the threshold
+                            // is an estimate (with a margin on the count), checked against the
+                            // exact candidate count before it is used
   int K;
   int32_t* out_idx;         // [BQ][K]
   float* out_scores;        // optional [BQ][K]
+  const uint8_t* prefetch_kv;  // optional [B][prefetch_N][288]: FP4 rows the attention reads next,
+  int64_t prefetch_N;          // pulled into L2 as their indices are written
+  int Q;                       // queries per batch row (bq / Q = batch row)
 };
 
 struct TopkShared {
@@ -61,6 +68,8 @@ struct TopkShared {
   uint32_t warp_tot[kTopkWarps];
   uint32_t cnt[kTopkMaxCluster];   // candidates found by each CTA of the cluster
   int d, gt, eq, total, tb, above;  // above: visible slots in bins higher than tb
+  int abort_flag;
+  alignas(8) uint64_t full_bar[kTopkStages];
 };
 
 __device__ __forceinline__ int64_t topk_valid_slots(const TopkParams& p, int bq) {
@@ -186,11 +195,28 @@ __device__ uint64_t topk_radix_select(TopkShared& S, int64_t n, int need, int bi
   }
 }
 
-__device__ __forceinline__ void topk_emit(const TopkParams& p, int32_t* out_idx, float* out_sc, uint32_t slot,
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" :: "l"(ptr));
+}
+
+__device__ __forceinline__ void topk_emit(const TopkParams& p, int bq, int32_t* out_idx, float* out_sc, uint32_t slot,
                                           uint64_t k) {
   if (slot >= static_cast<uint32_t>(p.K)) return;
-  out_idx[slot] = static_cast<int32_t>(~static_cast<uint32_t>(k));
+  const int32_t pos = static_cast<int32_t>(~static_cast<uint32_t>(k));
+  out_idx[slot] = pos;
   if (out_sc) out_sc[slot] = okey_to_float(static_cast<uint32_t>(k >> 32));
+  if (p.prefetch_kv && pos >= 0 && pos < p.prefetch_N) {
+    // the 288-byte row spans three or four 128-byte lines
+    const uint8_t* row = p.prefetch_kv + (static_cast<int64_t>(bq / p.Q) * p.prefetch_N + pos) * 288;
+    prefetch_l2(row);
+    prefetch_l2(row + 128);
+    prefetch_l2(row + 256);
+    prefetch_l2(row + 287);
+  }
+}
+
+__device__ __forceinline__ void fence_async_smem_generic() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(kTopkThreads, 1)
@@ -211,35 +237,33 @@ topk_select_kernel(TopkParams p) {
   pdl_wait();
   pdl_launch_dependents();
   const float* row = p.scores + static_cast<int64_t>(bq) * p.ld;
+  float* stage_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(keys_s) + static_cast<size_t>(kTopkCap) * 8);
 
-  // this CTA's slice of the visible slots, streamed kTopkChunkSlots at a
-  // time: warp w owns the chunk's slots [1024w, 1024w + 1024) and its lane l
-  // holds the four slots at 128j + 4l (j < kTopkVec) of them
-  // slices split all n_elems slots, so the first loads go out before the
-  // visible count arrives; slots at or past it are masked afterwards
+  // this CTA's slice of the slots, streamed kTopkChunkSlots at a time by
+  // bulk copies into a kTopkStages-deep ring of shared memory; warp w reads
+  // the chunk's slots [512w, 512w + 512), lane l the four at 128j + 4l.
+  // Slices split all n_elems slots, so the first copies go out before the
+  // visible count arrives; slots at or past it are masked afterwards.
   const int64_t span = (((p.n_elems + C - 1) / C) + 3) & ~static_cast<int64_t>(3);
   const int64_t lo = min(p.n_elems, static_cast<int64_t>(rank) * span);
   int64_t hi = min(p.n_elems, lo + span);
-  const int lane_slot = warp * kTopkWarpSlots + 4 * lane;   // this lane's first slot in a chunk
-  auto load_chunk = [&](int64_t c0, float4 (&x)[kTopkVec]) {
-    const int64_t left = hi - c0 - lane_slot;          // slots of the slice from this lane's first on
-    const float4* src = reinterpret_cast<const float4*>(row + c0 + lane_slot);
-#pragma unroll
-    for (int j = 0; j < kTopkVec; ++j) {
-      x[j] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      if (128 * j < left) {
-        x[j] = __ldcg(src + 32 * j);
-        const int64_t rem = left - 128 * j;             // slots of this vector inside the slice
-        if (rem < 4) {
-          x[j].w = -INFINITY;
-          if (rem < 3) x[j].z = -INFINITY;
-          if (rem < 2) x[j].y = -INFINITY;
-        }
-      }
-    }
+  const int64_t hi_copy = hi;                          // copies stay inside the slice's padded row
+  auto issue_chunk = [&](int64_t c0, int k) {          // thread 0: chunk at slot c0 into stage k % kTopkStages
+    if (c0 >= hi_copy) return;
+    const int st = k % kTopkStages;
+    const uint32_t n4 = static_cast<uint32_t>(min(static_cast<int64_t>(kTopkChunkSlots), hi_copy - c0) + 3) & ~3u;
+    mbar_arrive_expect_tx(&S.full_bar[st], n4 * 4);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(stage_s + st * kTopkChunkSlots)), "l"(row + c0), "r"(n4 * 4), "r"(smem_u32(&S.full_bar[st]))
+        : "memory");
   };
-  float4 cur[kTopkVec];
-  load_chunk(lo, cur);                                 // in flight while the histogram is read
+  if (tid == 0) {
+    for (int k = 0; k < kTopkStages; ++k) mbar_init(&S.full_bar[k], 1);
+    S.abort_flag = 0;
+    fence_barrier_init();
+    for (int k = 0; k < kTopkStages; ++k) issue_chunk(lo + static_cast<int64_t>(k) * kTopkChunkSlots, k);
+  }
   const int64_t nvalid = topk_valid_slots(p, bq);
   hi = min(hi, nvalid);
 
@@ -248,7 +272,7 @@ topk_select_kernel(TopkParams p) {
   int need;
   {
     const int nbins = 1 << p.hb;
-    const int per = nbins / kTopkThreads;             // 8 (12-bit) or 2 (10-bit)
+    const int per = nbins / kTopkThreads;             // 8 (12-bit), 4 (11-bit) or 2 (10-bit)
     const uint32_t* hq = p.hist + static_cast<int64_t>(bq) * nbins;
     const int lo_bin = nbins - per * (tid + 1);
     uint32_t c[8];
@@ -256,6 +280,11 @@ topk_select_kernel(TopkParams p) {
       const uint4 v0 = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin));
       const uint4 v1 = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin) + 1);
       c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w; c[4] = v1.x; c[5] = v1.y; c[6] = v1.z; c[7] = v1.w;
+    } else if (per == 4) {
+      const uint4 v0 = __ldcg(reinterpret_cast<const uint4*>(hq + lo_bin));
+      c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w;
+#pragma unroll
+      for (int j = 4; j < 8; ++j) c[j] = 0;
     } else {
       const uint2 v0 = __ldcg(reinterpret_cast<const uint2*>(hq + lo_bin));
       c[0] = v0.x; c[1] = v0.y;
@@ -267,16 +296,28 @@ topk_select_kernel(TopkParams p) {
     for (int j = 0; j < 8; ++j) local += c[j];
     uint32_t total;
     uint32_t above = topk_block_scan(local, S, &total);   // bins above this thread's range
-    need = static_cast<int>(total < static_cast<uint32_t>(p.K) ? total : static_cast<uint32_t>(p.K));
-    if (tid == 0) { S.tb = nbins; S.above = 0; }
+    // target: the suffix count the threshold bin must reach
+    uint32_t target;
+    if (p.hist_sample == 1) {
+      need = static_cast<int>(total < static_cast<uint32_t>(p.K) ? total : static_cast<uint32_t>(p.K));
+      target = static_cast<uint32_t>(need);
+    } else {
+      // a quarter more than the expected sampled count, plus 8 (about three
+      // standard deviations of the sample at K = 512, s = 8)
+      need = static_cast<int>(min(static_cast<int64_t>(p.K), nvalid));
+      target = static_cast<uint32_t>((5 * need + 4 * p.hist_sample - 1) / (4 * p.hist_sample)) + 8;
+    }
+    if (tid == 0) { S.tb = (p.hist_sample == 1) ? nbins : 0; S.above = 0; }
     __syncthreads();
-    if (need > 0 && above < static_cast<uint32_t>(need) && above + local >= static_cast<uint32_t>(need)) {
+    if (need > 0 && above < target && above + local >= target) {
       bool found = false;
 #pragma unroll
       for (int j = 7; j >= 0; --j) {
         if (j < per && !found) {
-          if (above + c[j] >= static_cast<uint32_t>(need)) {
-            S.tb = lo_bin + j; S.above = static_cast<int>(above); found = true;
+          if (above + c[j] >= target) {
+            S.tb = lo_bin + j;
+            S.above = static_cast<int>(above);
+            found = true;
           }
           above += c[j];
         }
@@ -288,27 +329,31 @@ topk_select_kernel(TopkParams p) {
 
   // -- 1. this CTA's slice: candidates into shared memory, in position order
   uint32_t n = 0;                                     // candidates so far (uniform over the block)
-  if (need > 0) {
+  {
     const uint32_t lt = (1u << lane) - 1u;             // lanes below this one
-    for (int64_t c0 = lo; c0 < hi; c0 += kTopkChunkSlots) {
-      float4 nxt[kTopkVec];
-      load_chunk(c0 + kTopkChunkSlots, nxt);           // the next chunk's loads overlap this one's work
-      // position order inside the warp is (j, lane, component): four
-      // ballots per j give each lane its offset without a serial scan
-      if (c0 + kTopkChunkSlots > hi) {
-        // the chunk reaches the end of the visible slots: mask the rest
-        const int64_t left = hi - c0 - lane_slot;
+    const int lane_slot = warp * kTopkWarpSlots + 4 * lane;   // this lane's first slot in a chunk
+    int k = 0;
+    for (int64_t c0 = lo; c0 < hi; c0 += kTopkChunkSlots, ++k) {
+      const int st = k % kTopkStages;
+      const bool ok = mbar_wait(&S.full_bar[st], (k / kTopkStages) & 1, kErrWaitOperand, &S.abort_flag);
+      float4 cur[kTopkVec];
+      const int64_t left = hi - c0 - lane_slot;        // visible slots from this lane's first on
+      const float4* src = reinterpret_cast<const float4*>(stage_s + st * kTopkChunkSlots + lane_slot);
 #pragma unroll
-        for (int j = 0; j < kTopkVec; ++j) {
-          const int64_t rem = left - 128 * j;
+      for (int j = 0; j < kTopkVec; ++j) {
+        cur[j] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        const int64_t rem = left - 128 * j;
+        if (ok && need > 0 && rem > 0) {
+          cur[j] = src[32 * j];
           if (rem < 4) {
             cur[j].w = -INFINITY;
             if (rem < 3) cur[j].z = -INFINITY;
             if (rem < 2) cur[j].y = -INFINITY;
-            if (rem < 1) cur[j].x = -INFINITY;
           }
         }
       }
+      // position order inside the warp is (j, lane, component): four
+      // ballots per j give each lane its offset without a serial scan
       uint32_t fl[kTopkVec], pre[kTopkVec], wtot = 0;
 #pragma unroll
       for (int j = 0; j < kTopkVec; ++j) {
@@ -322,6 +367,11 @@ topk_select_kernel(TopkParams p) {
       }
       uint32_t btot;
       const uint32_t wofs = n + topk_block_scan(lane == 0 ? wtot : 0u, S, &btot);
+      // every thread holds its values: the stage can be refilled
+      if (tid == 0) {
+        fence_async_smem_generic();
+        issue_chunk(c0 + static_cast<int64_t>(kTopkStages) * kTopkChunkSlots, k + kTopkStages);
+      }
       const uint32_t wbase_ofs = __shfl_sync(0xffffffffu, wofs, 0);
       if (wtot != 0) {
         const int64_t s_lane = c0 + lane_slot;
@@ -340,8 +390,15 @@ topk_select_kernel(TopkParams p) {
         }
       }
       n += btot;
-#pragma unroll
-      for (int j = 0; j < kTopkVec; ++j) cur[j] = nxt[j];
+    }
+    // copies issued past the visible end (speculatively) land before exit
+    if (tid == 0) {
+      const int64_t kcopy = (hi_copy - lo + kTopkChunkSlots - 1) / kTopkChunkSlots;   // chunks in the slice
+      const int64_t kissued = min(kcopy, static_cast<int64_t>(k) + kTopkStages);
+      volatile int keep_waiting = 0;                   // bounded even after an earlier wait gave up
+      for (int64_t kk = k; kk < kissued; ++kk)
+        mbar_wait(&S.full_bar[kk % kTopkStages], static_cast<uint32_t>((kk / kTopkStages) & 1), kErrWaitOperand,
+                  &keep_waiting);
     }
   }
 
@@ -369,10 +426,16 @@ topk_select_kernel(TopkParams p) {
   int32_t* out_idx = p.out_idx + static_cast<int64_t>(bq) * p.K;
   float* out_sc = p.out_scores ? p.out_scores + static_cast<int64_t>(bq) * p.K : nullptr;
   uint32_t written = 0;
+  // an estimated threshold holds when at least `need` keys sit at or above it
+  if (p.hist_sample != 1 && n_all < static_cast<uint32_t>(need)) fits = false;
   if (need > 0) {
     if (fits) {
-      const uint64_t P = topk_radix_select<false>(S, n_all, need, p.hb, static_cast<uint64_t>(tb) << (64 - p.hb), S.above,
-                                           [&](int64_t i) { return keys_s[i]; });
+      uint64_t P;
+      if (p.hist_sample == 1)
+        P = topk_radix_select<false>(S, n_all, need, p.hb, static_cast<uint64_t>(tb) << (64 - p.hb), S.above,
+                                     [&](int64_t i) { return keys_s[i]; });
+      else    // the K-th key's bin is unknown: full-width passes, equal digits aggregated
+        P = topk_radix_select<true>(S, n_all, need, 0, 0, 0, [&](int64_t i) { return keys_s[i]; });
       // ordered compaction of the keys >= P (4 consecutive keys per thread)
       for (uint32_t i0 = 0; i0 < n_all; i0 += 4 * kTopkThreads) {
         uint64_t k[4];
@@ -388,20 +451,34 @@ topk_select_kernel(TopkParams p) {
         uint32_t o = written + topk_block_scan(m, S, &tot);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (k[i] != 0) topk_emit(p, out_idx, out_sc, o++, k[i]);
+          if (k[i] != 0) topk_emit(p, bq, out_idx, out_sc, o++, k[i]);
         written += tot;
       }
     } else {
-      // candidates do not fit: select and compact over the scores themselves
-      const uint64_t P = topk_radix_select<true>(S, nvalid, need, p.hb, static_cast<uint64_t>(tb) << (64 - p.hb), S.above,
-                                           [&](int64_t e) { return topk_slot_key(p, bq, e, tb); });
-      for (int64_t e0 = 0; e0 < nvalid; e0 += 4 * kTopkThreads) {
+      // candidates do not fit (or an estimated threshold failed): select
+      // and compact over the scores themselves.  With an estimate, every
+      // visible finite score takes part and `need` is counted exactly.
+      const int tbf = (p.hist_sample == 1) ? tb : 0;
+      uint64_t P;
+      if (p.hist_sample == 1) {
+        P = topk_radix_select<true>(S, nvalid, need, p.hb, static_cast<uint64_t>(tb) << (64 - p.hb), S.above,
+                                    [&](int64_t e) { return topk_slot_key(p, bq, e, tbf); });
+      } else {
+        uint32_t cnt = 0;
+        for (int64_t e = tid; e < nvalid; e += kTopkThreads) cnt += (row[e] != -INFINITY);
+        uint32_t tot;
+        topk_block_scan(cnt, S, &tot);
+        need = static_cast<int>(min(tot, static_cast<uint32_t>(p.K)));
+        P = need > 0 ? topk_radix_select<true>(S, nvalid, need, 0, 0, 0, [&](int64_t e) { return topk_slot_key(p, bq, e, 0); })
+                     : ~0ull;
+      }
+      for (int64_t e0 = 0; need > 0 && e0 < nvalid; e0 += 4 * kTopkThreads) {
         uint64_t k[4];
         uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int64_t e = e0 + 4 * tid + i;
-          k[i] = (e < nvalid) ? topk_slot_key(p, bq, e, tb) : 0;
+          k[i] = (e < nvalid) ? topk_slot_key(p, bq, e, tbf) : 0;
           if (k[i] < P) k[i] = 0;
           m += (k[i] != 0);
         }
@@ -409,7 +486,7 @@ topk_select_kernel(TopkParams p) {
         uint32_t o = written + topk_block_scan(m, S, &tot);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (k[i] != 0) topk_emit(p, out_idx, out_sc, o++, k[i]);
+          if (k[i] != 0) topk_emit(p, bq, out_idx, out_sc, o++, k[i]);
         written += tot;
       }
     }
@@ -422,7 +499,8 @@ topk_select_kernel(TopkParams p) {
 }
 
 inline size_t topk_smem_bytes() {
-  return ((sizeof(TopkShared) + 15) & ~size_t(15)) + static_cast<size_t>(kTopkCap) * 8;
+  return ((sizeof(TopkShared) + 15) & ~size_t(15)) + static_cast<size_t>(kTopkCap) * 8 +
+         static_cast<size_t>(kTopkStages) * kTopkChunkSlots * 4;
 }
 
 // CTAs per selection problem: enough to spread a long score row over SMs

@@ -274,6 +274,11 @@ csa2_status csa2_device_status(int32_t* code, void* stream);
 /* Human-readable name of a status code (static string). */
 const char* csa2_status_string(int32_t status);
 
+/* The CUDA runtime's description of the last launch or runtime failure
+ * behind a CSA2_ERR_CUDA on the calling host thread ("no error" if none);
+ * static string. */
+const char* csa2_cuda_error_string(void);
+
 /* Library ABI version: 100 * major + minor. */
 int32_t csa2_version(void);
 

@@ -123,7 +123,7 @@ def test_index_validation_null_struct(L):
     (dict(B=0), 2), (dict(B=3, Q=30000), 2), (dict(K=-1), 2), (dict(K=0, W=0), 2), (dict(W=1025), 2),
     (dict(swa_rows=100), 2), (dict(Q=2, swa_step=1, swa_rows=128), 2),
     (dict(out=FAKE + 8), 3), (dict(lse=FAKE + 4), 3),
-    (dict(), 4),
+    (dict(), 4),                       # valid arguments, zero-byte workspace
 ])
 def test_attn_validation(L, kw, status):
     assert _call_attn(L, _attn(**kw)) == status
@@ -171,3 +171,36 @@ def test_group_validation(L):
     n = L.csa2_workspace_size(ctypes.byref(g), csa2.WS_GROUP)
     assert n > 0
     assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), n - 1, None) == 4
+
+
+def test_arg_structs_keep_their_tensors_alive():
+    """The ctypes structs hold raw pointers: the binding must keep every
+    tensor they point to alive, or a temporary's memory can be handed to the
+    next allocation (a workspace) before the call runs."""
+    import gc
+    import weakref
+
+    import torch
+    n_vis = torch.zeros(1, 1, dtype=torch.int32)
+    ref = weakref.ref(n_vis)
+    a = csa2.index_args(0, torch.zeros(1, 1, 32, 128), torch.zeros(1, 1, 32), torch.zeros(1, 8, 128), n_vis,
+                        torch.zeros(1, 1, 4, dtype=torch.int32))
+    del n_vis
+    gc.collect()
+    assert ref() is not None
+    q = torch.zeros(1, 1, 64, 512)
+    ref_q = weakref.ref(q)
+    at = csa2.attn_args(q, torch.zeros(1, 8, 288, dtype=torch.uint8), torch.zeros(1, 1, 4, dtype=torch.int32),
+                        torch.zeros(1, 128, 512), torch.zeros(1, 1, 64, 512))
+    del q
+    gc.collect()
+    assert ref_q() is not None
+    nv = torch.zeros(1, 1, dtype=torch.int32)
+    ref_nv = weakref.ref(nv)
+    layer = dict(mode=0, qI=torch.zeros(1), w=torch.zeros(1), q=torch.zeros(1), swa=torch.zeros(1),
+                 out=torch.zeros(1), lse=None, idx=torch.zeros(1, dtype=torch.int32))
+    g = csa2.group_args(1, 1, 4, 128, 8, nv, torch.zeros(1), torch.zeros(1, dtype=torch.uint8), [layer])
+    del nv, layer
+    gc.collect()
+    assert ref_nv() is not None
+    assert a is not None and at is not None and g is not None
