@@ -42,11 +42,12 @@ METRIC = "CSA2 decode queries/s and HBM GB/s vs peak at 128K ctx, FP4 main KV"
 UNIT = "queries/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
-# DRAM traffic of one index_scan_kernel launch, from the ncu capture
-# summarised in profiles/index_scan_kernel_group4_ctx128k.md, valid only
-# while the kernel sources hash to the recorded value.
-SCAN_TRAFFIC = {"sha": None, "bytes_per_launch": None}
+# DRAM traffic (read + write) of one index_scan_kernel launch of the
+# default workload, from an ncu capture of that kernel (profiles/), valid
+# only while the scan's sources hash to the recorded value.
+SCAN_TRAFFIC = {"sha": "9ce00fdab63c1568", "bytes_per_launch": 138217984}
 
 
 def parse():
@@ -180,6 +181,21 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Sustained bf16 TFLOP/s: the prefill scan runs inside a long step."""
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
+
+
+def scan_algorithmic_flops(wl):
+    """Flops of one index_scan_kernel launch: 32 heads x 128 dims x 2 per
+    (query, visible entry)."""
+    return wl.B * sum(wl.n_vis) * 32 * 128 * 2
 
 
 # ---------------------------------------------------------------------------
@@ -416,8 +432,18 @@ def run_ours(args, world, rank, local):
     scan_ms = t_scan / max(n_scan, 1)
     scan_bytes = scan_algorithmic_bytes(wl)
     achieved = scan_bytes / (scan_ms * 1e-3) / 1e9 if n_scan else None
+    if wl.prefill:
+        # eight queries per MMA group make the prefill scan a contraction
+        scan_flops = scan_algorithmic_flops(wl)
+        t_peak, t_kind = tensor_peak()
+        t_achieved = scan_flops / (scan_ms * 1e-3) / 1e12 if n_scan else None
+        roofline = {"kernel": "index_scan_kernel", "bound": "tensor", "achieved": t_achieved, "peak": t_peak,
+                    "peak_source": f"{t_kind} (MEASURED_PEAKS.json bf16_tflops_sustained)" if t_kind == "measured"
+                    else "fallback 1.4 PFLOP/s sustained", "unit": "TFLOP/s",
+                    "frac": (t_achieved / t_peak) if t_achieved else None, "traffic": None,
+                    "algorithmic_flops_per_launch": scan_flops, "ms_per_launch": scan_ms, "launches": n_scan}
     sha = kernel_source_sha()
-    traffic = SCAN_TRAFFIC["bytes_per_launch"] if SCAN_TRAFFIC["sha"] == sha else None
+    traffic = SCAN_TRAFFIC["bytes_per_launch"] if (SCAN_TRAFFIC["sha"] == sha and args.workload == 2) else None
     step_bytes = step_algorithmic_bytes(wl)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -430,7 +456,8 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "hbm_gbs_step": step_bytes / (mean_ms * 1e-3) / 1e9,
         "hbm_frac_step": step_bytes / (mean_ms * 1e-3) / 1e9 / peak,
-        "roofline": {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+        "roofline": roofline if wl.prefill else
+                    {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s", "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
