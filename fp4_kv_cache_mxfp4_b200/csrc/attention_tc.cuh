@@ -1,22 +1,30 @@
-// attention_tc.cuh -- sparse MQA slice kernel on the 5th-generation tensor
-// cores ("DeepSeek V4.1-Flash 技术报告深度解析" §3.2 attention, §3.4
-// dequantise before the attention math).
+// attention_tc.cuh -- sparse MQA on the 5th-generation tensor cores
+// ("DeepSeek V4.1-Flash 技术报告深度解析" §3.2 attention, §3.4 dequantise
+// before the attention math).
 //
-// One CTA (512 threads) per (128-key slice, query).  The slice's keys (FP4
-// entries, each 288-byte row fetched by one bulk copy and dequantised by the
-// CTA's threads, or window rows brought by TMA) form a 128 x 512 bf16 tile
-// K in shared memory, stored K-major with the 128-byte swizzle.  The
-// query's 64 heads form Q (64 x 512, TMA).  Then:
+// A query's keys are cut into 128-key slices: ceil(K/128) slices of selected
+// FP4 entries, then ceil(W/128) slices of window rows.  A CTA (512 threads)
+// takes one slice (split mode: many CTAs per query, for few queries) or all
+// slices of its query in turn (one CTA per query, for many queries).  Per
+// slice the keys (FP4 entries, each 288-byte row fetched by one bulk copy
+// and dequantised by the CTA's threads, or window rows brought by TMA) form
+// a 128 x 512 bf16 tile K in shared memory, stored K-major with the 128-byte
+// swizzle; the query's 64 heads form Q (64 x 512, TMA, loaded once).  Then:
 //   MMA 1   S^T[key, head] = K . Q^T            M = 128 keys, N = 64, K = 512
-//   softmax per head over the slice's keys (fp32, from TMEM via shared
-//           memory), P^T[head, key] = exp2(S^T - max) rounded to bf16 and
-//           stored as a K-major operand
-//   MMA 2   O^T[dim, head] = V^T . P^T          the same key tile read
+//   softmax per head over the slice's keys in registers (fp32; shuffles and
+//           a 2 KB exchange between key quarters) against a running
+//           reference max that only moves when a slice's max exceeds it by
+//           more than 2^8 (the accumulator is then rescaled in TMEM);
+//           P^T[key, head] = exp2(S^T - ref) rounded to bf16, stored
+//           [key][head] as an MN-major operand
+//   MMA 2   O^T[dim, head] += V^T . P^T         the same key tile read
 //           MN-major (M = 128 dims per MMA, 4 tiles), N = 64, K = 128 keys
 //   epilogue: O^T from TMEM to shared memory as [head][dim] fp32, then
-//           coalesced 16-byte stores to the slice's partial output; with the
-//           slice's (max, sum) per head, sparse_attn_combine_kernel merges the
-//           slices.
+//     split mode:  coalesced 16-byte stores of the unnormalised partial and
+//                  the slice's (max, sum) per head; sparse_attn_combine_kernel
+//                  merges the slices;
+//     one CTA per query: normalised by the running sum, written as bf16 with
+//                  the log-sum-exp.
 // Accumulators: S^T in TMEM columns [0, 64), O^T tile t in [64 + 64t, 128 + 64t).
 #pragma once
 #include "common.cuh"
@@ -29,9 +37,10 @@ constexpr int kTcAttnWarps = kTcAttnThreads / 32;
 constexpr int kTcAttnKeys = 128;                       // keys per slice (MMA M)
 constexpr uint32_t kTcKeyTileBytes = 128 * 512 * 2;    // 128 KB: 8 chunks of [128 rows x 64 dims]
 constexpr uint32_t kTcQTileBytes = 64 * 512 * 2;       // 64 KB: 8 chunks of [64 rows x 64 dims]
-constexpr int kTcSPitch = kTcAttnKeys + 4;             // fp32 row pitch of the transposed scores
-constexpr uint32_t kTcMiscBytes = 2048;
-constexpr uint32_t kTcAttnSmem = kTcKeyTileBytes + kTcQTileBytes + kTcMiscBytes + 1024;
+constexpr uint32_t kTcPTileBytes = 128 * 64 * 2;       // 16 KB: P^T [128 keys][64 heads]
+constexpr uint32_t kTcMiscBytes = 4096;
+constexpr uint32_t kTcAttnSmem = kTcKeyTileBytes + kTcQTileBytes + kTcPTileBytes + kTcMiscBytes + 1024;
+constexpr float kTcRefSlack = 8.0f;                    // log2 units a slice max may exceed the reference
 
 struct TcAttnParams {
   int B, Q, K, W;
@@ -42,8 +51,11 @@ struct TcAttnParams {
   int kv_slices;             // ceil(K / 128): slices 0..kv_slices-1 hold FP4 entries, the rest window rows
   int slices;
   float scale_log2;
-  float* opart;              // [BQ][slices][64][512]
-  float* ml;                 // [BQ][slices][64][2]
+  int per_query;             // 1: one CTA per query over all slices, final output; 0: one slice per CTA
+  float* opart;              // split: [BQ][slices][64][512]
+  float* ml;                 // split: [BQ][slices][64][2]
+  __nv_bfloat16* out;        // per query: [BQ][64][512]
+  float* lse;                // per query, optional: [BQ][64]
 };
 
 // byte offset of the 16-byte unit u (0..7) of row r in a K-major operand
@@ -97,6 +109,56 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+         "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+         "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Reduce 16 per-lane values (16 heads) over the 32 lanes of a warp with 16
+// shuffles: each halving step trades half of the values with the partner
+// lane, so afterwards lane l holds the reduction of head l >> 1.
+template <bool MAX>
+__device__ __forceinline__ float warp_reduce_heads16(const float (&v)[16], int lane) {
+  float a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {                        // lane bit 4 keeps heads 8..15, else 0..7
+    const bool hi = lane & 16;
+    const float keep = hi ? v[j + 8] : v[j], give = hi ? v[j] : v[j + 8];
+    const float got = __shfl_xor_sync(0xffffffffu, give, 16);
+    a[j] = MAX ? fmaxf(keep, got) : keep + got;
+  }
+  float b[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const bool hi = lane & 8;
+    const float keep = hi ? a[j + 4] : a[j], give = hi ? a[j] : a[j + 4];
+    const float got = __shfl_xor_sync(0xffffffffu, give, 8);
+    b[j] = MAX ? fmaxf(keep, got) : keep + got;
+  }
+  float c[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const bool hi = lane & 4;
+    const float keep = hi ? b[j + 2] : b[j], give = hi ? b[j] : b[j + 2];
+    const float got = __shfl_xor_sync(0xffffffffu, give, 4);
+    c[j] = MAX ? fmaxf(keep, got) : keep + got;
+  }
+  const bool hi = lane & 2;
+  const float keep = hi ? c[1] : c[0], give = hi ? c[0] : c[1];
+  const float got = __shfl_xor_sync(0xffffffffu, give, 2);
+  float d = MAX ? fmaxf(keep, got) : keep + got;
+  const float e = __shfl_xor_sync(0xffffffffu, d, 1);
+  return MAX ? fmaxf(d, e) : d + e;
+}
+
 __global__ void __launch_bounds__(kTcAttnThreads, 1)
 sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_swa,
@@ -104,212 +166,282 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   extern __shared__ __align__(1024) uint8_t tc_attn_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_attn_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* kt = smem;                                   // key tile (K-major), later read MN-major as V^T
-  uint8_t* qt = smem + kTcKeyTileBytes;                 // Q (K-major); after MMA 1: scores and P^T
-  float* st = reinterpret_cast<float*>(qt);             // [64 heads][kTcSPitch] scaled scores
-  uint8_t* pt = qt + 64 * kTcSPitch * 4;                // P^T: 2 chunks of [64 rows x 64 keys] (1024-aligned)
-  uint8_t* misc = qt + kTcQTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(misc);   // [0] q/window TMA, [1] MMA 1 done, [2] MMA 2 done,
-                                                        // [3] FP4 row gather
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* qt = smem + kTcKeyTileBytes;                 // Q (K-major), kept for every slice
+  uint8_t* pt = qt + kTcQTileBytes;                     // P^T [128 keys][64 heads] bf16, swizzled (MN-major)
+  uint8_t* misc = pt + kTcPTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc);   // [0] Q TMA, [1] MMA 1 done, [2] MMA 2 done,
+                                                        // [3] FP4 row gather, [4] window rows TMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 48);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 52);
+  int* rescale_flag = reinterpret_cast<int*>(misc + 56);
   int* valid_s = reinterpret_cast<int*>(misc + 64);                  // [128]
+  float* red_s = reinterpret_cast<float*>(misc + 576);               // [2][4 quarters][64 heads]: max, sum
+  float* ref_s = reinterpret_cast<float*>(misc + 2624);              // [64] running reference max (log2 units)
+  float* sum_s = reinterpret_cast<float*>(misc + 2880);              // [64] running sum of P
+  float* fac_s = reinterpret_cast<float*>(misc + 3136);              // [64] rescale factor of this slice
 
-  const int slice = blockIdx.x, bq = blockIdx.y;
+  const int bq = blockIdx.y;
   const int b = bq / p.Q, qi = bq % p.Q;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool window = slice >= p.kv_slices;
-  const int key0 = window ? (slice - p.kv_slices) * kTcAttnKeys : slice * kTcAttnKeys;   // first key of the slice
-  const int nkeys = window ? min(kTcAttnKeys, p.W - key0) : min(kTcAttnKeys, p.K - key0);
+  const int first_slice = p.per_query ? 0 : static_cast<int>(blockIdx.x);
+  const int n_iter = p.per_query ? p.slices : 1;
 
   if (tid == 0) {
-    mbar_init(&bars[0], 1); mbar_init(&bars[1], 1); mbar_init(&bars[2], 1); mbar_init(&bars[3], 1);
+    for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
     *abort_flag = 0;
+    *rescale_flag = 0;
     fence_barrier_init();
   }
+  if (tid < 64) { ref_s[tid] = -INFINITY; sum_s[tid] = 0.0f; }
   if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   if (tid == 0) { tma_prefetch_desc(&tmap_q); tma_prefetch_desc(&tmap_swa); }
   pdl_wait();                                           // idx, q and the FP4 rows come from earlier kernels
   pdl_launch_dependents();
-  int v = 0;
-  if (tid < kTcAttnKeys) {
-    if (tid < nkeys) {
-      if (window) {
-        v = 1;
-      } else {
-        const int32_t e = p.idx[static_cast<int64_t>(bq) * p.K + key0 + tid];
-        v = (e >= 0 && e < p.N) ? e + 1 : 0;            // entry + 1, 0 = empty slot
-      }
-    }
-    valid_s[tid] = v;
+  if (tid == 0) {                                       // this thread initialised the barrier
+    mbar_arrive_expect_tx(&bars[0], kTcQTileBytes);
+    const uint64_t pol = l2_policy_evict_last();
+    for (int c = 0; c < 8; ++c) tma_load_2d(qt + c * 8192, &tmap_q, &bars[0], 64 * c, bq * 64, pol);
   }
   tc_fence_before();
-  const int n_rows = __syncthreads_count(!window && v != 0);   // FP4 rows to gather
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // ---- operands: Q (and window rows) by TMA; FP4 rows by one bulk copy
-  //      each into a staging area inside the key tile, then dequantised
-  uint8_t* stage = kt;                                  // [128][288] raw rows (overwritten below)
-  if (tid == 0) {
-    const uint64_t pol = l2_policy_evict_last();
-    if (n_rows) mbar_arrive_expect_tx(&bars[3], static_cast<uint32_t>(n_rows) * 288u);
-    else mbar_arrive(&bars[3]);
-    mbar_arrive_expect_tx(&bars[0], kTcQTileBytes + (window ? kTcKeyTileBytes : 0));
-    for (int c = 0; c < 8; ++c) tma_load_2d(qt + c * 8192, &tmap_q, &bars[0], 64 * c, bq * 64, pol);
-    if (window) {
-      const int32_t y = b * p.swa_rows + qi * p.swa_step + key0;
-      for (int c = 0; c < 8; ++c) tma_load_2d(kt + c * 16384, &tmap_swa, &bars[0], 64 * c, y, pol);
-    }
-  }
-  if (!window) {
-    __syncthreads();                                    // expect_tx is posted before any copy lands
-    if (tid < kTcAttnKeys && v != 0) {
-      const uint8_t* row = p.kv + (static_cast<int64_t>(b) * p.N + (v - 1)) * 288;
-      asm volatile(
-          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 288, [%2];"
-          :: "r"(smem_u32(stage + tid * 288)), "l"(row), "r"(smem_u32(&bars[3])) : "memory");
-    }
-    // item = (key r, 32-channel chunk c): 16 nibble bytes + 2 scales -> four
-    // 16-byte units of the key tile.  A warp takes 32 consecutive keys of one
-    // chunk (conflict-free swizzled stores).  All raw items go to registers
-    // before anything is written, since the tile overwrites the staging area.
-    constexpr int kItems = kTcAttnKeys * 16 / kTcAttnThreads;
-    const bool ok = mbar_wait(&bars[3], 0, kErrWaitOperand, abort_flag);
-    uint4 nib[kItems];
-    uint32_t sc[kItems];
-#pragma unroll
-    for (int k = 0; k < kItems; ++k) {
-      const int i = tid + k * kTcAttnThreads;
-      const int r = i & (kTcAttnKeys - 1), c = i >> 7;
-      nib[k] = make_uint4(0, 0, 0, 0);
-      sc[k] = 0;
-      if (ok && valid_s[r]) {
-        nib[k] = *reinterpret_cast<const uint4*>(stage + r * 288 + c * 16);
-        sc[k] = *reinterpret_cast<const uint16_t*>(stage + r * 288 + 256 + 2 * c);
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kItems; ++k) {
-      const int i = tid + k * kTcAttnThreads;
-      const int r = i & (kTcAttnKeys - 1), c = i >> 7;
-      const float s0 = e4m3_code_to_float(sc[k] & 0xFF), s1 = e4m3_code_to_float(sc[k] >> 8);
-      const __nv_bfloat162 S0 = __floats2bfloat162_rn(s0, s0), S1 = __floats2bfloat162_rn(s1, s1);
-      uint32_t o[4][4];
-      e2m1x8_to_bf16(nib[k].x, S0, o[0]);          // channels 32c .. 32c+7
-      e2m1x8_to_bf16(nib[k].y, S0, o[1]);          //          .. 32c+15 (first scale block)
-      e2m1x8_to_bf16(nib[k].z, S1, o[2]);
-      e2m1x8_to_bf16(nib[k].w, S1, o[3]);          // empty slot: zero nibbles and scale -> zero key
-      // channels 32c..32c+31 = chunk c/2 of the tile, units 4(c&1)..4(c&1)+3
-      uint8_t* chunk = kt + (c >> 1) * 16384;
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        *reinterpret_cast<uint4*>(chunk + sw128_off(r, 4 * (c & 1) + t)) = make_uint4(o[t][0], o[t][1], o[t][2], o[t][3]);
-    }
-    fence_async_smem();
-  }
-  __syncthreads();
+  for (int it = 0; it < n_iter; ++it) {
+    const int slice = first_slice + it;
+    const bool window = slice >= p.kv_slices;
+    const int key0 = window ? (slice - p.kv_slices) * kTcAttnKeys : slice * kTcAttnKeys;   // first key of the slice
+    const int nkeys = window ? min(kTcAttnKeys, p.W - key0) : min(kTcAttnKeys, p.K - key0);
+    const uint32_t ph = static_cast<uint32_t>(it & 1);                 // MMA barriers complete once per slice
+    // row-gather and window barriers complete once per slice of their kind
+    // (KV slices come first); in split mode each is used once
+    const uint32_t ph_rows = p.per_query ? static_cast<uint32_t>(slice & 1) : 0u;
+    const uint32_t ph_win = p.per_query ? static_cast<uint32_t>((slice - p.kv_slices) & 1) : 0u;
 
-  // ---- MMA 1: S^T = K . Q^T  (M = 128 keys, N = 64 heads, K = 512 dims)
-  if (warp == 1 && lane == 0) {
-    if (mbar_wait(&bars[0], 0, kErrWaitOperand, abort_flag)) {
+    // the key tile and P^T are free once the previous slice's MMA 2 is done
+    if (it > 0) {
+      mbar_wait(&bars[2], ph ^ 1, kErrWaitTmemFull, abort_flag);
       tc_fence_after();
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(128, 64);
-      const uint32_t ka = smem_u32(kt), qa = smem_u32(qt);
-#pragma unroll
-      for (int kk = 0; kk < 32; ++kk) {
-        const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        const uint32_t qoff = (kk >> 2) * 8192 + (kk & 3) * 32;
-        umma_bf16(tmem, umma_desc_sw128_kmajor(ka + koff), umma_desc_sw128_kmajor(qa + qoff), idesc, kk > 0);
-      }
     }
-    umma_commit(&bars[1]);
-  }
-
-  // ---- scores: TMEM -> scaled, masked, transposed into shared memory.
-  //      Warp w reads TMEM lanes 32(w%4).. (its keys) and heads 16(w/4)..
-  {
-    const bool ok = mbar_wait(&bars[1], 0, kErrWaitTmemFull, abort_flag);
-    if (__all_sync(0xffffffffu, ok)) {
-      tc_fence_after();
-      const int quarter = warp & 3, hg = warp >> 2;
-      const int key = quarter * 32 + lane;
-      const bool kv_ok = valid_s[key] != 0;
-      uint32_t r[16];
-      tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 16 * hg, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        st[(16 * hg + j) * kTcSPitch + key] = kv_ok ? __uint_as_float(r[j]) * p.scale_log2 : -INFINITY;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-
-  // ---- softmax statistics per head; P^T in bf16 as the K-major B operand
-  {
-    const int h = tid >> 3, part = tid & 7;               // 8 threads per head, 16 keys each
-    const float* srow = st + h * kTcSPitch + part * 16;
-    float m = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) m = fmaxf(m, srow[j]);
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    const float mu = (m == -INFINITY) ? 0.0f : m;
-    float l = 0.0f;
-    uint32_t pk[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const __nv_bfloat162 v = __floats2bfloat162_rn(exp2f(srow[2 * j] - mu), exp2f(srow[2 * j + 1] - mu));
-      const float2 f = __bfloat1622float2(v);
-      l += f.x + f.y;
-      pk[j] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    l += __shfl_xor_sync(0xffffffffu, l, 4);
-    __syncthreads();                                      // every thread has read the scores it needs
-    // keys 16part .. 16part+15 = chunk part/4, units 2(part&3), 2(part&3)+1 of row h
-    uint8_t* chunk = pt + (part >> 2) * 8192;
-#pragma unroll
-    for (int t = 0; t < 2; ++t)
-      *reinterpret_cast<uint4*>(chunk + sw128_off(h, 2 * (part & 3) + t)) =
-          make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-    if (part == 0) {
-      float* ml = p.ml + ((static_cast<int64_t>(bq) * p.slices + slice) * 64 + h) * 2;
-      ml[0] = m;
-      ml[1] = l;
-    }
-    fence_async_smem();
-  }
-  tc_fence_before();
-  __syncthreads();
-
-  // ---- MMA 2: O^T = V^T . P^T  (M = 128 dims per tile, N = 64 heads, K = 128 keys)
-  if (warp == 1 && lane == 0) {
-    tc_fence_after();
-    if (!*abort_flag) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(128, 64) | (1u << 15);   // A MN-major
-      const uint32_t ka = smem_u32(kt), pa = smem_u32(pt);
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t adesc = umma_desc_sw128_mnmajor(ka + (2 * t) * 16384 + kk * 2048, 16384);
-          const uint64_t bdesc = umma_desc_sw128_kmajor(pa + (kk >> 2) * 8192 + (kk & 3) * 32);
-          umma_bf16(tmem + 64 + 64 * t, adesc, bdesc, idesc, kk > 0);
+    int v = 0;
+    if (tid < kTcAttnKeys) {
+      if (tid < nkeys) {
+        if (window) {
+          v = 1;
+        } else {
+          const int32_t e = p.idx[static_cast<int64_t>(bq) * p.K + key0 + tid];
+          v = (e >= 0 && e < p.N) ? e + 1 : 0;            // entry + 1, 0 = empty slot
         }
       }
+      valid_s[tid] = v;
     }
-    umma_commit(&bars[2]);
+    const int n_rows = __syncthreads_count(!window && v != 0);   // FP4 rows to gather
+
+    // ---- operands: window rows by TMA; FP4 rows by one bulk copy each into
+    //      a staging area inside the key tile, then dequantised
+    uint8_t* stage = kt;                                  // [128][288] raw rows (overwritten below)
+    if (tid == 0) {
+      const uint64_t pol = l2_policy_evict_last();
+      if (!window) {
+        if (n_rows) mbar_arrive_expect_tx(&bars[3], static_cast<uint32_t>(n_rows) * 288u);
+        else mbar_arrive(&bars[3]);
+      } else {
+        mbar_arrive_expect_tx(&bars[4], kTcKeyTileBytes);
+        const int32_t y = b * p.swa_rows + qi * p.swa_step + key0;
+        for (int c = 0; c < 8; ++c) tma_load_2d(kt + c * 16384, &tmap_swa, &bars[4], 64 * c, y, pol);
+      }
+    }
+    if (!window) {
+      __syncthreads();                                    // expect_tx is posted before any copy lands
+      if (tid < kTcAttnKeys && v != 0) {
+        const uint8_t* row = p.kv + (static_cast<int64_t>(b) * p.N + (v - 1)) * 288;
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 288, [%2];"
+            :: "r"(smem_u32(stage + tid * 288)), "l"(row), "r"(smem_u32(&bars[3])) : "memory");
+      }
+      // item = (key r, 32-channel chunk c): 16 nibble bytes + 2 scales -> four
+      // 16-byte units of the key tile.  A warp takes 32 consecutive keys of one
+      // chunk (conflict-free swizzled stores).  All raw items go to registers
+      // before anything is written, since the tile overwrites the staging area.
+      constexpr int kItems = kTcAttnKeys * 16 / kTcAttnThreads;
+      const bool ok = mbar_wait(&bars[3], ph_rows, kErrWaitOperand, abort_flag);
+      uint4 nib[kItems];
+      uint32_t sc[kItems];
+#pragma unroll
+      for (int k = 0; k < kItems; ++k) {
+        const int i = tid + k * kTcAttnThreads;
+        const int r = i & (kTcAttnKeys - 1), c = i >> 7;
+        nib[k] = make_uint4(0, 0, 0, 0);
+        sc[k] = 0;
+        if (ok && valid_s[r]) {
+          nib[k] = *reinterpret_cast<const uint4*>(stage + r * 288 + c * 16);
+          sc[k] = *reinterpret_cast<const uint16_t*>(stage + r * 288 + 256 + 2 * c);
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < kItems; ++k) {
+        const int i = tid + k * kTcAttnThreads;
+        const int r = i & (kTcAttnKeys - 1), c = i >> 7;
+        const float s0 = e4m3_code_to_float(sc[k] & 0xFF), s1 = e4m3_code_to_float(sc[k] >> 8);
+        const __nv_bfloat162 S0 = __floats2bfloat162_rn(s0, s0), S1 = __floats2bfloat162_rn(s1, s1);
+        uint32_t o[4][4];
+        e2m1x8_to_bf16(nib[k].x, S0, o[0]);          // channels 32c .. 32c+7
+        e2m1x8_to_bf16(nib[k].y, S0, o[1]);          //          .. 32c+15 (first scale block)
+        e2m1x8_to_bf16(nib[k].z, S1, o[2]);
+        e2m1x8_to_bf16(nib[k].w, S1, o[3]);          // empty slot: zero nibbles and scale -> zero key
+        // channels 32c..32c+31 = chunk c/2 of the tile, units 4(c&1)..4(c&1)+3
+        uint8_t* chunk = kt + (c >> 1) * 16384;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          *reinterpret_cast<uint4*>(chunk + sw128_off(r, 4 * (c & 1) + t)) = make_uint4(o[t][0], o[t][1], o[t][2], o[t][3]);
+      }
+      fence_async_smem();
+    }
+    __syncthreads();
+
+    // ---- MMA 1: S^T = K . Q^T  (M = 128 keys, N = 64 heads, K = 512 dims)
+    if (warp == 1 && lane == 0) {
+      bool ok = mbar_wait(&bars[0], 0, kErrWaitOperand, abort_flag);
+      if (ok && window) ok = mbar_wait(&bars[4], ph_win, kErrWaitOperand, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        constexpr uint32_t idesc = umma_idesc_bf16_f32(128, 64);
+        const uint32_t ka = smem_u32(kt), qa = smem_u32(qt);
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_bf16(tmem, umma_desc_sw128_kmajor(ka + koff), umma_desc_sw128_kmajor(qa + qoff), idesc, kk > 0);
+        }
+      }
+      umma_commit(&bars[1]);
+    }
+
+    // ---- softmax in registers.  Warp w reads TMEM lanes 32(w%4).. (its 32
+    //      keys) for heads 16(w/4)..16(w/4)+15; per-head max and sum reduce
+    //      over the lanes by shuffles and over the four key quarters through
+    //      shared memory.
+    {
+      const int quarter = warp & 3, hg = warp >> 2;
+      const int key = quarter * 32 + lane;
+      float sv[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) sv[j] = -INFINITY;
+      const bool ok = mbar_wait(&bars[1], ph, kErrWaitTmemFull, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const bool kv_ok = valid_s[key] != 0;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 16 * hg, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) sv[j] = kv_ok ? __uint_as_float(r[j]) * p.scale_log2 : -INFINITY;
+      }
+      {
+        const float m = warp_reduce_heads16<true>(sv, lane);
+        if ((lane & 1) == 0) red_s[quarter * 64 + 16 * hg + (lane >> 1)] = m;
+      }
+      __syncthreads();
+      // reference max per head: the running one unless this slice's max
+      // exceeds it by more than kTcRefSlack
+      float lj[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int h = 16 * hg + j;
+        const float mt = fmaxf(fmaxf(red_s[h], red_s[64 + h]), fmaxf(red_s[128 + h], red_s[192 + h]));
+        const float ref = ref_s[h];
+        const float nref = (mt > ref + kTcRefSlack) ? mt : ref;
+        lj[j] = exp2f(sv[j] - ((nref == -INFINITY) ? 0.0f : nref));
+      }
+      uint32_t pk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(lj[2 * j], lj[2 * j + 1]);
+        pk[j] = *reinterpret_cast<const uint32_t*>(&v2);
+        const float2 f = __bfloat1622float2(v2);        // the sum uses the rounded weights MMA 2 sees
+        lj[2 * j] = f.x;
+        lj[2 * j + 1] = f.y;
+      }
+      *reinterpret_cast<uint4*>(pt + sw128_off(key, 2 * hg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(pt + sw128_off(key, 2 * hg + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      {
+        const float l = warp_reduce_heads16<false>(lj, lane);
+        if ((lane & 1) == 0) red_s[256 + quarter * 64 + 16 * hg + (lane >> 1)] = l;
+      }
+      fence_async_smem();
+      __syncthreads();
+      if (tid < 64) {
+        const int h = tid;
+        const float mt = fmaxf(fmaxf(red_s[h], red_s[64 + h]), fmaxf(red_s[128 + h], red_s[192 + h]));
+        const float l = (red_s[256 + h] + red_s[320 + h]) + (red_s[384 + h] + red_s[448 + h]);
+        const float ref = ref_s[h];
+        const float nref = (mt > ref + kTcRefSlack) ? mt : ref;
+        const float f = (nref == ref || ref == -INFINITY) ? 1.0f : exp2f(ref - nref);
+        fac_s[h] = f;
+        if (f != 1.0f && it > 0) *rescale_flag = 1;       // the accumulator holds earlier slices
+        ref_s[h] = nref;
+        sum_s[h] = sum_s[h] * f + l;
+        if (!p.per_query) {
+          float* ml = p.ml + ((static_cast<int64_t>(bq) * p.slices + slice) * 64 + h) * 2;
+          ml[0] = nref;
+          ml[1] = l;
+        }
+      }
+      // one slice per CTA: nothing below reads the running state, and P^T is
+      // already published to the MMA issuer by the barrier above
+      if (p.per_query) {
+        tc_fence_before();
+        __syncthreads();
+      }
+    }
+
+    // ---- rescale the accumulator (rare: a slice max far above the reference)
+    if (p.per_query && *rescale_flag) {
+      const int quarter = warp & 3, t = warp >> 2;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64 + 64 * t + 32 * hh;
+        tc_fence_after();
+        tmem_ld_32x32b_x32(taddr, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * fac_s[32 * hh + j]);
+        tmem_st_32x32b_x32(taddr, r);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) *rescale_flag = 0;
+    }
+
+    // ---- MMA 2: O^T += V^T . P^T  (M = 128 dims per tile, N = 64 heads, K = 128 keys)
+    if (warp == 1 && lane == 0) {
+      tc_fence_after();
+      if (!*abort_flag) {
+        // A (V^T) and B (P^T) both MN-major
+        constexpr uint32_t idesc = umma_idesc_bf16_f32(128, 64) | (1u << 15) | (1u << 16);
+        const uint32_t ka = smem_u32(kt), pa = smem_u32(pt);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t adesc = umma_desc_sw128_mnmajor(ka + (2 * t) * 16384 + kk * 2048, 16384);
+            const uint64_t bdesc = umma_desc_sw128_mnmajor(pa + kk * 2048, 16384);
+            umma_bf16(tmem + 64 + 64 * t, adesc, bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+      }
+      umma_commit(&bars[2]);
+    }
   }
 
   // ---- epilogue: O^T tile (warp / 4), dims 32(warp % 4).. -> shared
   //      [head][dim] (the key tile is free now)
   float* obuf = reinterpret_cast<float*>(kt);
   {
-    const bool ok = mbar_wait(&bars[2], 0, kErrWaitTmemFull, abort_flag);
+    const bool ok = mbar_wait(&bars[2], static_cast<uint32_t>((n_iter - 1) & 1), kErrWaitTmemFull, abort_flag);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int quarter = warp & 3, t = warp >> 2;
@@ -319,8 +451,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64 + 64 * t + 32 * hh, r);
         tmem_ld_wait();
+        if (p.per_query) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) obuf[(32 * hh + j) * 512 + d] = __uint_as_float(r[j]);
+          for (int j = 0; j < 32; ++j) {
+            const float l = sum_s[32 * hh + j];
+            obuf[(32 * hh + j) * 512 + d] = (l > 0.0f) ? __uint_as_float(r[j]) / l : 0.0f;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) obuf[(32 * hh + j) * 512 + d] = __uint_as_float(r[j]);
+        }
       }
     }
   }
@@ -330,12 +470,26 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-
-  if (!*abort_flag) {
-    float4* op = reinterpret_cast<float4*>(p.opart + (static_cast<int64_t>(bq) * p.slices + slice) * 64 * 512);
+  if (*abort_flag) return;
+  if (!p.per_query) {
+    float4* op = reinterpret_cast<float4*>(p.opart + (static_cast<int64_t>(bq) * p.slices + first_slice) * 64 * 512);
     const float4* src = reinterpret_cast<const float4*>(obuf);
 #pragma unroll 4
     for (int j = tid; j < 64 * 512 / 4; j += kTcAttnThreads) op[j] = src[j];
+  } else {
+    // bf16 output, 8 dims (16 bytes) per store
+    uint4* op = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(bq) * 64 * 512);
+#pragma unroll 4
+    for (int j = tid; j < 64 * 512 / 8; j += kTcAttnThreads) {
+      const float4 a = reinterpret_cast<const float4*>(obuf)[2 * j];
+      const float4 c = reinterpret_cast<const float4*>(obuf)[2 * j + 1];
+      op[j] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
+    }
+    if (p.lse && tid < 64) {
+      const float l = sum_s[tid];
+      p.lse[static_cast<int64_t>(bq) * 64 + tid] =
+          (l > 0.0f) ? (ref_s[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
   }
 }
 

@@ -366,7 +366,16 @@ bool make_map_bf16_512(CUtensorMap* m, const void* base, uint64_t rows, uint32_t
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// With this many queries one CTA per query (all its slices in turn, final
+// output) fills the GPU; fewer queries split their slices over CTAs and
+// merge fp32 partials in sparse_attn_combine_kernel.
+constexpr int64_t kAttnPerQueryMinBQ = 128;
+inline bool attn_per_query(const csa2_attn_args* a) {
+  return static_cast<int64_t>(a->B) * a->Q >= kAttnPerQueryMinBQ;
+}
+
 size_t attn_ws_bytes(const csa2_attn_args* a) {
+  if (attn_per_query(a)) return 256;            // unused; the size query stays non-zero for valid arguments
   const size_t bq = static_cast<size_t>(a->B) * a->Q, s = attn_slices(a);
   return up256(bq * s * 64 * 512 * 4) + up256(bq * s * 64 * 2 * 4);
 }
@@ -386,8 +395,12 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
   t.kv_slices = attn_kv_slices(a);
   t.slices = slices;
   t.scale_log2 = scale * 1.4426950408889634f;
-  t.opart = opart;
-  t.ml = ml;
+  const bool per_query = attn_per_query(a);
+  t.per_query = per_query ? 1 : 0;
+  t.opart = per_query ? nullptr : opart;
+  t.ml = per_query ? nullptr : ml;
+  t.out = static_cast<__nv_bfloat16*>(a->out);
+  t.lse = a->lse;
   CUtensorMap tq, tw;
   if (!make_map_bf16_512(&tq, a->q, bq * 64, 64)) return CSA2_ERR_CUDA;
   if (a->W > 0) {
@@ -396,10 +409,11 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
     tw = tq;                                    // no window slices: never used
   }
   trace_pre(kKAttnSlice, st);
-  const cudaError_t e1 = launch_ex(sparse_attn_tc_kernel, dim3(slices, static_cast<unsigned>(bq)), dim3(kTcAttnThreads),
-                                   kTcAttnSmem, st, 0, tq, tw, t);
+  const cudaError_t e1 = launch_ex(sparse_attn_tc_kernel, dim3(per_query ? 1 : slices, static_cast<unsigned>(bq)),
+                                   dim3(kTcAttnThreads), kTcAttnSmem, st, 0, tq, tw, t);
   trace_post(st);
   if (e1 != cudaSuccess) return CSA2_ERR_CUDA;
+  if (per_query) return CSA2_OK;
 
   AttnParams p;
   p.slices = slices;

@@ -60,6 +60,8 @@ def _oracle(kv, q, swa, idx, W, swa_step, scale=None):
     (1, 2, 300, 100, 37, 1, 2, 0.0),       # ragged slices, causal windows
     (3, 1, 64, 64, 0, 0, 3, 0.0),          # selected entries only
     (1, 1, 10, 0, 128, 0, 4, 0.0),         # window only
+    (1, 130, 3000, 512, 128, 1, 7, 0.05),  # 130 queries: one CTA per query over all its slices
+    (2, 70, 900, 200, 100, 1, 8, 0.0),     # per query, ragged slices
 ])
 def test_attention_parity(B, Q, N, K, W, step, seed, m1):
     kv, q, swa, idx = _case(B, Q, N, K, W, step, seed, minus_one=m1)
@@ -77,9 +79,22 @@ def test_peaked_softmax_and_explicit_scale():
     np.testing.assert_allclose(lse, lse_ref, rtol=1e-3, atol=1e-2)
 
 
+def test_per_query_reference_max_moves():
+    """One CTA per query with a very peaked softmax (unit query scale and
+    softmax scale 1): slice maxima differ by tens of log2 units, so later
+    slices often move the running reference max and the accumulated output
+    of the earlier slices is rescaled."""
+    kv, q, swa, idx = _case(1, 128, 2000, 384, 128, 1, 9, q_std=1.0)
+    out, lse = _run(kv, q, swa, idx, 128, 1, scale=1.0)
+    o_ref, lse_ref = _oracle(kv, q, swa, idx, 128, 1, scale=1.0)
+    check_attention(out, o_ref, what="rescaled")
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-3, atol=1e-2)
+
+
 def test_no_keys_at_all():
-    kv, q, swa, idx = _case(1, 2, 100, 64, 0, 0, 6)
-    idx[:] = -1
-    out, lse = _run(kv, q, swa, idx, 0, 0)
-    assert np.all(out == 0)
-    assert np.all(np.isneginf(lse))
+    for Q in (2, 128):                     # split slices and one CTA per query
+        kv, q, swa, idx = _case(1, Q, 100, 64, 0, 0, 6)
+        idx[:] = -1
+        out, lse = _run(kv, q, swa, idx, 0, 0)
+        assert np.all(out == 0)
+        assert np.all(np.isneginf(lse))
