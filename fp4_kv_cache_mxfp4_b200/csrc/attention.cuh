@@ -31,8 +31,8 @@ sparse_attn_combine_kernel(AttnParams p) {
   __shared__ float m_s[kAttnMaxSlices], l_s[kAttnMaxSlices];
   const int bq = blockIdx.x >> 6, h = blockIdx.x & 63;
   const int t = threadIdx.x;
-  pdl_wait();
   pdl_launch_dependents();
+  pdl_wait();
   const float* ml = p.ml + static_cast<int64_t>(bq) * p.slices * 128;
   if (t < p.slices) { m_s[t] = ml[t * 128 + h * 2]; l_s[t] = ml[t * 128 + h * 2 + 1]; }
   __syncthreads();

@@ -52,6 +52,8 @@ struct TcAttnParams {
   int slices;
   float scale_log2;
   int per_query;             // 1: one CTA per query over all slices, final output; 0: one slice per CTA
+  int early_inputs;          // 1: q and the window rows are complete at launch (the predecessor is a
+                             // kernel of this library): load them before waiting on it
   float* opart;              // split: [BQ][slices][64][512]
   float* ml;                 // split: [BQ][slices][64][2]
   __nv_bfloat16* out;        // per query: [BQ][64][512]
@@ -195,8 +197,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   if (tid < 64) { ref_s[tid] = -INFINITY; sum_s[tid] = 0.0f; }
   if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   if (tid == 0) { tma_prefetch_desc(&tmap_q); tma_prefetch_desc(&tmap_swa); }
-  pdl_wait();                                           // idx, q and the FP4 rows come from earlier kernels
   pdl_launch_dependents();
+  // idx comes from the previous kernel, and the partial outputs overwrite a
+  // buffer the previous layer's merge reads: those wait for the predecessor
+  if (!p.early_inputs) pdl_wait();
   if (tid == 0) {                                       // this thread initialised the barrier
     mbar_arrive_expect_tx(&bars[0], kTcQTileBytes);
     const uint64_t pol = l2_policy_evict_last();
@@ -223,6 +227,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       mbar_wait(&bars[2], ph ^ 1, kErrWaitTmemFull, abort_flag);
       tc_fence_after();
     }
+    if (p.early_inputs && !window && it == 0) pdl_wait();
     int v = 0;
     if (tid < kTcAttnKeys) {
       if (tid < nkeys) {
@@ -383,6 +388,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         ref_s[h] = nref;
         sum_s[h] = sum_s[h] * f + l;
         if (!p.per_query) {
+          if (p.early_inputs && window) pdl_wait();
           float* ml = p.ml + ((static_cast<int64_t>(bq) * p.slices + slice) * 64 + h) * 2;
           ml[0] = nref;
           ml[1] = l;
@@ -470,6 +476,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (p.early_inputs) pdl_wait();                       // window-only CTAs have not waited yet
   if (*abort_flag) return;
   if (!p.per_query) {
     float4* op = reinterpret_cast<float4*>(p.opart + (static_cast<int64_t>(bq) * p.slices + first_slice) * 64 * 512);

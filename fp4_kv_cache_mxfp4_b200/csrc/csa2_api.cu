@@ -380,7 +380,9 @@ size_t attn_ws_bytes(const csa2_attn_args* a) {
   return up256(bq * s * 64 * 512 * 4) + up256(bq * s * 64 * 2 * 4);
 }
 
-csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
+// early_inputs: the attention follows a kernel of this library in the same
+// call (group), so q and the window rows are already complete
+csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st, bool early_inputs = false) {
   const float scale = a->scale > 0.0f ? a->scale : 1.0f / sqrtf(512.0f);
   const size_t bq = static_cast<size_t>(a->B) * a->Q;
   const int slices = attn_slices(a);
@@ -397,6 +399,7 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st) {
   t.scale_log2 = scale * 1.4426950408889634f;
   const bool per_query = attn_per_query(a);
   t.per_query = per_query ? 1 : 0;
+  t.early_inputs = early_inputs ? 1 : 0;
   t.opart = per_query ? nullptr : opart;
   t.ml = per_query ? nullptr : ml;
   t.out = static_cast<__nv_bfloat16*>(a->out);
@@ -600,7 +603,7 @@ csa2_status csa2_group_decode(const csa2_group_args* g, void* ws, size_t ws_byte
       last_idx = L.idx;
     }
     const csa2_attn_args aa = layer_attn_args(g, L, last_idx);
-    s = run_attn(&aa, aws, st);
+    s = run_attn(&aa, aws, st, true);
     if (s != CSA2_OK) return s;
   }
   return CSA2_OK;

@@ -125,9 +125,12 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) hist_s[i] = 0;
   if (HSI) for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) bhist_s[i] = 0;
 
-  // the inputs below, and the score buffers this kernel overwrites, belong
-  // to earlier kernels in the stream until they have completed
-  pdl_wait();
+  // Index-K, index-Q, weights and n_vis are the caller's: complete before
+  // this kernel can start (its predecessor is the call's memset node or a
+  // kernel of this library that waited for everything before it), so the
+  // pipeline fills at once.  What waits for the predecessor: the HSI pool
+  // (a previous top-K wrote it) and every global store (the score buffer is
+  // shared with the previous layer's top-K).
   pdl_launch_dependents();
 
   // this CTA's tile range; in scan mode, tiles past every query's n_vis are skipped
@@ -154,6 +157,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && ntiles > 0) {
+      if (p.pool_mode) pdl_wait();
       const uint64_t pol_stream = l2_policy_evict_first();
       const uint64_t pol_keep = l2_policy_evict_last();
       uint8_t* qi = smem + L.qi0;
@@ -215,6 +219,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    pdl_wait();                                   // before the first score store
     const int quarter = warp & 3;                 // TMEM lanes this warp may read
     const int set = (warp - 2) >> 2;              // tiles set, set+2, set+4, ...
     const int row = quarter * 32 + lane;          // entry within the tile

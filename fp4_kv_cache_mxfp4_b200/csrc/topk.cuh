@@ -234,8 +234,8 @@ topk_select_kernel(TopkParams p) {
 
   const int bq = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_wait();
   pdl_launch_dependents();
+  pdl_wait();
   const float* row = p.scores + static_cast<int64_t>(bq) * p.ld;
   float* stage_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(keys_s) + static_cast<size_t>(kTopkCap) * 8);
 
