@@ -7,22 +7,25 @@
 //
 // One thread-block cluster of C CTAs per selection problem (grid (C,
 // queries), 512 threads per CTA); CTA r of the cluster owns the r-th of C
-// contiguous slices of the query's visible slots.
+// contiguous slices of the query's slots, and warp w of a CTA the w-th of
+// 16 contiguous ranges of its slice.
 //  0. every CTA reads the query's score histogram (built by the scan
 //     epilogue, coalesced) and finds the threshold bin tb, the highest bin
 //     whose suffix count reaches need = min(K, visible): every top-K key has
 //     its top bits >= tb;
-//  1. every CTA streams its slice with 16-byte loads and compacts the keys
-//     whose bin is >= tb into its own shared memory, in position order
-//     (warp prefix sums, one block scan per 8192 slots);
-//  2. the CTAs publish their counts to the cluster's first CTA, which pulls
-//     the other CTAs' candidates over distributed shared memory (in slice
-//     order, so the list stays in position order), radix-selects the
-//     need-th largest key (8-bit digits from the top) and writes the keys at
-//     or above it by an ordered compaction: the result comes out in
-//     ascending position order, deterministically, without a sort.
-// If the candidates do not fit in the first CTA's shared memory (massive
-// ties), step 2 runs over the scores themselves with the same filter
+//  1. every warp streams its range in 2 KB bulk copies through its own
+//     three-stage ring (issued before the histogram is read) and compacts
+//     the keys whose bin is >= tb into its own region, in position order
+//     (four ballots per vector, no block-wide barrier); the warp lists are
+//     then joined into the CTA's list;
+//  2. the CTAs exchange their counts over distributed shared memory and push
+//     their lists into the cluster's first CTA (in slice order, so the list
+//     stays in position order), which radix-selects the need-th largest key
+//     (8-bit digits) and writes the keys at or above it by an ordered
+//     compaction: the result comes out in ascending position order,
+//     deterministically, without a sort.
+// If the candidates do not fit (massive ties) or an estimated threshold
+// fails, step 2 runs over the scores themselves with the same filter
 // (slower, exact).
 // HBM roofline: 4 B per score read (normally still resident in L2).
 #pragma once
@@ -36,9 +39,9 @@ namespace cg = cooperative_groups;
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkVec = 4;                                  // float4 per lane per chunk
-constexpr int kTopkWarpSlots = 32 * 4 * kTopkVec;            // 512 contiguous slots per warp per chunk
-constexpr int kTopkChunkSlots = kTopkWarps * kTopkWarpSlots; // 8192 slots (32 KB) per chunk
-constexpr int kTopkStages = 3;                               // chunks in flight (bulk copies into shared memory)
+constexpr int kTopkWarpSlots = 32 * 4 * kTopkVec;            // 512 slots (2 KB) per warp chunk
+constexpr int kTopkStages = 3;                               // chunks in flight per warp (bulk copies)
+constexpr int kTopkWarpCap = 768;                            // candidates a warp may hold (kTopkCap / 16)
 constexpr int kTopkCap = 12288;                             // candidate keys a CTA holds (the cluster's total)
 constexpr int kTopkMaxCluster = 16;                         // 16 needs the non-portable cluster attribute
 
@@ -69,7 +72,8 @@ struct TopkShared {
   uint32_t cnt[kTopkMaxCluster];   // candidates found by each CTA of the cluster
   int d, gt, eq, total, tb, above;  // above: visible slots in bins higher than tb
   int abort_flag;
-  alignas(8) uint64_t full_bar[kTopkStages];
+  uint32_t wcnt[kTopkWarps];                 // candidates found by each warp
+  alignas(8) uint64_t wbar[kTopkWarps][kTopkStages];
 };
 
 __device__ __forceinline__ int64_t topk_valid_slots(const TopkParams& p, int bq) {
@@ -237,35 +241,43 @@ topk_select_kernel(TopkParams p) {
   pdl_launch_dependents();
   pdl_wait();
   const float* row = p.scores + static_cast<int64_t>(bq) * p.ld;
-  float* stage_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(keys_s) + static_cast<size_t>(kTopkCap) * 8);
+  // stage ring [warp][stage][512 floats]; after streaming the same bytes hold
+  // the CTA's contiguous candidate list (kTopkCap keys)
+  float* ring_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(keys_s) + static_cast<size_t>(kTopkCap) * 8);
+  uint64_t* cand_s = reinterpret_cast<uint64_t*>(ring_s);
 
-  // this CTA's slice of the slots, streamed kTopkChunkSlots at a time by
-  // bulk copies into a kTopkStages-deep ring of shared memory; warp w reads
-  // the chunk's slots [512w, 512w + 512), lane l the four at 128j + 4l.
-  // Slices split all n_elems slots, so the first copies go out before the
-  // visible count arrives; slots at or past it are masked afterwards.
+  // this CTA's slice of the slots, cut into 16 contiguous warp ranges; each
+  // warp streams its range in 512-slot chunks through its own ring of bulk
+  // copies and compacts its candidates into its own region of keys_s, in
+  // position order, without block-wide barriers.  Slices split all n_elems
+  // slots, so the first copies go out before the visible count arrives;
+  // slots at or past it are masked afterwards.
   const int64_t span = (((p.n_elems + C - 1) / C) + 3) & ~static_cast<int64_t>(3);
   const int64_t lo = min(p.n_elems, static_cast<int64_t>(rank) * span);
-  int64_t hi = min(p.n_elems, lo + span);
-  const int64_t hi_copy = hi;                          // copies stay inside the slice's padded row
-  auto issue_chunk = [&](int64_t c0, int k) {          // thread 0: chunk at slot c0 into stage k % kTopkStages
-    if (c0 >= hi_copy) return;
+  const int64_t hi_copy = min(p.n_elems, lo + span);   // copies stay inside the slice's padded row
+  const int64_t wspan = (((hi_copy - lo + kTopkWarps - 1) / kTopkWarps) + 3) & ~static_cast<int64_t>(3);
+  const int64_t wlo = min(hi_copy, lo + warp * wspan);
+  const int64_t whi_copy = min(hi_copy, wlo + wspan);
+  float* wring = ring_s + warp * kTopkStages * kTopkWarpSlots;
+  uint64_t* wbar = S.wbar[warp];
+  auto issue_chunk = [&](int64_t c0, int k) {          // lane 0: chunk at slot c0 into stage k % kTopkStages
+    if (c0 >= whi_copy) return;
     const int st = k % kTopkStages;
-    const uint32_t n4 = static_cast<uint32_t>(min(static_cast<int64_t>(kTopkChunkSlots), hi_copy - c0) + 3) & ~3u;
-    mbar_arrive_expect_tx(&S.full_bar[st], n4 * 4);
+    const uint32_t n4 = static_cast<uint32_t>(min(static_cast<int64_t>(kTopkWarpSlots), whi_copy - c0) + 3) & ~3u;
+    mbar_arrive_expect_tx(&wbar[st], n4 * 4);
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        :: "r"(smem_u32(stage_s + st * kTopkChunkSlots)), "l"(row + c0), "r"(n4 * 4), "r"(smem_u32(&S.full_bar[st]))
+        :: "r"(smem_u32(wring + st * kTopkWarpSlots)), "l"(row + c0), "r"(n4 * 4), "r"(smem_u32(&wbar[st]))
         : "memory");
   };
-  if (tid == 0) {
-    for (int k = 0; k < kTopkStages; ++k) mbar_init(&S.full_bar[k], 1);
-    S.abort_flag = 0;
+  if (lane == 0) {
+    for (int k = 0; k < kTopkStages; ++k) mbar_init(&wbar[k], 1);
     fence_barrier_init();
-    for (int k = 0; k < kTopkStages; ++k) issue_chunk(lo + static_cast<int64_t>(k) * kTopkChunkSlots, k);
+    for (int k = 0; k < kTopkStages; ++k) issue_chunk(wlo + static_cast<int64_t>(k) * kTopkWarpSlots, k);
   }
+  if (tid == 0) S.abort_flag = 0;
   const int64_t nvalid = topk_valid_slots(p, bq);
-  hi = min(hi, nvalid);
+  const int64_t whi = min(whi_copy, nvalid);
 
   // -- 0. threshold bin: thread t owns the `per` bins just below bin
   //       nbins - per*t (descending ranges), read with coalesced loads
@@ -327,18 +339,19 @@ topk_select_kernel(TopkParams p) {
   }
   const int tb = S.tb;
 
-  // -- 1. this CTA's slice: candidates into shared memory, in position order
-  uint32_t n = 0;                                     // candidates so far (uniform over the block)
+  // -- 1. this warp's range: candidates into its region, in position order
+  uint32_t n = 0;                                     // the CTA's candidates (after the gather below)
   {
     const uint32_t lt = (1u << lane) - 1u;             // lanes below this one
-    const int lane_slot = warp * kTopkWarpSlots + 4 * lane;   // this lane's first slot in a chunk
+    uint64_t* wkeys = keys_s + warp * kTopkWarpCap;
+    uint32_t wn = 0;                                   // this warp's candidates so far (uniform in the warp)
     int k = 0;
-    for (int64_t c0 = lo; c0 < hi; c0 += kTopkChunkSlots, ++k) {
+    for (int64_t c0 = wlo; c0 < whi; c0 += kTopkWarpSlots, ++k) {
       const int st = k % kTopkStages;
-      const bool ok = mbar_wait(&S.full_bar[st], (k / kTopkStages) & 1, kErrWaitOperand, &S.abort_flag);
+      const bool ok = mbar_wait(&wbar[st], (k / kTopkStages) & 1, kErrWaitOperand, &S.abort_flag);
       float4 cur[kTopkVec];
-      const int64_t left = hi - c0 - lane_slot;        // visible slots from this lane's first on
-      const float4* src = reinterpret_cast<const float4*>(stage_s + st * kTopkChunkSlots + lane_slot);
+      const int64_t left = whi - c0 - 4 * lane;        // visible slots from this lane's first on
+      const float4* src = reinterpret_cast<const float4*>(wring + st * kTopkWarpSlots) + lane;
 #pragma unroll
       for (int j = 0; j < kTopkVec; ++j) {
         cur[j] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
@@ -352,54 +365,60 @@ topk_select_kernel(TopkParams p) {
           }
         }
       }
-      // position order inside the warp is (j, lane, component): four
+      __syncwarp();
+      if (lane == 0) {                                 // every lane holds its values: refill the stage
+        fence_async_smem_generic();
+        issue_chunk(c0 + static_cast<int64_t>(kTopkStages) * kTopkWarpSlots, k + kTopkStages);
+      }
+      // position order inside the chunk is (j, lane, component): four
       // ballots per j give each lane its offset without a serial scan
-      uint32_t fl[kTopkVec], pre[kTopkVec], wtot = 0;
 #pragma unroll
       for (int j = 0; j < kTopkVec; ++j) {
         const bool f0 = topk_is_cand(cur[j].x, tb, p.hb), f1 = topk_is_cand(cur[j].y, tb, p.hb);
         const bool f2 = topk_is_cand(cur[j].z, tb, p.hb), f3 = topk_is_cand(cur[j].w, tb, p.hb);
         const uint32_t b0 = __ballot_sync(0xffffffffu, f0), b1 = __ballot_sync(0xffffffffu, f1);
         const uint32_t b2 = __ballot_sync(0xffffffffu, f2), b3 = __ballot_sync(0xffffffffu, f3);
-        fl[j] = (f0 ? 1u : 0u) | (f1 ? 2u : 0u) | (f2 ? 4u : 0u) | (f3 ? 8u : 0u);
-        pre[j] = wtot + __popc(b0 & lt) + __popc(b1 & lt) + __popc(b2 & lt) + __popc(b3 & lt);
-        wtot += __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
-      }
-      uint32_t btot;
-      const uint32_t wofs = n + topk_block_scan(lane == 0 ? wtot : 0u, S, &btot);
-      // every thread holds its values: the stage can be refilled
-      if (tid == 0) {
-        fence_async_smem_generic();
-        issue_chunk(c0 + static_cast<int64_t>(kTopkStages) * kTopkChunkSlots, k + kTopkStages);
-      }
-      const uint32_t wbase_ofs = __shfl_sync(0xffffffffu, wofs, 0);
-      if (wtot != 0) {
-        const int64_t s_lane = c0 + lane_slot;
-#pragma unroll
-        for (int j = 0; j < kTopkVec; ++j) {
-          if (fl[j] == 0) continue;
-          uint32_t o = wbase_ofs + pre[j];
+        const uint32_t tot = __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
+        if (tot != 0) {
+          uint32_t o = wn + __popc(b0 & lt) + __popc(b1 & lt) + __popc(b2 & lt) + __popc(b3 & lt);
+          const int64_t s0 = c0 + 128 * j + 4 * lane;
           const float v[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+          const bool f[4] = {f0, f1, f2, f3};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            if (fl[j] & (1u << c)) {
-              if (o < static_cast<uint32_t>(kTopkCap)) keys_s[o] = topk_make_key(p, bq, s_lane + 128 * j + c, v[c]);
+            if (f[c]) {
+              if (o < static_cast<uint32_t>(kTopkWarpCap)) wkeys[o] = topk_make_key(p, bq, s0 + c, v[c]);
               ++o;
             }
           }
         }
+        wn += tot;
       }
-      n += btot;
     }
-    // copies issued past the visible end (speculatively) land before exit
-    if (tid == 0) {
-      const int64_t kcopy = (hi_copy - lo + kTopkChunkSlots - 1) / kTopkChunkSlots;   // chunks in the slice
+    // copies issued past the visible end (speculatively) land before the
+    // ring is reused
+    if (lane == 0) {
+      const int64_t kcopy = (whi_copy - wlo + kTopkWarpSlots - 1) / kTopkWarpSlots;   // chunks in the range
       const int64_t kissued = min(kcopy, static_cast<int64_t>(k) + kTopkStages);
       volatile int keep_waiting = 0;                   // bounded even after an earlier wait gave up
       for (int64_t kk = k; kk < kissued; ++kk)
-        mbar_wait(&S.full_bar[kk % kTopkStages], static_cast<uint32_t>((kk / kTopkStages) & 1), kErrWaitOperand,
+        mbar_wait(&wbar[kk % kTopkStages], static_cast<uint32_t>((kk / kTopkStages) & 1), kErrWaitOperand,
                   &keep_waiting);
+      S.wcnt[warp] = wn;
     }
+    __syncthreads();
+    // the warp lists, in warp order, into one contiguous list over the ring
+    bool wfit = true;
+    uint32_t off = 0;
+    for (int w = 0; w < kTopkWarps; ++w) {
+      const uint32_t c = S.wcnt[w];
+      wfit = wfit && c <= static_cast<uint32_t>(kTopkWarpCap);
+      if (w < warp) off += min(c, static_cast<uint32_t>(kTopkWarpCap));
+      n += c;
+    }
+    for (uint32_t i = lane; i < min(wn, static_cast<uint32_t>(kTopkWarpCap)); i += 32) cand_s[off + i] = wkeys[i];
+    if (!wfit) n = kTopkCap + 1;                       // a warp overflowed: take the exact path
+    __syncthreads();
   }
 
   // -- 2. counts to every CTA; the others push their lists into the first
@@ -417,8 +436,8 @@ topk_select_kernel(TopkParams p) {
   }
   fits = fits && n_all <= static_cast<uint32_t>(kTopkCap);
   if (fits && need > 0 && rank > 0) {
-    uint64_t* dst = cluster.map_shared_rank(keys_s, 0) + my_off;
-    for (uint32_t i = tid; i < n; i += kTopkThreads) dst[i] = keys_s[i];
+    uint64_t* dst = cluster.map_shared_rank(cand_s, 0) + my_off;
+    for (uint32_t i = tid; i < n; i += kTopkThreads) dst[i] = cand_s[i];
   }
   cluster.sync();                                     // the first CTA holds every list; the rest may exit
   if (rank != 0) return;
@@ -433,9 +452,9 @@ topk_select_kernel(TopkParams p) {
       uint64_t P;
       if (p.hist_sample == 1)
         P = topk_radix_select<false>(S, n_all, need, p.hb, static_cast<uint64_t>(tb) << (64 - p.hb), S.above,
-                                     [&](int64_t i) { return keys_s[i]; });
+                                     [&](int64_t i) { return cand_s[i]; });
       else    // the K-th key's bin is unknown: full-width passes, equal digits aggregated
-        P = topk_radix_select<true>(S, n_all, need, 0, 0, 0, [&](int64_t i) { return keys_s[i]; });
+        P = topk_radix_select<true>(S, n_all, need, 0, 0, 0, [&](int64_t i) { return cand_s[i]; });
       // ordered compaction of the keys >= P (4 consecutive keys per thread)
       for (uint32_t i0 = 0; i0 < n_all; i0 += 4 * kTopkThreads) {
         uint64_t k[4];
@@ -443,7 +462,7 @@ topk_select_kernel(TopkParams p) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t j = i0 + 4 * tid + i;
-          k[i] = (j < n_all) ? keys_s[j] : 0;
+          k[i] = (j < n_all) ? cand_s[j] : 0;
           if (k[i] < P) k[i] = 0;
           m += (k[i] != 0);
         }
@@ -499,8 +518,10 @@ topk_select_kernel(TopkParams p) {
 }
 
 inline size_t topk_smem_bytes() {
+  // warp regions of candidates, then the stage rings (which later hold the
+  // contiguous candidate list: both are kTopkCap keys)
   return ((sizeof(TopkShared) + 15) & ~size_t(15)) + static_cast<size_t>(kTopkCap) * 8 +
-         static_cast<size_t>(kTopkStages) * kTopkChunkSlots * 4;
+         static_cast<size_t>(kTopkWarps) * kTopkStages * kTopkWarpSlots * 4;
 }
 
 // CTAs per selection problem: enough to spread a long score row over SMs
