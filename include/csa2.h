@@ -194,6 +194,12 @@ csa2_status csa2_index_score_topk_noalloc(const csa2_index_args* a, void* stream
  *
  * idx entries must be -1 or in [0, N); the window rows read must lie inside
  * [0, swa_rows).
+ *
+ * With fewer than 128 queries per call (B*Q) the keys of a query are split
+ * into 128-key slices over several CTAs whose fp32 partial outputs go to
+ * the workspace and are merged by a second kernel; with 128 or more, one
+ * CTA per query walks all its slices and the workspace is not used
+ * (csa2_workspace_size still returns a small non-zero size).
  * ---------------------------------------------------------------------- */
 typedef struct csa2_attn_args {
     int32_t        B, Q;        /* batch rows >= 1; queries per row, B*Q <= CSA2_MAX_BQ */
@@ -259,7 +265,13 @@ csa2_status csa2_group_decode(const csa2_group_args* g, void* ws,
 
 /* Workspace bytes needed by a call.  which = 1: csa2_index_args,
  * 2: csa2_attn_args, 3: csa2_group_args.  Returns 0 when the arguments are
- * invalid for that call. */
+ * invalid for that call.
+ *
+ * Launches: every kernel is launched with programmatic stream serialisation
+ * (it may start while the previous kernel in the stream finishes, and waits
+ * for it before touching memory that kernel owns).  Setting the environment
+ * variable CSA2_PDL=0 before the first call launches them in plain stream
+ * order. */
 #define CSA2_WS_INDEX 1
 #define CSA2_WS_ATTN  2
 #define CSA2_WS_GROUP 3
