@@ -64,16 +64,22 @@ def parse():
 # distributed plumbing (barrier and max-reduction only)
 # ---------------------------------------------------------------------------
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE).
+    Ranks are replicas: each runs its own batch rows, and the only traffic
+    between them is the barrier and the max-reduction of timings."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -84,11 +90,19 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The slowest rank's figure (every rank gets it)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_queries_per_s(queries_per_rank, world, max_ms_per_step):
+    """Whole-job throughput: every rank's queries over the slowest rank's
+    step time (weak scaling: the work per rank is fixed)."""
+    return queries_per_rank * world / (max_ms_per_step * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -426,7 +440,7 @@ def run_ours(args, world, rank, local):
     if rank != 0:
         return
     queries = wl.B * wl.Q * world
-    value = queries / (mean_ms * 1e-3)
+    value = aggregate_queries_per_s(wl.B * wl.Q, world, mean_ms)
     peak, peak_kind = hbm_peak()
     n_scan, t_scan = per_kernel.get("index_scan_kernel", (0, 0.0))
     scan_ms = t_scan / max(n_scan, 1)
