@@ -93,3 +93,22 @@ def test_window_rows_follow_the_query_position():
     for i in range(Q):
         want = sum(range(i * step, i * step + W)) / (K + W)
         np.testing.assert_allclose(res[0]["o"][i][:, 0], want, rtol=1e-12)
+
+
+def test_prefill_visibility_follows_token_coverage():
+    """Causal prefill inputs: entry j covers tokens [j*r, (j+1)*r) and a query
+    at token p sees it once all its tokens are at or before p; the visible
+    count per query, counted entry by entry, matches the workload's n_vis,
+    and the window of query i starts at row i (one new window row per token)."""
+    from fp4_kv_cache_mxfp4_b200 import workloads
+    for r, n_prefix, n_new in [(2, 40, 12), (1, 17, 5), (4, 9, 6)]:
+        N = n_prefix + n_new
+        Q = n_new * r
+        wl = workloads.Workload("t", 0, B=1, Q=Q, N=N, r=r, modes=[0], n_new=n_new, prefill=True, swa_step=1)
+        p0 = n_prefix * r                             # first query's token
+        for i in range(Q):
+            p = p0 + i
+            visible = sum(1 for j in range(N) if (j + 1) * r <= p + 1)
+            assert wl.n_vis[i] == visible, (r, i)
+        assert wl.n_vis[-1] == N                      # the last query sees every entry
+        assert wl.swa_rows == wl.W + Q - 1
