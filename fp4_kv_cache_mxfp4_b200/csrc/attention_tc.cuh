@@ -33,7 +33,6 @@
 namespace csa2 {
 
 constexpr int kTcAttnThreads = 512;
-constexpr int kTcAttnWarps = kTcAttnThreads / 32;
 constexpr int kTcAttnKeys = 128;                       // keys per slice (MMA M)
 constexpr uint32_t kTcKeyTileBytes = 128 * 512 * 2;    // 128 KB: 8 chunks of [128 rows x 64 dims]
 constexpr uint32_t kTcQTileBytes = 64 * 512 * 2;       // 64 KB: 8 chunks of [64 rows x 64 dims]
