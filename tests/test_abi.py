@@ -204,3 +204,18 @@ def test_arg_structs_keep_their_tensors_alive():
     gc.collect()
     assert ref_nv() is not None
     assert a is not None and at is not None and g is not None
+
+
+def test_workspace_sizes_for_prefill_shapes(L):
+    """4096 causal queries over 133,120 entries: scores padded to a multiple
+    of 4 slots per query, 2048-bin histograms for 8-query MMA groups, and
+    attention with one CTA per query needs no partials."""
+    a = _index(B=1, Q=4096, K=512, N=133121)
+    n = L.csa2_workspace_size(ctypes.byref(a), csa2.WS_INDEX)
+    ld = (133121 + 3) // 4 * 4
+    assert n >= 4096 * ld * 4 + 4096 * 2048 * 4
+    assert n < 4096 * ld * 4 + 4096 * 2048 * 4 + 4096
+    at = _attn(B=1, Q=4096, K=512, W=128, swa_step=1, swa_rows=128 + 4095)
+    assert 0 < L.csa2_workspace_size(ctypes.byref(at), csa2.WS_ATTN) <= 256
+    small = _attn(B=1, Q=127, K=512, W=128, swa_step=1, swa_rows=128 + 126)
+    assert L.csa2_workspace_size(ctypes.byref(small), csa2.WS_ATTN) >= 127 * 5 * 64 * 512 * 4
