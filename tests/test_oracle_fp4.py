@@ -64,6 +64,36 @@ def test_golden_blocks_through_entry_packing():
             assert nib == codes[i], (name, i)
 
 
+def test_golden_entry_dequantises_to_the_golden_values():
+    """The packed golden entry through unpack_codes and dequantize_kv_fp4:
+    every channel equals the hand-worked dequantised value bit for bit,
+    the sign of zero included (a swapped nibble order, a scale applied to
+    the wrong block or a dropped sign fails here).  The blocks are placed
+    in reverse order in the second row, so the block-to-scale pairing is
+    tested at two different offsets."""
+    blocks = _golden_blocks()
+    n = len(blocks)
+    x = np.zeros((2, 512), dtype=np.float32)
+    want = np.zeros((2, 512), dtype=np.float64)
+    want_codes = np.zeros((2, 512), dtype=np.uint8)
+    want_scales = np.zeros((2, 32), dtype=np.uint8)
+    for k, (_, xs, sc, codes, deq) in enumerate(blocks):
+        for row, blk in ((0, k), (1, 31 - k)):
+            x[row, 16 * blk:16 * blk + 16] = xs
+            want[row, 16 * blk:16 * blk + 16] = deq
+            want_codes[row, 16 * blk:16 * blk + 16] = codes
+            want_scales[row, blk] = sc
+    packed = fp4.quantize_kv_fp4(x)
+    codes, scales = fp4.unpack_codes(packed)
+    np.testing.assert_array_equal(codes, want_codes)
+    np.testing.assert_array_equal(scales, want_scales)
+    got = fp4.dequantize_kv_fp4(packed)
+    assert got.dtype == np.float64 and got.shape == (2, 512)
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(np.signbit(got), np.signbit(want))
+    assert n >= 11 and np.signbit(want).any()
+
+
 def test_e4m3_decode_matches_torch_for_all_codes():
     codes = np.arange(256, dtype=np.uint8)
     ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float32).numpy().astype(np.float64)
