@@ -15,7 +15,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcsa2.so")
 
 FULL, REINDEX, REINDEX_POOL, REUSE = 0, 1, 2, 3
-WS_INDEX, WS_ATTN, WS_GROUP = 1, 2, 3
+WS_INDEX, WS_ATTN, WS_GROUP, WS_STACK = 1, 2, 3, 4
+GROUP_INPUTS_READY, GROUP_SERIAL = 1, 2
 ENTRY_BYTES = 288
 
 _c_i32, _c_i64, _c_f32, _c_p = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
@@ -50,7 +51,11 @@ class GroupArgs(ctypes.Structure):
                 ("n_vis", _c_p), ("kI", _c_p), ("kv_fp4", _c_p), ("kv_new", _c_p), ("n_new", _c_i64),
                 ("new_rows", _c_p), ("swa_rows", _c_i32), ("swa_step", _c_i32),
                 ("hsi_blocks", _c_i32), ("hsi_block", _c_i32), ("pool", _c_p), ("scale", _c_f32),
-                ("n_layers", _c_i32), ("layers", ctypes.POINTER(Layer))]
+                ("n_layers", _c_i32), ("layers", ctypes.POINTER(Layer)), ("pool_in", _c_p), ("flags", _c_i32)]
+
+
+class StackArgs(ctypes.Structure):
+    _fields_ = [("n_groups", _c_i32), ("groups", ctypes.POINTER(GroupArgs))]
 
 
 _lib = None
@@ -70,6 +75,9 @@ def load(path=LIB_PATH):
     lib.csa2_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexArgs), _c_p]
     lib.csa2_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_group_decode.argtypes = [ctypes.POINTER(GroupArgs), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_stack_decode.argtypes = [ctypes.POINTER(StackArgs), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_noalloc_scratch_bytes.argtypes = []
+    lib.csa2_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.csa2_workspace_size.argtypes = [_c_p, _c_i32]
     lib.csa2_workspace_size.restype = ctypes.c_size_t
     lib.csa2_device_status.argtypes = [ctypes.POINTER(_c_i32), _c_p]
@@ -84,7 +92,7 @@ def load(path=LIB_PATH):
     lib.csa2_kernel_name.argtypes = [_c_i32]
     lib.csa2_kernel_name.restype = ctypes.c_char_p
     for name in ("csa2_quantize_kv_fp4", "csa2_index_score_topk", "csa2_index_score_topk_noalloc", "csa2_sparse_attn",
-                 "csa2_group_decode", "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
+                 "csa2_group_decode", "csa2_stack_decode", "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
                  "csa2_trace_end", "csa2_trace_get"):
         getattr(lib, name).restype = _c_i32
     _lib = lib
@@ -156,7 +164,10 @@ def csa2_index_score_topk_noalloc(args, stream=None):
            "csa2_index_score_topk_noalloc")
 
 
-NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+def noalloc_scratch_bytes():
+    """Size of the library's fixed scratch array behind the no-allocation
+    index call, as compiled into libcsa2.so."""
+    return int(load().csa2_noalloc_scratch_bytes())
 
 
 def attn_args(q, kv_fp4, idx, swa, out, lse=None, W=128, swa_step=0, scale=0.0):
@@ -177,10 +188,11 @@ def csa2_sparse_attn(args, ws, stream=None):
 
 
 def group_args(B, Q, K, W, N, n_vis, kI, kv_fp4, layers, kv_new=None, new_rows=None, swa_rows=128, swa_step=0,
-               hsi_blocks=0, hsi_block=8, pool=None, scale=0.0):
+               hsi_blocks=0, hsi_block=8, pool=None, scale=0.0, pool_in=None, flags=0):
     """``layers`` is a list of dicts with keys mode, qI, w, q, swa, out, lse,
-    idx, scores (tensors or None).  The returned struct keeps its layer
-    array alive."""
+    idx, scores (tensors or None).  ``pool_in`` is an HSI pool built by an
+    earlier group; ``flags`` a combination of GROUP_INPUTS_READY and
+    GROUP_SERIAL.  The returned struct keeps its layer array alive."""
     arr = (Layer * len(layers))()
     for i, L in enumerate(layers):
         arr[i] = Layer(mode=L["mode"], qI=_ptr(L.get("qI")), w=_ptr(L.get("w")), q=_ptr(L["q"]),
@@ -190,11 +202,27 @@ def group_args(B, Q, K, W, N, n_vis, kI, kv_fp4, layers, kv_new=None, new_rows=N
                   kv_new=_ptr(kv_new), n_new=0 if kv_new is None else kv_new.shape[0], new_rows=_ptr(new_rows),
                   swa_rows=swa_rows, swa_step=swa_step, hsi_blocks=hsi_blocks, hsi_block=hsi_block,
                   pool=_ptr(pool), scale=scale, n_layers=len(layers),
-                  layers=ctypes.cast(arr, ctypes.POINTER(Layer)))
+                  layers=ctypes.cast(arr, ctypes.POINTER(Layer)), pool_in=_ptr(pool_in), flags=flags)
     g._layer_array = arr
     # the structs hold raw pointers: keep every tensor alive with them
-    g._tensors = (n_vis, kI, kv_fp4, kv_new, new_rows, pool, [dict(L) for L in layers])
+    g._tensors = (n_vis, kI, kv_fp4, kv_new, new_rows, pool, pool_in, [dict(L) for L in layers])
     return g
+
+
+def stack_args(groups):
+    """csa2_stack_args over a list of group_args structs (kept alive)."""
+    arr = (GroupArgs * len(groups))()
+    for i, g in enumerate(groups):
+        arr[i] = g
+    s = StackArgs(n_groups=len(groups), groups=ctypes.cast(arr, ctypes.POINTER(GroupArgs)))
+    s._group_array = arr
+    s._groups = list(groups)
+    return s
+
+
+def csa2_stack_decode(args, ws, stream=None):
+    _check(load().csa2_stack_decode(ctypes.byref(args), _ptr(ws), ws.numel() * ws.element_size(),
+                                    _stream(stream)), "csa2_stack_decode")
 
 
 def csa2_group_decode(args, ws, stream=None):

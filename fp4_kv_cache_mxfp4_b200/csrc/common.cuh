@@ -32,6 +32,9 @@ static LaunchTrace g_trace;
 // cluster_x > 0 adds a (cluster_x, 1, 1) thread-block cluster shape.
 // Tracing records events between launches, which serialises them as usual.
 static bool g_pdl = true;
+// set for the duration of a call whose kernels must run in plain stream
+// order (CSA2_GROUP_SERIAL); launches happen on the calling host thread
+static thread_local bool g_serial_launch = false;
 // last CUDA failure seen by a launch on this host thread (csa2_cuda_error_string)
 static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 template <typename... KArgs, typename... Args>
@@ -45,7 +48,7 @@ inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   unsigned n = 0;
-  if (g_pdl) {
+  if (g_pdl && !g_serial_launch) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;

@@ -250,8 +250,10 @@ int scan_ctas_per_group(int groups, int tiles, int sms) {
 // zero: the call's counter region (already zeroed); data: its data region
 // kv_prefetch: optional FP4 cache whose selected rows are pulled into L2 as
 // the top-K writes their indices (the group call's attention reads them next)
+// early_q: index-Q and w are complete when the scan starts (the caller's,
+// not a result of the kernel before it)
 csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zero, void* data, cudaStream_t st,
-                      const void* kv_prefetch = nullptr) {
+                      const void* kv_prefetch = nullptr, bool early_q = true) {
   const IndexPlan P = plan_index(a);
   uint8_t* z = static_cast<uint8_t*>(zero);
   uint8_t* w = static_cast<uint8_t*>(data);
@@ -279,6 +281,7 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   uint32_t cols = 32;
   while (cols < scan_acc_bufs(QG) * n_mma) cols <<= 1;
   sp.tmem_cols = cols;
+  sp.early_q = early_q ? 1 : 0;
   const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi);
   // three 32 KB stages per SM measured fastest (fewer bytes in flight per
   // stream keep DRAM pages open longer; 2, 4 and 6 stages were slower)
@@ -432,7 +435,9 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st, bool ea
 }
 
 // ---------------------------------------------------------------- group call
-csa2_index_args layer_index_args(const csa2_group_args* g, const csa2_layer& L) {
+// cur_pool: the pool REINDEX_POOL layers read at this point of the group
+// (the call's own pool once a FULL layer built it, else pool_in)
+csa2_index_args layer_index_args(const csa2_group_args* g, const csa2_layer& L, const int32_t* cur_pool) {
   csa2_index_args a;
   memset(&a, 0, sizeof(a));
   a.mode = L.mode; a.B = g->B; a.Q = g->Q; a.K = g->K; a.N = g->N;
@@ -441,7 +446,7 @@ csa2_index_args layer_index_args(const csa2_group_args* g, const csa2_layer& L) 
   a.hsi_blocks = (L.mode == CSA2_FULL || L.mode == CSA2_REINDEX_POOL) ? g->hsi_blocks : 0;
   a.hsi_block = g->hsi_block;
   a.pool_out = (L.mode == CSA2_FULL && g->hsi_blocks > 0) ? g->pool : nullptr;
-  a.pool_in = (L.mode == CSA2_REINDEX_POOL) ? g->pool : nullptr;
+  a.pool_in = (L.mode == CSA2_REINDEX_POOL) ? cur_pool : nullptr;
   return a;
 }
 
@@ -457,25 +462,28 @@ csa2_attn_args layer_attn_args(const csa2_group_args* g, const csa2_layer& L, co
 
 csa2_status validate_group(const csa2_group_args* g, size_t* index_zero, size_t* index_ws, size_t* attn_ws) {
   if (!g || !g->layers || g->n_layers < 1 || g->n_layers > 64) return CSA2_ERR_ARG;
+  if (g->flags & ~(CSA2_GROUP_INPUTS_READY | CSA2_GROUP_SERIAL)) return CSA2_ERR_ARG;
   if (g->n_new < 0) return CSA2_ERR_SHAPE;
   if (g->n_new > 0 && (!g->kv_new || !g->new_rows || !g->kv_fp4)) return CSA2_ERR_ARG;
   if (g->n_new > 0 && (!aligned16(g->kv_new) || !aligned16(g->kv_fp4) || !aligned16(g->new_rows))) return CSA2_ERR_ALIGN;
+  if (g->pool_in && !aligned16(g->pool_in)) return CSA2_ERR_ALIGN;
   size_t iz = 0, idata = 0;
-  bool have_idx = false, have_pool = false;
+  bool have_idx = false;
+  const int32_t* cur_pool = g->pool_in;
   for (int i = 0; i < g->n_layers; ++i) {
     const csa2_layer& L = g->layers[i];
     if (L.mode == CSA2_REUSE) {
       if (!have_idx) return CSA2_ERR_ARG;
     } else {
-      if (L.mode == CSA2_REINDEX_POOL && !have_pool) return CSA2_ERR_ARG;
-      const csa2_index_args a = layer_index_args(g, L);
+      if (L.mode == CSA2_REINDEX_POOL && !cur_pool) return CSA2_ERR_ARG;
+      const csa2_index_args a = layer_index_args(g, L, cur_pool);
       const csa2_status s = validate_index(&a);
       if (s != CSA2_OK) return s;
       const IndexPlan P = plan_index(&a);
       iz += P.zero_bytes;
       idata = std::max(idata, P.data_bytes);
       have_idx = true;
-      if (L.mode == CSA2_FULL && g->hsi_blocks > 0) have_pool = true;
+      if (L.mode == CSA2_FULL && g->hsi_blocks > 0) cur_pool = g->pool;
     }
     const csa2_attn_args aa = layer_attn_args(g, L, L.idx ? L.idx : g->layers[0].idx);
     const csa2_status s = validate_attn(&aa);
@@ -489,6 +497,69 @@ csa2_status validate_group(const csa2_group_args* g, size_t* index_zero, size_t*
   return CSA2_OK;
 }
 
+// Validation of a group beyond validate_group: every indexing layer has an
+// output index buffer.  *need = workspace bytes.
+csa2_status check_group(const csa2_group_args* g, size_t* iz, size_t* iw, size_t* need) {
+  size_t aw = 0;
+  const csa2_status s = validate_group(g, iz, iw, &aw);
+  if (s != CSA2_OK) return s;
+  for (int i = 0; i < g->n_layers; ++i)
+    if (g->layers[i].mode != CSA2_REUSE && !g->layers[i].idx) return CSA2_ERR_ARG;
+  *need = *iw + aw;
+  return CSA2_OK;
+}
+
+// Enqueue one validated group on `st` (workspace already large enough).
+csa2_status run_group(const csa2_group_args* g, size_t iz, size_t iw, const DeviceInfo& dev, void* ws,
+                      cudaStream_t st) {
+  struct SerialScope {                             // CSA2_GROUP_SERIAL: plain stream order for this call
+    bool prev;
+    explicit SerialScope(bool on) : prev(g_serial_launch) { if (on) g_serial_launch = true; }
+    ~SerialScope() { g_serial_launch = prev; }
+  } serial((g->flags & CSA2_GROUP_SERIAL) != 0);
+  const bool inputs_ready = (g->flags & CSA2_GROUP_INPUTS_READY) != 0;
+  uint8_t* zws = static_cast<uint8_t*>(ws);     // one counter region per indexing layer
+  uint8_t* dws = zws + iz;                         // data region shared by the layers in turn
+  uint8_t* aws = zws + iw;
+  if (cudaMemsetAsync(zws, 0, iz, st) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (g->n_new > 0) {
+    if (launch_quantize(g->kv_new, g->n_new, 512, g->kv_fp4, g->new_rows, 0, st) != cudaSuccess) return CSA2_ERR_CUDA;
+  }
+  const int32_t* last_idx = nullptr;
+  const int32_t* cur_pool = g->pool_in;
+  for (int i = 0; i < g->n_layers; ++i) {
+    const csa2_layer& L = g->layers[i];
+    // the first layer's inputs precede the call; a later layer's are, in a
+    // model, the previous layer's results unless the caller says otherwise
+    const bool early = inputs_ready || i == 0;
+    if (L.mode != CSA2_REUSE) {
+      const csa2_index_args a = layer_index_args(g, L, cur_pool);
+      const csa2_status s = run_index(&a, dev, zws, dws, st, g->kv_fp4, early);
+      if (s != CSA2_OK) return s;
+      zws += plan_index(&a).zero_bytes;
+      last_idx = L.idx;
+      if (L.mode == CSA2_FULL && g->hsi_blocks > 0) cur_pool = g->pool;
+    }
+    const csa2_attn_args aa = layer_attn_args(g, L, last_idx);
+    const csa2_status s = run_attn(&aa, aws, st, early);
+    if (s != CSA2_OK) return s;
+  }
+  return CSA2_OK;
+}
+
+csa2_status validate_stack(const csa2_stack_args* sa, size_t* need) {
+  if (!sa || !sa->groups || sa->n_groups < 1 || sa->n_groups > 64) return CSA2_ERR_ARG;
+  size_t mx = 0;
+  for (int i = 0; i < sa->n_groups; ++i) {
+    size_t iz = 0, iw = 0, n = 0;
+    const csa2_status s = check_group(&sa->groups[i], &iz, &iw, &n);
+    if (s != CSA2_OK) return s;
+    mx = std::max(mx, n);
+  }
+  *need = mx;
+  return CSA2_OK;
+}
+
 // ---------------------------------------------------------------- no-allocation variant
 // Scratch of csa2_index_score_topk_noalloc: one file-scope device array.
 // Every GPU that loads the library holds it until the process exits, and
@@ -497,20 +568,47 @@ csa2_status validate_group(const csa2_group_args* g, size_t* index_zero, size_t*
 // cudaGetSymbolAddress returns for the current device.
 constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(CSA2_NOALLOC_SCRATCH_BYTES);
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-void* g_noalloc_addr[kMaxDevices];
+// the address and the CUDA context it belongs to, per device: a context
+// destroyed and re-created (cudaDeviceReset) reloads the module, and the
+// array may then sit elsewhere
+struct NoAllocAddr {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+NoAllocAddr g_noalloc_addr[kMaxDevices];
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the first call on each device does it).
+CUcontext current_context() {
+  if (!g_ctx_get_current) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return nullptr;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  }
+  CUcontext c = nullptr;
+  if (g_ctx_get_current(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of the scratch array on the current device, looked up on
+// the first call in each device context (without a context handle, on
+// every call).
 csa2_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_noalloc_addr[dev]) {
+  NoAllocAddr& slot = g_noalloc_addr[dev];
+  CUcontext ctx = current_context();
+  if (!ctx || ctx != slot.ctx || !slot.addr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CSA2_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
+    slot.addr = p;
+    slot.ctx = current_context();                  // the lookup made the device's context current
   }
-  *out = g_noalloc_addr[dev];
+  *out = slot.addr;
   return CSA2_OK;
 }
 
@@ -574,40 +672,36 @@ csa2_status csa2_sparse_attn(const csa2_attn_args* a, void* ws, size_t ws_bytes,
   return run_attn(a, ws, static_cast<cudaStream_t>(stream));
 }
 
+
 csa2_status csa2_group_decode(const csa2_group_args* g, void* ws, size_t ws_bytes, void* stream) {
-  size_t iz = 0, iw = 0, aw = 0;
-  csa2_status s = validate_group(g, &iz, &iw, &aw);
+  size_t iz = 0, iw = 0, need = 0;
+  csa2_status s = check_group(g, &iz, &iw, &need);
   if (s != CSA2_OK) return s;
-  if (!ws || ws_bytes < iw + aw || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
-  for (int i = 0; i < g->n_layers; ++i)
-    if (g->layers[i].mode != CSA2_REUSE && !g->layers[i].idx) return CSA2_ERR_ARG;
+  if (!ws || ws_bytes < need || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
   DeviceInfo* dev = nullptr;
   s = device_info(&dev);
   if (s != CSA2_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* zws = static_cast<uint8_t*>(ws);     // one counter region per indexing layer
-  uint8_t* dws = zws + iz;                         // data region shared by the layers in turn
-  uint8_t* aws = zws + iw;
-  if (cudaMemsetAsync(zws, 0, iz, st) != cudaSuccess) return CSA2_ERR_CUDA;
-  if (g->n_new > 0) {
-    if (launch_quantize(g->kv_new, g->n_new, 512, g->kv_fp4, g->new_rows, 0, st) != cudaSuccess) return CSA2_ERR_CUDA;
-  }
-  const int32_t* last_idx = nullptr;
-  for (int i = 0; i < g->n_layers; ++i) {
-    const csa2_layer& L = g->layers[i];
-    if (L.mode != CSA2_REUSE) {
-      const csa2_index_args a = layer_index_args(g, L);
-      s = run_index(&a, *dev, zws, dws, st, g->kv_fp4);
-      if (s != CSA2_OK) return s;
-      zws += plan_index(&a).zero_bytes;
-      last_idx = L.idx;
-    }
-    const csa2_attn_args aa = layer_attn_args(g, L, last_idx);
-    s = run_attn(&aa, aws, st, true);
+  return run_group(g, iz, iw, *dev, ws, static_cast<cudaStream_t>(stream));
+}
+
+csa2_status csa2_stack_decode(const csa2_stack_args* sa, void* ws, size_t ws_bytes, void* stream) {
+  size_t need = 0;
+  csa2_status s = validate_stack(sa, &need);
+  if (s != CSA2_OK) return s;
+  if (!ws || ws_bytes < need || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  for (int i = 0; i < sa->n_groups; ++i) {
+    size_t iz = 0, iw = 0, n = 0;
+    check_group(&sa->groups[i], &iz, &iw, &n);
+    s = run_group(&sa->groups[i], iz, iw, *dev, ws, static_cast<cudaStream_t>(stream));
     if (s != CSA2_OK) return s;
   }
   return CSA2_OK;
 }
+
+size_t csa2_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 size_t csa2_workspace_size(const void* args, int32_t which) {
   if (!args) return 0;
@@ -620,8 +714,12 @@ size_t csa2_workspace_size(const void* args, int32_t which) {
     return validate_attn(a) == CSA2_OK ? attn_ws_bytes(a) : 0;
   }
   if (which == CSA2_WS_GROUP) {
-    size_t iz = 0, iw = 0, aw = 0;
-    return validate_group(static_cast<const csa2_group_args*>(args), &iz, &iw, &aw) == CSA2_OK ? iw + aw : 0;
+    size_t iz = 0, iw = 0, need = 0;
+    return check_group(static_cast<const csa2_group_args*>(args), &iz, &iw, &need) == CSA2_OK ? need : 0;
+  }
+  if (which == CSA2_WS_STACK) {
+    size_t need = 0;
+    return validate_stack(static_cast<const csa2_stack_args*>(args), &need) == CSA2_OK ? need : 0;
   }
   return 0;
 }
@@ -659,7 +757,7 @@ const char* csa2_status_string(int32_t s) {
   }
 }
 
-int32_t csa2_version(void) { return 100; }
+int32_t csa2_version(void) { return 101; }
 
 csa2_status csa2_trace_begin(int32_t max_launches) {
   if (max_launches < 1 || max_launches > (1 << 20)) return CSA2_ERR_SHAPE;

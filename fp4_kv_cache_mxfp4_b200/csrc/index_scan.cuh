@@ -62,6 +62,8 @@ struct ScanParams {
   int ctas_per_group;
   int stages;
   uint32_t tmem_cols;
+  int early_q;            // 1: index-Q and w are complete at launch (load them before waiting on
+                          // the predecessor); 0: they may be the predecessor's results
 };
 
 struct ScanSmem {
@@ -125,12 +127,14 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) hist_s[i] = 0;
   if (HSI) for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) bhist_s[i] = 0;
 
-  // Index-K, index-Q, weights and n_vis are the caller's: complete before
-  // this kernel can start (its predecessor is the call's memset node or a
-  // kernel of this library that waited for everything before it), so the
-  // pipeline fills at once.  What waits for the predecessor: the HSI pool
-  // (a previous top-K wrote it) and every global store (the score buffer is
-  // shared with the previous layer's top-K).
+  // Index-K and n_vis are the caller's cache and step metadata: complete
+  // before this kernel can start (its predecessor is the call's memset node
+  // or a kernel of this library that waited for everything before it), so
+  // the first index-K tiles are requested at once.  What waits for the
+  // predecessor: index-Q and w unless early_q (in a model they come from
+  // the previous layer's output), the HSI pool (a previous top-K wrote it)
+  // and every global store (the score buffer is shared with the previous
+  // layer's top-K).
   pdl_launch_dependents();
 
   // this CTA's tile range; in scan mode, tiles past every query's n_vis are skipped
@@ -146,7 +150,6 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     tile_hi = min(tile_hi, (nmax + kTileRows - 1) / kTileRows);
   }
   const int ntiles = max(0, tile_hi - tile_lo);
-  for (int i = threadIdx.x; i < QG * 32; i += blockDim.x) w_s[i] = (i < qn * 32) ? p.w[bq0 * 32 + i] : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -162,12 +165,19 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const uint64_t pol_keep = l2_policy_evict_last();
       uint8_t* qi = smem + L.qi0;
       constexpr uint32_t qbox = n_mma * 128;
-      mbar_arrive_expect_tx(q_bar, 2 * qbox);
-      tma_load_2d(qi, &tmap_q, q_bar, 0, bq0 * 32, pol_keep);
-      tma_load_2d(qi + qbox, &tmap_q, q_bar, 64, bq0 * 32, pol_keep);
+      auto load_q = [&]() {
+        mbar_arrive_expect_tx(q_bar, 2 * qbox);
+        tma_load_2d(qi, &tmap_q, q_bar, 0, bq0 * 32, pol_keep);
+        tma_load_2d(qi + qbox, &tmap_q, q_bar, 64, bq0 * 32, pol_keep);
+      };
+      // index-Q before the tiles when it is complete; otherwise after the
+      // first ring of index-K tiles is in flight and the predecessor is done
+      const bool q_late = !p.early_q && !p.pool_mode;
+      if (!q_late) load_q();
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % p.stages;
         const uint32_t ph = (i / p.stages) & 1;
+        if (q_late && i == min(p.stages, ntiles)) { pdl_wait(); load_q(); }
         if (!mbar_wait(&empty_bar[s], ph ^ 1, kErrWaitSmemEmpty, abort_flag)) break;
         uint8_t* st = smem + L.stage0 + s * kStageBytes;
         mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
@@ -189,6 +199,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
         }
       }
+      if (q_late && ntiles <= p.stages) { pdl_wait(); load_q(); }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -219,7 +230,12 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    pdl_wait();                                   // before the first score store
+    pdl_wait();                                   // before w and the first score store
+    {
+      const int et = threadIdx.x - 64;
+      for (int i = et; i < QG * 32; i += kScanEpiThreads) w_s[i] = (i < qn * 32) ? p.w[bq0 * 32 + i] : 0.0f;
+      named_bar_sync(1, kScanEpiThreads);
+    }
     const int quarter = warp & 3;                 // TMEM lanes this warp may read
     const int set = (warp - 2) >> 2;              // tiles set, set+2, set+4, ...
     const int row = quarter * 32 + lane;          // entry within the tile

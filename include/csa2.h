@@ -165,7 +165,10 @@ csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws,
  *
  * - The first call on each device looks up the array's device address with
  *   cudaGetSymbolAddress (with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept per device and per CUDA
+ *   context: after the device's context is destroyed and re-created (for
+ *   example by cudaDeviceReset), the next call looks it up again, so that
+ *   call too must come before any stream capture.
  * - A request whose scratch would exceed CSA2_NOALLOC_SCRATCH_BYTES
  *   (csa2_workspace_size(a, CSA2_WS_INDEX) tells the need) returns
  *   CSA2_ERR_WORKSPACE before anything is enqueued.
@@ -178,6 +181,11 @@ csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws,
  * ---------------------------------------------------------------------- */
 #define CSA2_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 csa2_status csa2_index_score_topk_noalloc(const csa2_index_args* a, void* stream);
+
+/* Size in bytes of the fixed scratch array behind
+ * csa2_index_score_topk_noalloc, as compiled into the library (equals
+ * CSA2_NOALLOC_SCRATCH_BYTES of the header it was built with). */
+size_t csa2_noalloc_scratch_bytes(void);
 
 /* ------------------------------------------------------------------------
  * csa2_sparse_attn -- [eogee] §3.2 sparse MQA: each query attends to its
@@ -227,9 +235,28 @@ csa2_status csa2_sparse_attn(const csa2_attn_args* a, void* ws,
  *      dst_rows = new_rows, absolute rows of the [B*N] cache);
  *   2. for each layer: FULL / REINDEX / REINDEX_POOL score and select
  *      (csa2_index_score_topk; FULL builds the pool when hsi_blocks > 0 and
- *      REINDEX_POOL uses the pool of the most recent FULL layer), REUSE
- *      takes the top-K of the most recent indexing layer; then sparse
- *      attention with the layer's own q and window (csa2_sparse_attn).
+ *      REINDEX_POOL uses the pool of the most recent FULL layer, or pool_in
+ *      before any such layer), REUSE takes the top-K of the most recent
+ *      indexing layer; then sparse attention with the layer's own q and
+ *      window (csa2_sparse_attn).
+ *
+ * pool_in carries the HSI pool across calls: [eogee] §3.3 has the pool built
+ * once by the decoder's first Full layer serve every later Reindex layer,
+ * and those sit in later groups (decoder groups 2..5 are Reindex + 3 Reuse,
+ * [eogee] §3.2 configuration paragraph).
+ *
+ * flags (launch order between the call's kernels):
+ *   0                        each layer's inputs (qI, w, q, window rows) are
+ *                            treated as results of the layer before it, as
+ *                            in the model, where a layer's queries come from
+ *                            the previous layer's output: a kernel may start
+ *                            its set-up and stream shared caches (index-K)
+ *                            early, but reads a layer's inputs only after
+ *                            the previous kernel has finished;
+ *   CSA2_GROUP_INPUTS_READY  every layer's inputs are complete when the call
+ *                            is made, so a kernel may load them early;
+ *   CSA2_GROUP_SERIAL        kernels run in plain stream order (no kernel
+ *                            starts before its predecessor has finished).
  * ---------------------------------------------------------------------- */
 typedef struct csa2_layer {
     int32_t        mode;        /* csa2_mode                                     */
@@ -258,14 +285,43 @@ typedef struct csa2_group_args {
     float            scale;
     int32_t          n_layers;  /* 1..64                                         */
     const csa2_layer* layers;   /* HOST array of n_layers descriptors            */
+    const int32_t*   pool_in;   /* optional int32 [B][Q][hsi_blocks]: the pool of
+                                   an earlier call, read by REINDEX_POOL layers
+                                   that come before any FULL layer of this call */
+    int32_t          flags;     /* CSA2_GROUP_* bits                             */
 } csa2_group_args;
+
+#define CSA2_GROUP_INPUTS_READY 1
+#define CSA2_GROUP_SERIAL       2
 
 csa2_status csa2_group_decode(const csa2_group_args* g, void* ws,
                               size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * csa2_stack_decode -- several sharing groups run one after another on one
+ * stream, as the model stacks them ([eogee] §3.2 configuration paragraph:
+ * the decoder's 20 layers are 5 groups of 4, the first Full + 3 Reuse, the
+ * others Reindex + 3 Reuse; the encoder's 18 are 3 groups of Full + 5
+ * Reuse).  Equivalent to calling csa2_group_decode for groups[0..n_groups)
+ * in order with one workspace: each group's pool_in may point at an earlier
+ * group's pool (the decoder's first Full layer builds the pool that every
+ * later Reindex layer re-scores, [eogee] §3.3).  The workspace is the
+ * largest any single group needs (csa2_workspace_size(&stack_args,
+ * CSA2_WS_STACK)); flags of the groups apply to their own kernels.
+ * Errors: those of csa2_group_decode, checked for every group before
+ * anything is enqueued; ARG when n_groups is outside 1..64.
+ * ---------------------------------------------------------------------- */
+typedef struct csa2_stack_args {
+    int32_t                n_groups;
+    const csa2_group_args* groups;   /* HOST array of n_groups descriptors       */
+} csa2_stack_args;
+
+csa2_status csa2_stack_decode(const csa2_stack_args* s, void* ws,
+                              size_t ws_bytes, void* stream);
+
 /* Workspace bytes needed by a call.  which = 1: csa2_index_args,
- * 2: csa2_attn_args, 3: csa2_group_args.  Returns 0 when the arguments are
- * invalid for that call.
+ * 2: csa2_attn_args, 3: csa2_group_args, 4: csa2_stack_args.  Returns 0
+ * when the arguments are invalid for that call.
  *
  * Launches: every kernel is launched with programmatic stream serialisation
  * (it may start while the previous kernel in the stream finishes, and waits
@@ -275,6 +331,7 @@ csa2_status csa2_group_decode(const csa2_group_args* g, void* ws,
 #define CSA2_WS_INDEX 1
 #define CSA2_WS_ATTN  2
 #define CSA2_WS_GROUP 3
+#define CSA2_WS_STACK 4
 size_t csa2_workspace_size(const void* args, int32_t which);
 
 /* Reads and clears the device-side failure word of the current device

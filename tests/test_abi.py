@@ -42,7 +42,7 @@ def test_every_declared_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert csa2.version() == 100
+    assert csa2.version() == 101
     assert csa2.status_string(0) == "ok"
     assert "workspace" in csa2.status_string(4)
     assert csa2.status_string(99) == "unknown status"
@@ -54,6 +54,7 @@ def _c_layout():
         "csa2_attn_args": [f for f, _ in csa2.AttnArgs._fields_],
         "csa2_layer": [f for f, _ in csa2.Layer._fields_],
         "csa2_group_args": [f for f, _ in csa2.GroupArgs._fields_],
+        "csa2_stack_args": [f for f, _ in csa2.StackArgs._fields_],
     }
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "csa2.h"', "int main(void) {"]
     for s, fs in fields.items():
@@ -72,7 +73,8 @@ def _c_layout():
 def test_struct_layouts_match_the_header():
     c = _c_layout()
     for cname, py in [("csa2_index_args", csa2.IndexArgs), ("csa2_attn_args", csa2.AttnArgs),
-                      ("csa2_layer", csa2.Layer), ("csa2_group_args", csa2.GroupArgs)]:
+                      ("csa2_layer", csa2.Layer), ("csa2_group_args", csa2.GroupArgs),
+                      ("csa2_stack_args", csa2.StackArgs)]:
         assert int(c[cname]) == ctypes.sizeof(py), cname
         for f, _ in py._fields_:
             assert int(c[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
@@ -171,6 +173,59 @@ def test_group_validation(L):
     n = L.csa2_workspace_size(ctypes.byref(g), csa2.WS_GROUP)
     assert n > 0
     assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), n - 1, None) == 4
+    g.flags = 4                                                           # unknown flag bit
+    assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), n, None) == 1
+    g.flags = csa2.GROUP_INPUTS_READY | csa2.GROUP_SERIAL
+    assert L.csa2_workspace_size(ctypes.byref(g), csa2.WS_GROUP) == n
+
+
+def _group(layers, **kw):
+    g = csa2.GroupArgs(B=1, Q=1, K=512, W=128, N=4096, n_vis=FAKE, kI=FAKE, kv_fp4=FAKE, kv_new=None, n_new=0,
+                       new_rows=None, swa_rows=128, swa_step=0, hsi_blocks=2048, hsi_block=8, pool=FAKE, scale=0.0,
+                       n_layers=len(layers), layers=ctypes.cast(layers, ctypes.POINTER(csa2.Layer)), pool_in=None,
+                       flags=0)
+    for k, v in kw.items():
+        setattr(g, k, v)
+    return g
+
+
+def test_group_pool_in_validation(L):
+    """A group that starts with a pool-restricted Reindex layer needs the
+    pool of an earlier call (pool_in); with it, it is valid."""
+    layers = (csa2.Layer * 2)()
+    layers[0] = csa2.Layer(mode=2, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)
+    layers[1] = csa2.Layer(mode=3, q=FAKE, swa=FAKE, out=FAKE)
+    g = _group(layers)
+    assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), 0, None) == 1
+    assert L.csa2_workspace_size(ctypes.byref(g), csa2.WS_GROUP) == 0
+    g.pool_in = FAKE + 4
+    assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), 0, None) == 3
+    g.pool_in = FAKE
+    n = L.csa2_workspace_size(ctypes.byref(g), csa2.WS_GROUP)
+    assert n > 0
+    assert L.csa2_group_decode(ctypes.byref(g), ctypes.c_void_p(FAKE), n - 1, None) == 4
+
+
+def test_stack_validation_and_workspace(L):
+    """The stack call's workspace is the largest single group's; every
+    group is validated before anything is enqueued."""
+    first = (csa2.Layer * 2)()
+    first[0] = csa2.Layer(mode=0, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)
+    first[1] = csa2.Layer(mode=3, q=FAKE, swa=FAKE, out=FAKE)
+    later = (csa2.Layer * 2)()
+    later[0] = csa2.Layer(mode=2, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)
+    later[1] = csa2.Layer(mode=3, q=FAKE, swa=FAKE, out=FAKE)
+    g1, g2 = _group(first), _group(later, pool_in=FAKE)
+    n1 = L.csa2_workspace_size(ctypes.byref(g1), csa2.WS_GROUP)
+    n2 = L.csa2_workspace_size(ctypes.byref(g2), csa2.WS_GROUP)
+    st = csa2.stack_args([g1, g2])
+    assert L.csa2_workspace_size(ctypes.byref(st), csa2.WS_STACK) == max(n1, n2)
+    assert L.csa2_stack_decode(ctypes.byref(st), ctypes.c_void_p(FAKE), max(n1, n2) - 1, None) == 4
+    bad = csa2.stack_args([g1, _group(later)])                            # second group lacks its pool
+    assert L.csa2_stack_decode(ctypes.byref(bad), ctypes.c_void_p(FAKE), 1 << 40, None) == 1
+    assert L.csa2_workspace_size(ctypes.byref(bad), csa2.WS_STACK) == 0
+    empty = csa2.StackArgs(n_groups=0, groups=None)
+    assert L.csa2_stack_decode(ctypes.byref(empty), ctypes.c_void_p(FAKE), 0, None) == 1
 
 
 def test_arg_structs_keep_their_tensors_alive():
