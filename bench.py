@@ -164,21 +164,117 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def scan_algorithmic_bytes(wl):
-    """Bytes one index_scan_kernel launch must move (Full / Reindex scan):
-    index-K rows once, one fp32 score per (query, entry), index-Q and w."""
+    """Bytes one Full / Reindex index_scan_kernel launch must move: index-K
+    rows once per batch row, one fp32 score per (query, entry), index-Q and
+    w of every query."""
     per_row = wl.N * 128 * 2 + wl.Q * wl.N * 4 + wl.Q * (32 * 128 * 2 + 32 * 4)
     return wl.B * per_row
+
+
+def pool_scan_algorithmic_bytes(wl):
+    """Bytes of one pool-restricted (HSI) index_scan_kernel launch: per query
+    the pool's block ids, 8 index-K rows per block, one fp32 score per pool
+    position, index-Q and w."""
+    P = wl.hsi_blocks * wl.hsi_block
+    return wl.B * wl.Q * (wl.hsi_blocks * 4 + P * 128 * 2 + P * 4 + 32 * 128 * 2 + 32 * 4)
+
+
+def scan_algorithmic_flops(wl):
+    """Flops of one index_scan_kernel launch: 32 heads x 128 dims x 2 per
+    (query, visible entry)."""
+    return wl.B * sum(wl.n_vis) * 32 * 128 * 2
+
+
+def topk_algorithmic_bytes(wl, blocks=False):
+    """Bytes of one topk_select_kernel launch: every score slot read once and
+    the selection written (positions: K indices; HSI blocks: the pool)."""
+    if blocks:
+        nblk = (wl.N + wl.hsi_block - 1) // wl.hsi_block
+        return wl.B * wl.Q * (nblk * 4 + wl.hsi_blocks * 4)
+    return wl.B * wl.Q * (wl.N * 4 + wl.K * 4)
+
+
+def attention_algorithmic_bytes(wl):
+    """Bytes of one attention launch: per query the K indices, K selected FP4
+    entries (288 B), W window rows (1 KB bf16), the 64 x 512 bf16 query and
+    the 64 x 512 bf16 output."""
+    return wl.B * wl.Q * (wl.K * 4 + wl.K * 288 + wl.W * 1024 + 2 * 64 * 512 * 2)
+
+
+def quantize_algorithmic_bytes(wl):
+    """New entries read as bf16 and written as 288-byte FP4 rows."""
+    return wl.B * wl.n_new * (1024 + 288)
+
+
+def label_launches(wl, names):
+    """Labels of one step's traced launches, in order, from the kernel names
+    and the layer schedule: quantise; per indexing layer its scan (Full /
+    Reindex scan, pool re-score or causal prefill scan) and selections
+    (positions, then the HSI blocks of a Full layer with a pool); per layer
+    its attention (and the merge of split slices, when launched)."""
+    labels = []
+    layer = -1
+    topk_seen = 0
+    for n in names:
+        if n == "quantize_kv_fp4_kernel":
+            labels.append("quantize")
+        elif n == "index_scan_kernel":
+            layer += 1
+            while wl.modes[layer] == workloads.REUSE:
+                layer += 1
+            mode = wl.modes[layer]
+            labels.append("scan_pool" if mode == workloads.REINDEX_POOL else
+                          "scan_prefill" if wl.prefill else "scan")
+            topk_seen = 0
+        elif n == "topk_select_kernel":
+            pool = wl.modes[max(layer, 0)] == workloads.REINDEX_POOL
+            labels.append("topk_blocks" if topk_seen == 1 else "topk_pool" if pool else "topk")
+            topk_seen += 1
+        elif n == "sparse_attn_tc_kernel":
+            if layer < 0 or labels and labels[-1] in ("attention", "attention_merge"):
+                layer += 1
+            labels.append("attention")
+        elif n == "sparse_attn_combine_kernel":
+            labels.append("attention_merge")
+        else:
+            labels.append(n)
+    return labels
+
+
+def label_work(wl, label):
+    """(bound, algorithmic amount per launch, unit) of a launch label."""
+    if label == "scan":
+        return "hbm", scan_algorithmic_bytes(wl), "B"
+    if label == "scan_pool":
+        return "hbm", pool_scan_algorithmic_bytes(wl), "B"
+    if label == "scan_prefill":
+        return "tensor", scan_algorithmic_flops(wl), "flop"
+    if label == "topk":
+        return "hbm", topk_algorithmic_bytes(wl), "B"
+    if label == "topk_blocks":
+        return "hbm", topk_algorithmic_bytes(wl, blocks=True), "B"
+    if label == "topk_pool":
+        P = wl.hsi_blocks * wl.hsi_block
+        return "hbm", wl.B * wl.Q * (P * 4 + wl.hsi_blocks * 4 + wl.K * 4), "B"
+    if label == "attention":
+        return "hbm", attention_algorithmic_bytes(wl), "B"
+    if label == "quantize":
+        return "hbm", quantize_algorithmic_bytes(wl), "B"
+    return "hbm", None, "B"
 
 
 def step_algorithmic_bytes(wl):
     """Algorithmic HBM bytes of one whole step (same accounting as the
     per-kernel figures): the scans, the new entries (read bf16, write FP4),
     and per layer the gathered FP4 entries, the window, q and the output."""
-    n_index = sum(1 for m in wl.modes if m in (workloads.FULL, workloads.REINDEX))
-    total = n_index * scan_algorithmic_bytes(wl)
-    total += wl.B * wl.n_new * (1024 + 288)
-    per_query_attn = wl.K * 288 + wl.W * 1024 + 64 * 512 * 2 * 2
-    total += len(wl.modes) * wl.B * wl.Q * per_query_attn
+    total = 0
+    for m in wl.modes:
+        if m in (workloads.FULL, workloads.REINDEX):
+            total += scan_algorithmic_bytes(wl)
+        elif m == workloads.REINDEX_POOL:
+            total += pool_scan_algorithmic_bytes(wl)
+    total += quantize_algorithmic_bytes(wl)
+    total += len(wl.modes) * attention_algorithmic_bytes(wl)
     return total
 
 
@@ -206,10 +302,14 @@ def tensor_peak():
         return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
 
 
-def scan_algorithmic_flops(wl):
-    """Flops of one index_scan_kernel launch: 32 heads x 128 dims x 2 per
-    (query, visible entry)."""
-    return wl.B * sum(wl.n_vis) * 32 * 128 * 2
+def bench_config(wl, world):
+    """The workload description both arms print."""
+    return {"workload": wl.name, "B": wl.B, "Q": wl.Q, "N_entries": wl.N, "r": wl.r,
+            "layers": ",".join(workloads.MODE_NAMES[m] for m in wl.modes), "K": wl.K, "W": wl.W,
+            "hsi_pool": f"{wl.hsi_blocks}x{wl.hsi_block}" if wl.hsi_blocks else None,
+            "kv_cache": "FP4 E2M1 + E4M3/16ch (288 B/entry)", "index_k": "bf16", "window": "bf16",
+            "l2": "flushed between steps (256 MB memset outside the timed events)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 # ---------------------------------------------------------------------------
@@ -315,9 +415,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "N_entries": wl.N,
-                       "layers": ",".join(workloads.MODE_NAMES[m] for m in wl.modes), "K": wl.K, "W": wl.W,
-                       "parallelism": "oracle on host cores"},
+            "config": bench_config(wl, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": f"every batch row of {wl.name} per step, {oracle_sample_text(wl)}, "
                                        f"through the oracle group schedule (numpy, float64); warm-up steps "
@@ -330,6 +428,42 @@ def run_reference(args, world, rank):
 # our arm
 # ---------------------------------------------------------------------------
 
+def time_steps(step, steps, flush, st, world, before=None, after=None):
+    """Mean ms of `steps` calls of step() bracketed by CUDA events on the
+    launching stream (L2 flushed before each, outside the events), after a
+    barrier and a synchronize; the slowest rank's mean.  before/after run
+    inside the events (host<->device copies)."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush.zero_()
+        a.record(st)
+        if before:
+            before()
+        step()
+        if after:
+            after()
+        b.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / steps, world)
+
+
+def capture(fn):
+    """One CUDA graph of fn() (warmed on a side stream first)."""
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(graph):
+        fn()
+    torch.cuda.synchronize()
+    return graph
+
+
 def run_ours(args, world, rank, local):
     if rank == 0:
         _build.build()
@@ -340,74 +474,54 @@ def run_ours(args, world, rank, local):
     T = make_device_workload(wl, csa2, seed_shift=rank)
     st = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    g = T["g"]
 
-    def eager_step():
-        csa2.csa2_group_decode(T["g"], T["ws"])
+    def call(flags):
+        def f():
+            g.flags = flags
+            csa2.csa2_group_decode(g, T["ws"])
+        return f
 
     clocks = ClockSampler(local)
     clocks.start()
     for _ in range(args.warmup):
         flush.zero_()
-        eager_step()
+        call(0)()
     torch.cuda.synchronize()
     st_code = csa2.csa2_device_status()
     if st_code != (0, 0):
         raise RuntimeError(f"device status after warm-up: {st_code}")
     # the step's launches (memset, quantise, scans, selections, attention)
-    # replayed as one CUDA graph
-    graph = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        eager_step()
-    torch.cuda.current_stream().wait_stream(side)
-    with torch.cuda.graph(graph):
-        eager_step()
-    torch.cuda.synchronize()
-    step = graph.replay
+    # replayed as one CUDA graph, in each launch order
+    graphs = {name: capture(call(flags)) for name, flags in
+              (("model", 0), ("inputs_ready", csa2.GROUP_INPUTS_READY), ("serial", csa2.GROUP_SERIAL))}
     for _ in range(args.warmup):
-        flush.zero_()
-        step()
+        for gr in graphs.values():
+            flush.zero_()
+            gr.replay()
     torch.cuda.synchronize()
 
-    # ---- timed: device-resident inputs
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for a, b in ev:
-        flush.zero_()
-        a.record(st)
-        step()
-        b.record(st)
-    torch.cuda.synchronize()
-    barrier(world)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    mean_ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+    # ---- timed: device-resident inputs, model launch order (headline)
+    mean_ms = time_steps(graphs["model"].replay, args.steps, flush, st, world)
+    ready_ms = time_steps(graphs["inputs_ready"].replay, args.steps, flush, st, world)
+    serial_ms = time_steps(graphs["serial"].replay, args.steps, flush, st, world)
 
     # ---- traced pass: per-kernel durations with events on the launch stream
-    launches_per_step = None
     csa2.csa2_trace_begin(64 * args.steps)
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for a, b in ev2:
-        flush.zero_()
-        a.record(st)
-        eager_step()
-        b.record(st)
-    torch.cuda.synchronize()
-    barrier(world)
+    traced_ms = time_steps(call(0), args.steps, flush, st, world)
     csa2.csa2_trace_stop()
     recs = csa2.csa2_trace_records()
     csa2.csa2_trace_end()
-    traced_ms = sum(a.elapsed_time(b) for a, b in ev2) / args.steps
-    launches_per_step = len(recs) / args.steps
-    per_kernel = {}
-    for name, ms in recs:
-        c, t = per_kernel.get(name, (0, 0.0))
-        per_kernel[name] = (c + 1, t + ms)
+    per_step = len(recs) // args.steps
+    labels = label_launches(wl, [n for n, _ in recs[:per_step]])
+    per_label = {}
+    for i, (name, ms) in enumerate(recs):
+        lab = labels[i % per_step]
+        c, t, _ = per_label.get(lab, (0, 0.0, name))
+        per_label[lab] = (c + 1, t + ms, name)
 
-    # ---- end to end: host inputs -> device -> csa2_group_decode -> host outputs
+    # ---- end to end through the C ABI: host inputs -> device ->
+    #      csa2_group_decode -> host outputs, every step
     host_in = [(T["new"], torch.empty_like(T["new"], device="cpu").pin_memory())]
     for L in T["layers"]:
         for k in ("qI", "w", "q"):
@@ -417,72 +531,87 @@ def run_ours(args, world, rank, local):
     host_out = [(L["out"], torch.empty_like(L["out"], device="cpu").pin_memory()) for L in T["layers"]]
     h2d = sum(h.numel() * h.element_size() for _, h in host_in)
     d2h = sum(h.numel() * h.element_size() for _, h in host_out)
-    ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for a, b in ev3:
-        flush.zero_()
-        a.record(st)
+
+    def h2d_copies():
         for dev_t, host_t in host_in:
             dev_t.copy_(host_t, non_blocking=True)
-        step()
+
+    def d2h_copies():
         for dev_t, host_t in host_out:
             host_t.copy_(dev_t, non_blocking=True)
-        b.record(st)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev3) / args.steps, world)
+
+    e2e_ms = time_steps(call(0), args.steps, flush, st, world, h2d_copies, d2h_copies)
+    e2e_graph_ms = time_steps(graphs["model"].replay, args.steps, flush, st, world, h2d_copies, d2h_copies)
     clk = clocks.stop()
     st_code = csa2.csa2_device_status()
     if st_code != (0, 0):
         raise RuntimeError(f"device status after the timed loops: {st_code}")
+    del graphs
 
     if rank != 0:
         return
     queries = wl.B * wl.Q * world
     value = aggregate_queries_per_s(wl.B * wl.Q, world, mean_ms)
-    peak, peak_kind = hbm_peak()
-    n_scan, t_scan = per_kernel.get("index_scan_kernel", (0, 0.0))
-    scan_ms = t_scan / max(n_scan, 1)
-    scan_bytes = scan_algorithmic_bytes(wl)
-    achieved = scan_bytes / (scan_ms * 1e-3) / 1e9 if n_scan else None
-    if wl.prefill:
-        # eight queries per MMA group make the prefill scan a contraction
-        scan_flops = scan_algorithmic_flops(wl)
-        t_peak, t_kind = tensor_peak()
-        t_achieved = scan_flops / (scan_ms * 1e-3) / 1e12 if n_scan else None
-        roofline = {"kernel": "index_scan_kernel", "bound": "tensor", "achieved": t_achieved, "peak": t_peak,
-                    "peak_source": f"{t_kind} (MEASURED_PEAKS.json bf16_tflops_sustained)" if t_kind == "measured"
-                    else "fallback 1.4 PFLOP/s sustained", "unit": "TFLOP/s",
-                    "frac": (t_achieved / t_peak) if t_achieved else None, "traffic": None,
-                    "algorithmic_flops_per_launch": scan_flops, "ms_per_launch": scan_ms, "launches": n_scan}
+    hbm, hbm_kind = hbm_peak()
+    tflops, t_kind = tensor_peak()
+    kernels = {}
+    for lab, (c, t, name) in sorted(per_label.items()):
+        bound, amount, unit = label_work(wl, lab)
+        ms = t / c
+        k = {"kernel": name, "launches_per_step": c // args.steps, "ms_mean": ms}
+        if amount is not None:
+            if bound == "tensor":
+                k.update(bound="tensor", algorithmic_flops=amount, achieved_tflops=amount / (ms * 1e-3) / 1e12,
+                         frac=amount / (ms * 1e-3) / 1e12 / tflops)
+            else:
+                k.update(bound="hbm", algorithmic_bytes=amount, achieved_gbs=amount / (ms * 1e-3) / 1e9,
+                         frac=amount / (ms * 1e-3) / 1e9 / hbm)
+        kernels[lab] = k
+    # the dominant kernel: the label with the most time per step
+    dom = max((lab for lab in kernels if "frac" in kernels[lab]),
+              key=lambda lab: kernels[lab]["ms_mean"] * kernels[lab]["launches_per_step"])
+    D = kernels[dom]
     sha = kernel_source_sha()
-    traffic = SCAN_TRAFFIC["bytes_per_launch"] if (SCAN_TRAFFIC["sha"] == sha and args.workload == 2) else None
+    if D["bound"] == "tensor":
+        roofline = {"kernel": f"{D['kernel']} ({dom})", "bound": "tensor", "achieved": D["achieved_tflops"],
+                    "peak": tflops, "unit": "TFLOP/s", "frac": D["frac"], "traffic": None,
+                    "peak_source": f"{t_kind} (MEASURED_PEAKS.json bf16_tflops_sustained)" if t_kind == "measured"
+                    else "fallback 1.4 PFLOP/s sustained",
+                    "algorithmic_flops_per_launch": D["algorithmic_flops"], "ms_per_launch": D["ms_mean"],
+                    "launches_per_step": D["launches_per_step"]}
+    else:
+        traffic = SCAN_TRAFFIC["bytes_per_launch"] if (SCAN_TRAFFIC["sha"] == sha and args.workload == 2
+                                                        and dom == "scan") else None
+        roofline = {"kernel": f"{D['kernel']} ({dom})", "bound": "hbm", "achieved": D["achieved_gbs"], "peak": hbm,
+                    "unit": "GB/s", "frac": D["frac"], "traffic": traffic,
+                    "peak_source": f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs)" if hbm_kind == "measured"
+                    else "fallback 6.65 TB/s",
+                    "algorithmic_bytes_per_launch": D["algorithmic_bytes"], "ms_per_launch": D["ms_mean"],
+                    "launches_per_step": D["launches_per_step"]}
     step_bytes = step_algorithmic_bytes(wl)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) caches and inputs)",
-        "config": {"workload": wl.name, "B": wl.B, "Q": wl.Q, "N_entries": wl.N, "r": wl.r,
-                   "layers": ",".join(workloads.MODE_NAMES[m] for m in wl.modes), "K": wl.K, "W": wl.W,
-                   "kv_cache": "FP4 E2M1 + E4M3/16ch (288 B/entry)", "index_k": "bf16",
-                   "l2": "flushed between steps (256 MB memset outside the timed events)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": bench_config(wl, world),
+        "launch": "CUDA graph of one csa2_group_decode call per step, model launch order (flags 0: a layer's "
+                  "inputs are read only after the previous kernel finished)",
+        "value_inputs_ready": aggregate_queries_per_s(wl.B * wl.Q, world, ready_ms),
+        "ms_per_step_inputs_ready": ready_ms,
+        "value_serial": aggregate_queries_per_s(wl.B * wl.Q, world, serial_ms),
+        "ms_per_step_serial": serial_ms,
         "hbm_gbs_step": step_bytes / (mean_ms * 1e-3) / 1e9,
-        "hbm_frac_step": step_bytes / (mean_ms * 1e-3) / 1e9 / peak,
-        "roofline": roofline if wl.prefill else
-                    {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback 6.65 TB/s", "unit": "GB/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": scan_bytes, "ms_per_launch": scan_ms,
-                     "launches": n_scan},
-        "kernels": {k: {"launches": c, "ms_mean": t / c} for k, (c, t) in sorted(per_kernel.items())},
+        "hbm_frac_step": step_bytes / (mean_ms * 1e-3) / 1e9 / hbm,
+        "roofline": roofline,
+        "kernels": kernels,
         "ms_per_step_eager_traced": traced_ms,
-        "launch": "CUDA graph of one csa2_group_decode call per step",
         "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": int(round(launches_per_step * args.steps)) if launches_per_step else 0,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "how": "eager csa2_group_decode call per step through the C ABI, H2D of the step's inputs from "
+                       "pinned host memory and D2H of every layer's output inside the events"},
+        "e2e_graph": {"value": queries / (e2e_graph_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_graph_ms,
+                      "how": "the same copies around a CUDA-graph replay of the call"},
+        "gpu_launches": per_step * args.steps,
         "clocks": clk,
     }
     if world == 1:
