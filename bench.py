@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 from fp4_kv_cache_mxfp4_b200 import build as _build  # noqa: E402
 from fp4_kv_cache_mxfp4_b200 import workloads  # noqa: E402
-from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload  # noqa: E402
+from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload, run_step, set_flags  # noqa: E402
 
 METRIC = "CSA2 decode queries/s and HBM GB/s vs peak at 128K ctx, FP4 main KV"
 UNIT = "queries/s"
@@ -273,7 +273,7 @@ def step_algorithmic_bytes(wl):
             total += scan_algorithmic_bytes(wl)
         elif m == workloads.REINDEX_POOL:
             total += pool_scan_algorithmic_bytes(wl)
-    total += quantize_algorithmic_bytes(wl)
+    total += quantize_algorithmic_bytes(wl) * (len(wl.groups) if wl.cache_per_group else 1)
     total += len(wl.modes) * attention_algorithmic_bytes(wl)
     return total
 
@@ -307,6 +307,7 @@ def bench_config(wl, world):
     return {"workload": wl.name, "B": wl.B, "Q": wl.Q, "N_entries": wl.N, "r": wl.r,
             "layers": ",".join(workloads.MODE_NAMES[m] for m in wl.modes), "K": wl.K, "W": wl.W,
             "hsi_pool": f"{wl.hsi_blocks}x{wl.hsi_block}" if wl.hsi_blocks else None,
+            "groups": len(wl.groups), "cache_per_group": wl.cache_per_group,
             "kv_cache": "FP4 E2M1 + E4M3/16ch (288 B/entry)", "index_k": "bf16", "window": "bf16",
             "l2": "flushed between steps (256 MB memset outside the timed events)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
@@ -474,12 +475,11 @@ def run_ours(args, world, rank, local):
     T = make_device_workload(wl, csa2, seed_shift=rank)
     st = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-    g = T["g"]
 
     def call(flags):
         def f():
-            g.flags = flags
-            csa2.csa2_group_decode(g, T["ws"])
+            set_flags(T, flags)
+            run_step(T, csa2)
         return f
 
     clocks = ClockSampler(local)
@@ -522,7 +522,7 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the C ABI: host inputs -> device ->
     #      csa2_group_decode -> host outputs, every step
-    host_in = [(T["new"], torch.empty_like(T["new"], device="cpu").pin_memory())]
+    host_in = [(C["new"], torch.empty_like(C["new"], device="cpu").pin_memory()) for C in T["caches"]]
     for L in T["layers"]:
         for k in ("qI", "w", "q"):
             host_in.append((L[k], torch.empty_like(L[k], device="cpu").pin_memory()))
@@ -594,8 +594,9 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) caches and inputs)",
         "config": bench_config(wl, world),
-        "launch": "CUDA graph of one csa2_group_decode call per step, model launch order (flags 0: a layer's "
-                  "inputs are read only after the previous kernel finished)",
+        "launch": ("CUDA graph of one csa2_group_decode call per step" if T["stack"] is None else
+                   f"CUDA graph of one csa2_stack_decode call ({len(wl.groups)} groups) per step") +
+                  ", model launch order (flags 0: a layer's inputs are read only after the previous kernel finished)",
         "value_inputs_ready": aggregate_queries_per_s(wl.B * wl.Q, world, ready_ms),
         "ms_per_step_inputs_ready": ready_ms,
         "value_serial": aggregate_queries_per_s(wl.B * wl.Q, world, serial_ms),
@@ -607,7 +608,7 @@ def run_ours(args, world, rank, local):
         "ms_per_step_eager_traced": traced_ms,
         "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "how": "eager csa2_group_decode call per step through the C ABI, H2D of the step's inputs from "
+                "how": "eager library call per step through the C ABI, H2D of the step's inputs from "
                        "pinned host memory and D2H of every layer's output inside the events"},
         "e2e_graph": {"value": queries / (e2e_graph_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_graph_ms,
                       "how": "the same copies around a CUDA-graph replay of the call"},

@@ -3,9 +3,15 @@
 The main-KV cache of every batch row (all entries but the step's new ones)
 is quantised into FP4 with csa2_quantize_kv_fp4 in 65,536-row chunks; the
 step's new entries, index-K and every layer's inputs are copied to the
-device; the returned dict holds the csa2_group_args of one step and a
+device; the returned dict holds the csa2_group_args of each sharing group
+(and, for a stack of groups, the csa2_stack_args) of one step, plus a
 workspace of the size the library asks for.  The bench and the full-size
 parity tests both build their step here, so both run the same launches.
+
+A stack of groups either shares one cache (the decoder: the first group's
+Full layer quantises the step's new entries and builds the HSI pool that
+the later groups' pool-restricted Reindex layers read) or gives every group
+its own cache (the encoder: each group quantises its own new entries).
 """
 
 import torch
@@ -17,22 +23,32 @@ def with_seed_shift(wl, shift):
     """The same workload drawn from another seed (one per replica)."""
     if not shift:
         return wl
-    return workloads.Workload(**{**wl.__dict__, "seed": wl.seed + 7919 * shift, "n_vis": list(wl.n_vis)})
+    return workloads.Workload(**{**wl.__dict__, "seed": wl.seed + 7919 * shift, "n_vis": list(wl.n_vis),
+                                 "groups": list(wl.groups)})
+
+
+def _stage_cache(cw, csa2, d):
+    """FP4 main KV of every row but the step's new entries, index-K, the
+    new entries and their absolute destination rows."""
+    B, N = cw.B, cw.N
+    kv = torch.empty(B, N, 288, dtype=torch.uint8, device=d)
+    for b in range(B):
+        for r0 in range(0, N - cw.n_new, workloads.KV_CHUNK):
+            n = min(workloads.KV_CHUNK, N - cw.n_new - r0)
+            x = workloads.main_kv_rows(cw, b, r0, n).to(d)
+            csa2.csa2_quantize_kv_fp4(x, kv[b], row_offset=r0)
+    kI = torch.stack([workloads.index_k(cw, b) for b in range(B)]).to(d)
+    new = torch.cat([workloads.main_kv_rows(cw, b, N - cw.n_new, cw.n_new) for b in range(B)]).to(d)
+    new_rows = torch.tensor([b * N + r for b in range(B) for r in cw.new_rows], dtype=torch.int64, device=d)
+    return dict(kv=kv, kI=kI, new=new, new_rows=new_rows)
 
 
 def make_device_workload(wl, csa2, seed_shift=0):
     d = "cuda"
     wl = with_seed_shift(wl, seed_shift)
-    B, Q, N, K = wl.B, wl.Q, wl.N, wl.K
-    kv = torch.empty(B, N, 288, dtype=torch.uint8, device=d)
-    for b in range(B):
-        for r0 in range(0, N - wl.n_new, workloads.KV_CHUNK):
-            n = min(workloads.KV_CHUNK, N - wl.n_new - r0)
-            x = workloads.main_kv_rows(wl, b, r0, n).to(d)
-            csa2.csa2_quantize_kv_fp4(x, kv[b], row_offset=r0)
-    kI = torch.stack([workloads.index_k(wl, b) for b in range(B)]).to(d)
-    new = torch.cat([workloads.main_kv_rows(wl, b, N - wl.n_new, wl.n_new) for b in range(B)]).to(d)
-    new_rows = torch.tensor([b * N + r for b in range(B) for r in wl.new_rows], dtype=torch.int64, device=d)
+    B, Q, K = wl.B, wl.Q, wl.K
+    n_groups = len(wl.groups)
+    caches = [_stage_cache(wl.cache_of_group(g), csa2, d) for g in range(n_groups if wl.cache_per_group else 1)]
     layers = []
     for l, mode in enumerate(wl.modes):
         li = workloads.layer_inputs(wl, l)
@@ -40,11 +56,47 @@ def make_device_workload(wl, csa2, seed_shift=0):
                            out=torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=d),
                            lse=torch.empty(B, Q, 64, device=d),
                            idx=torch.empty(B, Q, K, dtype=torch.int32, device=d) if mode != workloads.REUSE else None))
-    pool = torch.empty(B, Q, wl.hsi_blocks, dtype=torch.int32, device=d) if wl.hsi_blocks else None
     n_vis = workloads.n_vis_tensor(wl).to(d)
-    g = csa2.group_args(B, Q, K, wl.W, N, n_vis, kI, kv, layers, kv_new=new, new_rows=new_rows,
-                        swa_rows=wl.swa_rows, swa_step=wl.swa_step, hsi_blocks=wl.hsi_blocks,
-                        hsi_block=wl.hsi_block, pool=pool)
-    ws = csa2.workspace(g, csa2.WS_GROUP)
+    groups = []
+    pool = None                      # the most recent pool built by a Full layer (handed to later groups)
+    for g in range(n_groups):
+        C = caches[g if wl.cache_per_group else 0]
+        Ls = [layers[l] for l in wl.group_layers(g)]
+        builds_pool = wl.hsi_blocks > 0 and any(L["mode"] == workloads.FULL for L in Ls)
+        own_pool = torch.empty(B, Q, wl.hsi_blocks, dtype=torch.int32, device=d) if builds_pool else None
+        quantise = g == 0 or wl.cache_per_group
+        ga = csa2.group_args(B, Q, K, wl.W, wl.N, n_vis, C["kI"], C["kv"], Ls,
+                             kv_new=C["new"] if quantise else None, new_rows=C["new_rows"] if quantise else None,
+                             swa_rows=wl.swa_rows, swa_step=wl.swa_step, hsi_blocks=wl.hsi_blocks,
+                             hsi_block=wl.hsi_block, pool=own_pool, pool_in=pool)
+        groups.append(dict(g=ga, cache=C, layers=Ls, pool=own_pool, pool_in=pool))
+        if own_pool is not None:
+            pool = own_pool
+    if n_groups == 1:
+        stack = None
+        ws = csa2.workspace(groups[0]["g"], csa2.WS_GROUP)
+    else:
+        stack = csa2.stack_args([G["g"] for G in groups])
+        ws = csa2.workspace(stack, csa2.WS_STACK)
     torch.cuda.synchronize()
-    return dict(wl=wl, g=g, ws=ws, kv=kv, kI=kI, new=new, new_rows=new_rows, layers=layers, pool=pool, n_vis=n_vis)
+    C0 = caches[0]
+    return dict(wl=wl, g=groups[0]["g"], groups=groups, stack=stack, ws=ws, caches=caches, kv=C0["kv"], kI=C0["kI"],
+                new=C0["new"], new_rows=C0["new_rows"], layers=layers, pool=groups[0]["pool"], n_vis=n_vis)
+
+
+def set_flags(T, flags):
+    """Launch-order flags of every group call of a staged step."""
+    if T["stack"] is None:
+        T["g"].flags = flags
+    else:
+        for i in range(len(T["groups"])):
+            T["stack"]._group_array[i].flags = flags
+
+
+def run_step(T, csa2, stream=None):
+    """One step through the library's public call: csa2_group_decode for one
+    group, csa2_stack_decode for a stack."""
+    if T["stack"] is None:
+        csa2.csa2_group_decode(T["g"], T["ws"], stream)
+    else:
+        csa2.csa2_stack_decode(T["stack"], T["ws"], stream)

@@ -49,8 +49,14 @@ class Workload:
     swa_step: int = 0      # window of query i starts at row i*swa_step
     desc: str = ""
     n_vis: List[int] = field(default_factory=list)   # per query, filled in __post_init__
+    groups: List[int] = field(default_factory=list)  # layers per sharing group (default: one group)
+    cache_per_group: bool = False  # each group has its own main KV and index-K (encoder), else one
+                                   # cache for all groups (decoder)
 
     def __post_init__(self):
+        if not self.groups:
+            self.groups = [len(self.modes)]
+        assert sum(self.groups) == len(self.modes)
         if not self.n_vis:
             if self.prefill:
                 # query i sits at token p0 + i, with p0 = (N - n_new) * r; entry e
@@ -63,6 +69,20 @@ class Workload:
     @property
     def swa_rows(self):
         return self.W + (self.Q - 1) * self.swa_step
+
+    def group_layers(self, g):
+        """Indices (into modes) of the layers of group g."""
+        start = sum(self.groups[:g])
+        return list(range(start, start + self.groups[g]))
+
+    def cache_of_group(self, g):
+        """The workload whose seed draws group g's shared caches: the same
+        one for every group of a decoder stack, a derived seed per group of
+        an encoder stack."""
+        if not self.cache_per_group or g == 0:
+            return self
+        return Workload(**{**self.__dict__, "seed": self.seed + 97 * g, "n_vis": list(self.n_vis),
+                           "groups": list(self.groups)})
 
     @property
     def new_rows(self):
@@ -84,6 +104,17 @@ WORKLOADS = {
     4: Workload("prefill_t4096_prefix256k_r2", 4, B=1, Q=4096, N=131072 + 2048, r=2, modes=[FULL],
                 n_new=2048, prefill=True, swa_step=1,
                 desc="Prefill chunk of 4096 tokens after a 256K-token prefix at r=2, causal"),
+    6: Workload("decoder20_q5_ctx128k_b4", 6, B=4, Q=5, N=131072, r=1,
+                modes=[FULL, REUSE, REUSE, REUSE] + [REINDEX_POOL, REUSE, REUSE, REUSE] * 4, groups=[4] * 5,
+                hsi_blocks=2048, n_new=5, prefill=True, swa_step=1,
+                desc="The decoder's 20 CSA2 layers as 5 groups over one 128K-entry cache (group 1: Full + HSI "
+                     "pool + 3 Reuse; groups 2-5: pool Reindex + 3 Reuse), 5 query positions per row "
+                     "(a verified draft block), batch 4"),
+    7: Workload("encoder18_q5_ctx64k_r2_b4", 7, B=4, Q=5, N=32768, r=2,
+                modes=([FULL] + [REUSE] * 5) * 3, groups=[6] * 3, cache_per_group=True, n_new=2,
+                prefill=True, swa_step=1,
+                desc="The encoder's 18 CSA2 layers as 3 groups (Full + 5 Reuse), each group with its own "
+                     "cache of 32,768 entries (64K tokens at r=2), 5 query positions per row, batch 4"),
     5: Workload("prefill_t1024_prefix64k_r2", 5, B=1, Q=1024, N=32768 + 512, r=2, modes=[FULL],
                 n_new=512, prefill=True, swa_step=1,
                 desc="Prefill chunk of 1024 tokens after a 64K-token prefix at r=2, causal: the prefill "

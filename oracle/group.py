@@ -12,10 +12,17 @@ entries are quantised after RoPE, before they join the cache).
 Readings: Reuse takes the indices of the most recent indexing layer
 ([titansim] "核心机制与研究方法" describes Reuse as taking the previous
 layer's already-selected indices);
-REINDEX_POOL uses the pool built by the most recent Full layer.  The layers
-run strictly in order; each layer's inputs are given.
+REINDEX_POOL uses the pool built by the most recent Full layer, which may
+sit in an earlier group: [eogee] §3.3 has the decoder's first Full layer
+build the pool that every later Reindex layer re-scores, and the §3.2
+configuration paragraph puts those Reindex layers at the head of decoder
+groups 2..5 (each Reindex + 3 Reuse; group 1 is Full + 3 Reuse; the encoder
+is 3 groups of Full + 5 Reuse at r=2).  The layers run strictly in order;
+each layer's inputs are given.
 
-Parity: pinned through the mode identities in tests/test_oracle_group.py.
+Parity: pinned through the mode identities in tests/test_oracle_group.py,
+including "a pool handed to a later group = the pool built in the same
+group".
 """
 
 import numpy as np
@@ -27,7 +34,7 @@ FULL, REINDEX, REINDEX_POOL, REUSE = 0, 1, 2, 3
 
 def group_row(kv_fp4, kI, n_vis, layers, K=indexer.TOPK, W=attention.WIN,
               swa_step=0, hsi_blocks=0, hsi_block=indexer.HSI_BLOCK,
-              kv_new=None, new_rows=None, scale=None):
+              kv_new=None, new_rows=None, scale=None, pool_in=None):
     """Run a group for one batch row.
 
     kv_fp4   uint8 [N, 288] packed cache (modified in place by kv_new)
@@ -38,6 +45,8 @@ def group_row(kv_fp4, kI, n_vis, layers, K=indexer.TOPK, W=attention.WIN,
     swa_step query position i sees window rows [i*swa_step, i*swa_step+W)
     hsi_blocks  0 = no pool; else a FULL layer also builds the pool
     kv_new   [n_new, 512] new entries quantised into rows new_rows first
+    pool_in  [Q, hsi_blocks] pool built by an earlier group, used by
+             REINDEX_POOL layers until a FULL layer here builds its own
     Returns a list of per-layer dicts: idx [Q,K], o [Q,64,512], lse [Q,64],
     and pool [Q,hsi_blocks] for a FULL layer that built one.
     """
@@ -47,7 +56,7 @@ def group_row(kv_fp4, kI, n_vis, layers, K=indexer.TOPK, W=attention.WIN,
     Q = n_vis.shape[0]
     results = []
     last_idx = None
-    last_pool = None
+    last_pool = None if pool_in is None else np.asarray(pool_in)
     for L in layers:
         mode = L["mode"]
         res = {}
@@ -87,3 +96,25 @@ def group_row(kv_fp4, kI, n_vis, layers, K=indexer.TOPK, W=attention.WIN,
         res.update(idx=idx, o=o, lse=lse)
         results.append(res)
     return results
+
+
+def stack_row(groups, hsi_blocks=0, hsi_block=indexer.HSI_BLOCK, **kw):
+    """Several groups of one batch row, run in order ([eogee] §3.2
+    configuration paragraph).  ``groups`` is a list of dicts with the
+    group_row arguments kv_fp4, kI, n_vis, layers (and optionally kv_new,
+    new_rows): groups may share one cache (the decoder) or each hold their
+    own (the encoder).  The most recent pool built by any group's Full
+    layer is handed to the next groups (the decoder's first Full layer
+    builds the pool every later Reindex layer re-scores, [eogee] §3.3).
+    Returns the per-group lists of group_row."""
+    out = []
+    pool = None
+    for G in groups:
+        res = group_row(G["kv_fp4"], G["kI"], G["n_vis"], G["layers"], hsi_blocks=hsi_blocks,
+                        hsi_block=hsi_block, kv_new=G.get("kv_new"), new_rows=G.get("new_rows"),
+                        pool_in=pool, **kw)
+        for r in res:
+            if "pool" in r:
+                pool = r["pool"]
+        out.append(res)
+    return out

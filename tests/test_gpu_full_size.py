@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from fp4_kv_cache_mxfp4_b200 import csa2, workloads
-from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload
+from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload, run_step
 from oracle import attention, fp4, indexer
 from parity import check_attention, check_topk, f32
 
@@ -27,7 +27,8 @@ def _samples(wl):
     if wl.Q == 1:
         return [(b, 0) for b in range(wl.B)]
     rng = np.random.default_rng(wl.seed)
-    qs = sorted({0, 1, 7, 8, wl.Q // 2 - 1, wl.Q - 2, wl.Q - 1, *rng.integers(0, wl.Q, 3).tolist()})
+    qs = sorted({q for q in (0, 1, 7, 8, wl.Q // 2 - 1, wl.Q - 2, wl.Q - 1, *rng.integers(0, wl.Q, 3).tolist())
+                 if 0 <= q < wl.Q})
     return [(b, q) for b in range(wl.B) for q in qs]
 
 
@@ -41,58 +42,71 @@ def _attn_oracle(kv_host_b, sel, q, win):
     return attention.sparse_mqa(q, deq, local, win)
 
 
-@pytest.mark.parametrize("w", [1, 2, 3, 4], ids=lambda w: workloads.WORKLOADS[w].name)
+@pytest.mark.parametrize("w", [1, 2, 3, 4, 6, 7], ids=lambda w: workloads.WORKLOADS[w].name)
 def test_full_size_sampled(w):
+    """One step of a full-size workload (a stack of groups for 6 and 7)
+    through the library call the bench times."""
     wl = workloads.WORKLOADS[w]
     csa2.load()
     T = make_device_workload(wl, csa2)
-    csa2.csa2_group_decode(T["g"], T["ws"])
+    run_step(T, csa2)
     torch.cuda.synchronize()
     assert csa2.csa2_device_status() == (0, 0)
     B, N = wl.B, wl.N
     rng = np.random.default_rng(100 + w)
+    n_caches = len(T["caches"])
 
-    # FP4 bytes: every new entry, and 64 sampled older ones per row
-    for b in range(B):
-        new_host = T["kv"][b, N - wl.n_new:].cpu().numpy()
-        want = fp4.quantize_kv_fp4(f32(workloads.main_kv_rows(wl, b, N - wl.n_new, wl.n_new)))
-        np.testing.assert_array_equal(new_host, want, err_msg=f"new entries of row {b}")
-        for r in rng.integers(0, N - wl.n_new, 64).tolist():
-            got = T["kv"][b, r].cpu().numpy()
-            np.testing.assert_array_equal(got, fp4.quantize_kv_fp4(f32(workloads.main_kv_rows(wl, b, r, 1)))[0],
-                                          err_msg=f"entry {r} of row {b}")
+    # FP4 bytes of every cache: every new entry, and 64 sampled older ones per row
+    for c in range(n_caches):
+        cw = wl.cache_of_group(c)
+        kv = T["caches"][c]["kv"]
+        for b in range(B):
+            new_host = kv[b, N - wl.n_new:].cpu().numpy()
+            want = fp4.quantize_kv_fp4(f32(workloads.main_kv_rows(cw, b, N - wl.n_new, wl.n_new)))
+            np.testing.assert_array_equal(new_host, want, err_msg=f"new entries of cache {c} row {b}")
+            for r in rng.integers(0, N - wl.n_new, 64).tolist():
+                got = kv[b, r].cpu().numpy()
+                np.testing.assert_array_equal(got, fp4.quantize_kv_fp4(f32(workloads.main_kv_rows(cw, b, r, 1)))[0],
+                                              err_msg=f"entry {r} of cache {c} row {b}")
 
     samples = _samples(wl)
-    kv_host = {b: T["kv"][b].cpu().numpy() for b in range(B)}
+    kv_host = {(c, b): T["caches"][c]["kv"][b].cpu().numpy() for c in range(n_caches) for b in range(B)}
     n_vis = np.asarray(wl.n_vis)
-    pool = T["pool"].cpu().numpy() if T["pool"] is not None else None
+    pool = None
     last_idx = None
-    for l, mode in enumerate(wl.modes):
-        li = workloads.layer_inputs(wl, l)
-        L = T["layers"][l]
-        if mode != workloads.REUSE:
-            last_idx = L["idx"].cpu().numpy()
-        for b in range(B):
-            kI = f32(workloads.index_k(wl, b)) if mode != workloads.REUSE else None
-            for (bb, q) in samples:
-                if bb != b:
-                    continue
-                what = f"{wl.name} layer {l} b{b} q{q}"
-                nv = int(n_vis[q])
-                if mode in (workloads.FULL, workloads.REINDEX):
-                    s = indexer.index_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, nv)
-                    check_topk(last_idx[b, q], s, wl.K, what=what)
-                    if mode == workloads.FULL and wl.hsi_blocks:
-                        bs = indexer.block_scores(s, 8)
-                        gp = pool[b, q]
-                        v = gp[gp >= 0]
-                        assert np.all(np.diff(v) > 0), f"{what}: pool not ascending"
-                        check_topk(np.concatenate([v[np.argsort(-bs[v], kind="stable")], gp[gp < 0]]), bs,
-                                   wl.hsi_blocks, what=what + " pool")
-                elif mode == workloads.REINDEX_POOL:
-                    pos, ps = indexer.pool_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, pool[b, q], nv)
-                    check_topk(last_idx[b, q], ps, wl.K, positions=pos, what=what)
-                win = f32(li["swa"][b])[q * wl.swa_step: q * wl.swa_step + wl.W]
-                o, lse = _attn_oracle(kv_host[b], last_idx[b, q], f32(li["q"][b, q]), win)
-                check_attention(L["out"][b, q], o, what=what)
-                np.testing.assert_allclose(L["lse"][b, q].cpu().numpy(), lse, rtol=1e-3, atol=1e-3)
+    for g in range(len(wl.groups)):
+        c = g if wl.cache_per_group else 0
+        cw = wl.cache_of_group(c)
+        G = T["groups"][g]
+        if G["pool"] is not None:
+            pool = G["pool"].cpu().numpy()
+        for l in wl.group_layers(g):
+            mode = wl.modes[l]
+            li = workloads.layer_inputs(wl, l)
+            L = T["layers"][l]
+            if mode != workloads.REUSE:
+                last_idx = L["idx"].cpu().numpy()
+            for b in range(B):
+                kI = f32(workloads.index_k(cw, b)) if mode != workloads.REUSE else None
+                for (bb, q) in samples:
+                    if bb != b:
+                        continue
+                    what = f"{wl.name} group {g} layer {l} b{b} q{q}"
+                    nv = int(n_vis[q])
+                    if mode in (workloads.FULL, workloads.REINDEX):
+                        s = indexer.index_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, nv)
+                        check_topk(last_idx[b, q], s, wl.K, what=what)
+                        if mode == workloads.FULL and wl.hsi_blocks:
+                            bs = indexer.block_scores(s, 8)
+                            gp = pool[b, q]
+                            v = gp[gp >= 0]
+                            assert np.all(np.diff(v) > 0), f"{what}: pool not ascending"
+                            check_topk(np.concatenate([v[np.argsort(-bs[v], kind="stable")], gp[gp < 0]]), bs,
+                                       wl.hsi_blocks, what=what + " pool")
+                    elif mode == workloads.REINDEX_POOL:
+                        pos, ps = indexer.pool_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, pool[b, q], nv)
+                        check_topk(last_idx[b, q], ps, wl.K, positions=pos, what=what)
+                    win = f32(li["swa"][b])[q * wl.swa_step: q * wl.swa_step + wl.W]
+                    o, lse = _attn_oracle(kv_host[(c, b)], last_idx[b, q], f32(li["q"][b, q]), win)
+                    check_attention(L["out"][b, q], o, what=what)
+                    np.testing.assert_allclose(L["lse"][b, q].cpu().numpy(), lse, rtol=1e-3, atol=1e-3)

@@ -112,3 +112,61 @@ def test_prefill_visibility_follows_token_coverage():
             assert wl.n_vis[i] == visible, (r, i)
         assert wl.n_vis[-1] == N                      # the last query sees every entry
         assert wl.swa_rows == wl.W + Q - 1
+
+
+def test_pool_handed_to_a_later_group_equals_the_pool_built_in_the_group():
+    """Decoder schedule: the pool of group 1's Full layer serves the Reindex
+    layer heading group 2.  Running [Full, pool-Reindex, Reuse] as one group
+    or as [Full] then [pool-Reindex, Reuse] with the pool handed over gives
+    the same indices and outputs."""
+    kv, kI, n_vis, layer = _setup(5)
+    L0, L1, L2 = layer(group.FULL), layer(group.REINDEX_POOL), layer(group.REUSE)
+    one = group.group_row(kv.copy(), kI, n_vis, [L0, L1, L2], K=40, hsi_blocks=24, hsi_block=8)
+    first = group.group_row(kv.copy(), kI, n_vis, [L0], K=40, hsi_blocks=24, hsi_block=8)
+    second = group.group_row(kv.copy(), kI, n_vis, [L1, L2], K=40, hsi_blocks=24, hsi_block=8,
+                             pool_in=first[0]["pool"])
+    np.testing.assert_array_equal(one[0]["pool"], first[0]["pool"])
+    for a, b in ((one[1], second[0]), (one[2], second[1])):
+        np.testing.assert_array_equal(a["idx"], b["idx"])
+        np.testing.assert_array_equal(a["o"], b["o"])
+    # the pool restricts the search: 24 blocks of 8 cannot hold every top-40
+    # position of a fresh index-Q over 640 entries
+    assert np.all(second[0]["idx"] >= 0)
+    for i in range(2):
+        blocks = set((second[0]["idx"][i] // 8).tolist())
+        assert blocks <= set(first[0]["pool"][i].tolist())
+
+
+def test_pool_reindex_without_any_pool_is_refused():
+    kv, kI, n_vis, layer = _setup(6)
+    try:
+        group.group_row(kv, kI, n_vis, [layer(group.REINDEX_POOL)], K=8, hsi_blocks=4)
+    except AssertionError:
+        return
+    raise AssertionError("a pool-restricted Reindex ran without a pool")
+
+
+def test_stack_row_hands_the_decoder_pool_forward_and_keeps_encoder_caches_apart():
+    """stack_row: decoder groups share one cache and the Full layer's pool
+    reaches the later groups' Reindex layers; encoder groups each read their
+    own cache (a group's attention sees only its own entries)."""
+    kv, kI, n_vis, layer = _setup(7)
+    g1 = dict(kv_fp4=kv, kI=kI, n_vis=n_vis, layers=[layer(group.FULL), layer(group.REUSE)])
+    g2 = dict(kv_fp4=kv, kI=kI, n_vis=n_vis, layers=[layer(group.REINDEX_POOL), layer(group.REUSE)])
+    g3 = dict(kv_fp4=kv, kI=kI, n_vis=n_vis, layers=[layer(group.REINDEX_POOL), layer(group.REUSE)])
+    res = group.stack_row([g1, g2, g3], hsi_blocks=16, hsi_block=8, K=32)
+    pool = res[0][0]["pool"]
+    for gi in (1, 2):
+        for i in range(2):
+            assert set((res[gi][0]["idx"][i] // 8).tolist()) <= set(pool[i].tolist())
+        np.testing.assert_array_equal(res[gi][1]["idx"], res[gi][0]["idx"])
+    # encoder: two groups with their own caches; a zero cache gives outputs
+    # that only the window explains
+    kv_zero = fp4.quantize_kv_fp4(np.zeros((640, 512), np.float32))
+    e1 = dict(kv_fp4=kv, kI=kI, n_vis=n_vis, layers=[layer(group.FULL), layer(group.REUSE)])
+    L = layer(group.FULL)
+    L["swa"] = np.zeros((128, 512))
+    e2 = dict(kv_fp4=kv_zero, kI=kI, n_vis=n_vis, layers=[L])
+    enc = group.stack_row([e1, e2], K=32)
+    assert np.all(enc[1][0]["o"] == 0) and not np.all(enc[0][0]["o"] == 0)
+
