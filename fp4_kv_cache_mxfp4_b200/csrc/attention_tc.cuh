@@ -6,10 +6,11 @@
 // FP4 entries, then ceil(W/128) slices of window rows.  A CTA (512 threads)
 // takes one slice (split mode: many CTAs per query, for few queries) or all
 // slices of its query in turn (one CTA per query, for many queries).  Per
-// slice the keys (FP4 entries, each 288-byte row fetched by one bulk copy
-// and dequantised by the CTA's threads, or window rows brought by TMA) form
-// a 128 x 512 bf16 tile K in shared memory, stored K-major with the 128-byte
-// swizzle; the query's 64 heads form Q (64 x 512, TMA, loaded once).  Then:
+// slice the keys (FP4 entries, loaded straight into registers by the CTA's
+// threads, 16 nibble bytes and two scales per thread and item, and
+// dequantised there, or window rows brought by TMA) form a 128 x 512 bf16
+// tile K in shared memory, stored K-major with the 128-byte swizzle; the
+// query's 64 heads form Q (64 x 512, TMA, loaded once).  Then:
 //   MMA 1   S^T[key, head] = K . Q^T            M = 128 keys, N = 64, K = 512
 //   softmax per head over the slice's keys in registers (fp32; shuffles and
 //           a 2 KB exchange between key quarters) against a running
@@ -19,10 +20,20 @@
 //           [key][head] as an MN-major operand
 //   MMA 2   O^T[dim, head] += V^T . P^T         the same key tile read
 //           MN-major (M = 128 dims per MMA, 4 tiles), N = 64, K = 128 keys
-//   epilogue: O^T from TMEM to shared memory as [head][dim] fp32, then
-//     split mode:  coalesced 16-byte stores of the unnormalised partial and
-//                  the slice's (max, sum) per head; sparse_attn_combine_kernel
-//                  merges the slices;
+//   epilogue, by mode:
+//     cluster merge (split mode with at most 8 slices): the query's slice
+//                  CTAs form one thread-block cluster.  Each CTA sends its
+//                  per-head (max, sum) to all the others through distributed
+//                  shared memory; every CTA then knows the joint max M and
+//                  sum L, scales its own O^T by exp2(m - M) / L while reading
+//                  it from TMEM and sends each 32-dim chunk, rounded to bf16
+//                  (the output's precision; the sum is taken in fp32), to
+//                  the CTA that owns it (chunk c belongs to rank c mod C);
+//                  the owner adds the chunks and writes bf16.  No partial
+//                  leaves the SMs.
+//     split mode, more slices: coalesced 16-byte stores of the unnormalised
+//                  partial and the slice's (max, sum) per head;
+//                  sparse_attn_combine_kernel merges the slices;
 //     one CTA per query: normalised by the running sum, written as bf16 with
 //                  the log-sum-exp.
 // Accumulators: S^T in TMEM columns [0, 64), O^T tile t in [64 + 64t, 128 + 64t).
@@ -37,7 +48,9 @@ constexpr int kTcAttnKeys = 128;                       // keys per slice (MMA M)
 constexpr uint32_t kTcKeyTileBytes = 128 * 512 * 2;    // 128 KB: 8 chunks of [128 rows x 64 dims]
 constexpr uint32_t kTcQTileBytes = 64 * 512 * 2;       // 64 KB: 8 chunks of [64 rows x 64 dims]
 constexpr uint32_t kTcPTileBytes = 128 * 64 * 2;       // 16 KB: P^T [128 keys][64 heads]
-constexpr uint32_t kTcMiscBytes = 4096;
+constexpr uint32_t kTcMiscBytes = 8192;                // barriers, flags, softmax scratch, cluster statistics
+constexpr int kTcMaxClusterSlices = 8;                 // cluster merge: at most this many slices per query
+constexpr uint32_t kTcStatOff = 4096;                  // misc offset of the cluster statistics [8 ranks][64][2]
 constexpr uint32_t kTcAttnSmem = kTcKeyTileBytes + kTcQTileBytes + kTcPTileBytes + kTcMiscBytes + 1024;
 constexpr float kTcRefSlack = 8.0f;                    // log2 units a slice max may exceed the reference
 
@@ -51,6 +64,8 @@ struct TcAttnParams {
   int slices;
   float scale_log2;
   int per_query;             // 1: one CTA per query over all slices, final output; 0: one slice per CTA
+  int cluster_merge;         // split mode in clusters of `slices` CTAs: merge over distributed shared
+                             // memory and write the final output (no partials)
   int early_inputs;          // 1: q and the window rows are complete at launch (the predecessor is a
                              // kernel of this library): load them before waiting on it
   float* opart;              // split: [BQ][slices][64][512]
@@ -108,6 +123,43 @@ __device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, __nv_bfloat162 scale,
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Distributed shared memory: the address of the same shared-memory location
+// in CTA `rank` of the cluster, and a store there.
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void dsmem_st_f32x2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" :: "r"(addr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void dsmem_st_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
 }
 
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -194,6 +246,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     fence_barrier_init();
   }
   if (tid < 64) { ref_s[tid] = -INFINITY; sum_s[tid] = 0.0f; }
+  // cluster merge: every CTA of the cluster has started before another one
+  // writes its shared memory (arrive now, wait before the first remote store)
+  if (p.cluster_merge) cluster_arrive_relaxed();
   if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   if (tid == 0) { tma_prefetch_desc(&tmap_q); tma_prefetch_desc(&tmap_swa); }
   pdl_launch_dependents();
@@ -216,9 +271,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const int key0 = window ? (slice - p.kv_slices) * kTcAttnKeys : slice * kTcAttnKeys;   // first key of the slice
     const int nkeys = window ? min(kTcAttnKeys, p.W - key0) : min(kTcAttnKeys, p.K - key0);
     const uint32_t ph = static_cast<uint32_t>(it & 1);                 // MMA barriers complete once per slice
-    // row-gather and window barriers complete once per slice of their kind
-    // (KV slices come first); in split mode each is used once
-    const uint32_t ph_rows = p.per_query ? static_cast<uint32_t>(slice & 1) : 0u;
+    // the window barrier completes once per window slice (KV slices come
+    // first); in split mode it is used at most once
     const uint32_t ph_win = p.per_query ? static_cast<uint32_t>((slice - p.kv_slices) & 1) : 0u;
 
     // the key tile and P^T are free once the previous slice's MMA 2 is done
@@ -239,48 +293,49 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       }
       valid_s[tid] = v;
     }
-    const int n_rows = __syncthreads_count(!window && v != 0);   // FP4 rows to gather
+    __syncthreads();
 
-    // ---- operands: window rows by TMA; FP4 rows by one bulk copy each into
-    //      a staging area inside the key tile, then dequantised
-    uint8_t* stage = kt;                                  // [128][288] raw rows (overwritten below)
-    if (tid == 0) {
+    // ---- operands: window rows by TMA; FP4 rows loaded by the threads
+    //      (read-only path, 16 nibble bytes + 2 scales per item) and
+    //      dequantised in registers
+    if (tid == 0 && window) {
       const uint64_t pol = l2_policy_evict_last();
-      if (!window) {
-        if (n_rows) mbar_arrive_expect_tx(&bars[3], static_cast<uint32_t>(n_rows) * 288u);
-        else mbar_arrive(&bars[3]);
-      } else {
-        mbar_arrive_expect_tx(&bars[4], kTcKeyTileBytes);
-        const int32_t y = b * p.swa_rows + qi * p.swa_step + key0;
-        for (int c = 0; c < 8; ++c) tma_load_2d(kt + c * 16384, &tmap_swa, &bars[4], 64 * c, y, pol);
-      }
+      mbar_arrive_expect_tx(&bars[4], kTcKeyTileBytes);
+      const int32_t y = b * p.swa_rows + qi * p.swa_step + key0;
+      for (int c = 0; c < 8; ++c) tma_load_2d(kt + c * 16384, &tmap_swa, &bars[4], 64 * c, y, pol);
     }
     if (!window) {
-      __syncthreads();                                    // expect_tx is posted before any copy lands
-      if (tid < kTcAttnKeys && v != 0) {
-        const uint8_t* row = p.kv + (static_cast<int64_t>(b) * p.N + (v - 1)) * 288;
-        asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 288, [%2];"
-            :: "r"(smem_u32(stage + tid * 288)), "l"(row), "r"(smem_u32(&bars[3])) : "memory");
+      // Gather: warp w loads keys 8w..8w+7, one 288-byte row per load (lane
+      // l < 18 loads bytes 16l..16l+15), all eight loads in flight at once,
+      // into a staging area at the start of the key tile.  Then every thread
+      // takes four items (key r, 32-channel chunk c: 16 nibble bytes and two
+      // scales) from the staging area into registers, and after a barrier
+      // expands them into the tile, which overwrites the staging area.  A
+      // warp's items are 32 consecutive keys of one chunk, so its swizzled
+      // 16-byte stores hit 32 different bank groups.
+      uint8_t* stage = kt;                                // [128 keys][288 B]
+      uint4 raw[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int vr = valid_s[8 * warp + j];
+        raw[j] = make_uint4(0, 0, 0, 0);
+        if (vr != 0 && lane < 18)
+          raw[j] = __ldg(reinterpret_cast<const uint4*>(p.kv + (static_cast<int64_t>(b) * p.N + (vr - 1)) * 288) + lane);
       }
-      // item = (key r, 32-channel chunk c): 16 nibble bytes + 2 scales -> four
-      // 16-byte units of the key tile.  A warp takes 32 consecutive keys of one
-      // chunk (conflict-free swizzled stores).  All raw items go to registers
-      // before anything is written, since the tile overwrites the staging area.
+      if (lane < 18) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(stage + (8 * warp + j) * 288 + 16 * lane) = raw[j];
+      }
+      __syncthreads();
       constexpr int kItems = kTcAttnKeys * 16 / kTcAttnThreads;
-      const bool ok = mbar_wait(&bars[3], ph_rows, kErrWaitOperand, abort_flag);
       uint4 nib[kItems];
       uint32_t sc[kItems];
 #pragma unroll
       for (int k = 0; k < kItems; ++k) {
         const int i = tid + k * kTcAttnThreads;
         const int r = i & (kTcAttnKeys - 1), c = i >> 7;
-        nib[k] = make_uint4(0, 0, 0, 0);
-        sc[k] = 0;
-        if (ok && valid_s[r]) {
-          nib[k] = *reinterpret_cast<const uint4*>(stage + r * 288 + c * 16);
-          sc[k] = *reinterpret_cast<const uint16_t*>(stage + r * 288 + 256 + 2 * c);
-        }
+        nib[k] = *reinterpret_cast<const uint4*>(stage + r * 288 + c * 16);
+        sc[k] = *reinterpret_cast<const uint16_t*>(stage + r * 288 + 256 + 2 * c);
       }
       __syncthreads();
 #pragma unroll
@@ -386,7 +441,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (f != 1.0f && it > 0) *rescale_flag = 1;       // the accumulator holds earlier slices
         ref_s[h] = nref;
         sum_s[h] = sum_s[h] * f + l;
-        if (!p.per_query) {
+        if (!p.per_query && !p.cluster_merge) {
           if (p.early_inputs && window) pdl_wait();
           float* ml = p.ml + ((static_cast<int64_t>(bq) * p.slices + slice) * 64 + h) * 2;
           ml[0] = nref;
@@ -440,6 +495,114 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       }
       umma_commit(&bars[2]);
     }
+  }
+
+  if (p.cluster_merge) {
+    // ---- cluster merge.  Every CTA reaches both cluster barriers whatever
+    //      happened before (all earlier waits are bounded), so no CTA of the
+    //      cluster can be left waiting.
+    const uint32_t C = cluster_size(), rank = cluster_rank();
+    const uint32_t jmax = (16 + C - 1) / C;              // 32-dim chunks per owner
+    float* stat = reinterpret_cast<float*>(misc + kTcStatOff);    // [rank][64 heads][max, sum]
+    // recv[source rank][chunk j][head group 0..7][dim 0..31][8 heads bf16]:
+    // one warp store puts 32 consecutive 16-byte pieces (512 contiguous
+    // bytes) into the owner, the fewest and largest remote packets
+    uint8_t* recv = kt;
+    const bool ok = mbar_wait(&bars[2], 0, kErrWaitTmemFull, abort_flag);   // MMA 2 done
+    cluster_wait_acquire();                              // pairs with the arrive at the start
+    if (tid < 64) {
+      const uint32_t la = smem_u32(stat + (rank * 64 + tid) * 2);
+      for (uint32_t r = 0; r < C; ++r) dsmem_st_f32x2(dsmem_map(la, r), ref_s[tid], sum_s[tid]);
+    }
+    tc_fence_before();
+    cluster_arrive_release();
+    cluster_wait_acquire();                              // statistics everywhere; every CTA's MMA 2 done
+    tc_fence_after();
+    float* mj_s = red_s;                                 // [64] joint max, [64] joint sum (scratch reuse)
+    if (tid < 64) {
+      float M = -INFINITY;
+      for (uint32_t r = 0; r < C; ++r) M = fmaxf(M, stat[(r * 64 + tid) * 2]);
+      float L = 0.0f;
+      if (M != -INFINITY)
+        for (uint32_t r = 0; r < C; ++r) {
+          const float m = stat[(r * 64 + tid) * 2];
+          if (m != -INFINITY) L += exp2f(m - M) * stat[(r * 64 + tid) * 2 + 1];
+        }
+      const float m = ref_s[tid];
+      fac_s[tid] = (L > 0.0f && m != -INFINITY) ? exp2f(m - M) / L : 0.0f;
+      mj_s[tid] = M;
+      mj_s[64 + tid] = L;
+    }
+    __syncthreads();
+    {
+      // warp w holds dims 32w..32w+31 (TMEM lanes 32(w%4).., tile w/4) for
+      // all 64 heads; chunk w goes, scaled and rounded to bf16 (the final
+      // output's precision), to rank w mod C: 8 vector stores of 8 heads
+      const int quarter = warp & 3, t = warp >> 2;
+      const uint32_t owner = static_cast<uint32_t>(warp) % C, j = static_cast<uint32_t>(warp) / C;
+      const uint32_t base = smem_u32(recv + ((rank * jmax + j) * 8) * 512 + 16 * lane);
+      const uint32_t rbase = dsmem_map(base, owner);
+      const bool all_ok = __all_sync(0xffffffffu, ok);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[32];
+        if (all_ok) {
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64 + 64 * t + 32 * hh, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) r[jj] = 0u;
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h = 32 * hh + 8 * g + 2 * e;
+            pk[e] = pack_bf16x2(__uint_as_float(r[8 * g + 2 * e]) * fac_s[h],
+                                __uint_as_float(r[8 * g + 2 * e + 1]) * fac_s[h + 1]);
+          }
+          dsmem_st_v4(rbase + (4 * hh + g) * 512, pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    tc_fence_before();
+    cluster_arrive_release();
+    cluster_wait_acquire();                              // every chunk delivered to its owner
+    if (p.early_inputs) pdl_wait();                      // stores wait for the predecessor
+    if (!*abort_flag) {
+      // this CTA's chunks c = rank + C j: item (j, head group of 8, dim d) sums
+      // the C sources in fp32; lanes run over d, so each of the 8 bf16 stores
+      // of an item writes 64 contiguous bytes per warp
+      const uint32_t nown = (16 - rank + C - 1) / C;
+      for (uint32_t it = warp; it < nown * 8; it += kTcAttnThreads / 32) {
+        const uint32_t j = it >> 3, hg = it & 7, d = lane;
+        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (uint32_t r = 0; r < C; ++r) {
+          const uint4 v = *reinterpret_cast<const uint4*>(recv + ((r * jmax + j) * 8 + hg) * 512 + 16 * d);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            a[2 * e] += f.x;
+            a[2 * e + 1] += f.y;
+          }
+        }
+        const uint32_t c = rank + C * j;
+        __nv_bfloat16* o = p.out + (static_cast<int64_t>(bq) * 64 + 8 * hg) * 512 + 32 * c + d;
+  #pragma unroll
+        for (int e = 0; e < 8; ++e) o[e * 512] = __float2bfloat16_rn(a[e]);
+      }
+      if (rank == 0 && p.lse && tid < 64) {
+        const float L = mj_s[64 + tid];
+        p.lse[static_cast<int64_t>(bq) * 64 + tid] = (L > 0.0f) ? (mj_s[tid] + log2f(L)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+    if (warp == 1) {                                     // TMEM was last read before the second barrier
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+    return;
   }
 
   // ---- epilogue: O^T tile (warp / 4), dims 32(warp % 4).. -> shared

@@ -157,6 +157,7 @@ bool make_map_bf16_128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t
 }
 
 // ---------------------------------------------------------------- index call
+
 struct IndexPlan {
   bool pool, hsi;
   int BQ, qg, hb;
@@ -288,7 +289,6 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.stages = std::min(kScanStages, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / kStageBytes));
   if (sp.stages < 2) return CSA2_ERR_SHAPE;
   const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi);
-
   CUtensorMap tk, tq;
   if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : kTileRows)) return CSA2_ERR_CUDA;
   if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, n_mma)) return CSA2_ERR_CUDA;
@@ -377,8 +377,16 @@ inline bool attn_per_query(const csa2_attn_args* a) {
   return static_cast<int64_t>(a->B) * a->Q >= kAttnPerQueryMinBQ;
 }
 
+// Split mode with few enough slices: the slice CTAs of a query form one
+// cluster and merge over distributed shared memory (no partials, no merge
+// kernel).
+inline bool attn_cluster_merge(const csa2_attn_args* a) {
+  return !attn_per_query(a) && attn_slices(a) <= kTcMaxClusterSlices;
+}
+
 size_t attn_ws_bytes(const csa2_attn_args* a) {
-  if (attn_per_query(a)) return 256;            // unused; the size query stays non-zero for valid arguments
+  // unused in these modes; the size query stays non-zero for valid arguments
+  if (attn_per_query(a) || attn_cluster_merge(a)) return 256;
   const size_t bq = static_cast<size_t>(a->B) * a->Q, s = attn_slices(a);
   return up256(bq * s * 64 * 512 * 4) + up256(bq * s * 64 * 2 * 4);
 }
@@ -401,10 +409,12 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st, bool ea
   t.slices = slices;
   t.scale_log2 = scale * 1.4426950408889634f;
   const bool per_query = attn_per_query(a);
+  const bool cluster = attn_cluster_merge(a);
   t.per_query = per_query ? 1 : 0;
+  t.cluster_merge = cluster ? 1 : 0;
   t.early_inputs = early_inputs ? 1 : 0;
-  t.opart = per_query ? nullptr : opart;
-  t.ml = per_query ? nullptr : ml;
+  t.opart = (per_query || cluster) ? nullptr : opart;
+  t.ml = (per_query || cluster) ? nullptr : ml;
   t.out = static_cast<__nv_bfloat16*>(a->out);
   t.lse = a->lse;
   CUtensorMap tq, tw;
@@ -416,10 +426,11 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st, bool ea
   }
   trace_pre(kKAttnSlice, st);
   const cudaError_t e1 = launch_ex(sparse_attn_tc_kernel, dim3(per_query ? 1 : slices, static_cast<unsigned>(bq)),
-                                   dim3(kTcAttnThreads), kTcAttnSmem, st, 0, tq, tw, t);
+                                   dim3(kTcAttnThreads), kTcAttnSmem, st, cluster ? static_cast<unsigned>(slices) : 0u,
+                                   tq, tw, t);
   trace_post(st);
   if (e1 != cudaSuccess) return CSA2_ERR_CUDA;
-  if (per_query) return CSA2_OK;
+  if (per_query || cluster) return CSA2_OK;
 
   AttnParams p;
   p.slices = slices;

@@ -204,10 +204,13 @@ size_t csa2_noalloc_scratch_bytes(void);
  * [0, swa_rows).
  *
  * With fewer than 128 queries per call (B*Q) the keys of a query are split
- * into 128-key slices over several CTAs whose fp32 partial outputs go to
- * the workspace and are merged by a second kernel; with 128 or more, one
- * CTA per query walks all its slices and the workspace is not used
- * (csa2_workspace_size still returns a small non-zero size).
+ * into 128-key slices over several CTAs: up to 8 slices (K + W <= 1024)
+ * they form one thread-block cluster and merge their results through
+ * distributed shared memory; with more, their fp32 partial outputs go to
+ * the workspace and are merged by a second kernel.  With 128 or more
+ * queries, one CTA per query walks all its slices.  Only the second-kernel
+ * case uses the workspace (csa2_workspace_size still returns a small
+ * non-zero size for the others).
  * ---------------------------------------------------------------------- */
 typedef struct csa2_attn_args {
     int32_t        B, Q;        /* batch rows >= 1; queries per row, B*Q <= CSA2_MAX_BQ */

@@ -62,6 +62,10 @@ def _oracle(kv, q, swa, idx, W, swa_step, scale=None):
     (1, 1, 10, 0, 128, 0, 4, 0.0),         # window only
     (1, 130, 3000, 512, 128, 1, 7, 0.05),  # 130 queries: one CTA per query over all its slices
     (2, 70, 900, 200, 100, 1, 8, 0.0),     # per query, ragged slices
+    (2, 1, 1500, 512, 256, 0, 10, 0.0),    # 6 slices merged in one cluster
+    (1, 2, 1500, 896, 128, 0, 11, 0.02),   # 8 slices: the largest cluster
+    (1, 2, 1500, 1024, 128, 0, 12, 0.0),   # 9 slices: partials and the merge kernel
+    (3, 1, 500, 130, 0, 0, 13, 0.0),       # 2 slices, the second with 2 keys
 ])
 def test_attention_parity(B, Q, N, K, W, step, seed, m1):
     kv, q, swa, idx = _case(B, Q, N, K, W, step, seed, minus_one=m1)
