@@ -163,11 +163,21 @@ class ClockSampler:
 # algorithmic bytes
 # ---------------------------------------------------------------------------
 
+def index_k_entry_bytes(wl):
+    """Bytes of one index-K entry: 256 (bf16) or 68 (MXFP4)."""
+    return 68 if wl.index_k_format == 2 else 256
+
+
+def window_row_bytes(wl):
+    """Bytes of one window row: 1024 (bf16) or 516 (E4M3 codes + f32 scale)."""
+    return 516 if wl.window_format == 1 else 1024
+
+
 def scan_algorithmic_bytes(wl):
     """Bytes one Full / Reindex index_scan_kernel launch must move: index-K
     rows once per batch row, one fp32 score per (query, entry), index-Q and
     w of every query."""
-    per_row = wl.N * 128 * 2 + wl.Q * wl.N * 4 + wl.Q * (32 * 128 * 2 + 32 * 4)
+    per_row = wl.N * index_k_entry_bytes(wl) + wl.Q * wl.N * 4 + wl.Q * (32 * 128 * 2 + 32 * 4)
     return wl.B * per_row
 
 
@@ -176,7 +186,7 @@ def pool_scan_algorithmic_bytes(wl):
     the pool's block ids, 8 index-K rows per block, one fp32 score per pool
     position, index-Q and w."""
     P = wl.hsi_blocks * wl.hsi_block
-    return wl.B * wl.Q * (wl.hsi_blocks * 4 + P * 128 * 2 + P * 4 + 32 * 128 * 2 + 32 * 4)
+    return wl.B * wl.Q * (wl.hsi_blocks * 4 + P * index_k_entry_bytes(wl) + P * 4 + 32 * 128 * 2 + 32 * 4)
 
 
 def scan_algorithmic_flops(wl):
@@ -198,7 +208,7 @@ def attention_algorithmic_bytes(wl):
     """Bytes of one attention launch: per query the K indices, K selected FP4
     entries (288 B), W window rows (1 KB bf16), the 64 x 512 bf16 query and
     the 64 x 512 bf16 output."""
-    return wl.B * wl.Q * (wl.K * 4 + wl.K * 288 + wl.W * 1024 + 2 * 64 * 512 * 2)
+    return wl.B * wl.Q * (wl.K * 4 + wl.K * 288 + wl.W * window_row_bytes(wl) + 2 * 64 * 512 * 2)
 
 
 def quantize_algorithmic_bytes(wl):
@@ -308,7 +318,9 @@ def bench_config(wl, world):
             "layers": ",".join(workloads.MODE_NAMES[m] for m in wl.modes), "K": wl.K, "W": wl.W,
             "hsi_pool": f"{wl.hsi_blocks}x{wl.hsi_block}" if wl.hsi_blocks else None,
             "groups": len(wl.groups), "cache_per_group": wl.cache_per_group,
-            "kv_cache": "FP4 E2M1 + E4M3/16ch (288 B/entry)", "index_k": "bf16", "window": "bf16",
+            "kv_cache": "FP4 E2M1 + E4M3/16ch (288 B/entry)",
+            "index_k": "MXFP4 (68 B/entry)" if wl.index_k_format == 2 else "bf16",
+            "window": "FP8 E4M3 + f32 row scale" if wl.window_format == 1 else "bf16",
             "l2": "flushed between steps (256 MB memset outside the timed events)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
@@ -334,17 +346,22 @@ def oracle_row_setup(wl, b):
     queries: its FP4 cache built by the oracle's own quantiser (only the rows
     the oracle's layers will read are filled: attention reads nothing else),
     index-K and the sampled queries' layer inputs and windows."""
-    from oracle import fp4, group, indexer
+    from oracle import fp4, fp8, group, indexer, mxfp4
     q0, qn = oracle_query_sample(wl)
     x = workloads.main_kv_rows(wl, b, 0, wl.N).float().numpy()
     kI = workloads.index_k(wl, b).float().numpy()
+    if wl.index_k_format == 2:                  # the pages' FP4 index-K, dequantised
+        kI = mxfp4.dequantize_index_k_mxfp4(mxfp4.quantize_index_k_mxfp4(kI))
     n_vis = np.array(wl.n_vis[q0:q0 + qn])
     w0, w1 = q0 * wl.swa_step, (q0 + qn - 1) * wl.swa_step + wl.W
     layers = []
     for l, mode in enumerate(wl.modes):
         li = workloads.layer_inputs(wl, l)
+        swa = li["swa"][b].float().numpy()
+        if wl.window_format == 1:               # FP8 window rows, dequantised
+            swa = fp8.dequantize_window_fp8(*fp8.quantize_window_fp8(swa))
         layers.append(dict(mode=mode, qI=li["qI"][b, q0:q0 + qn].float().numpy(), w=li["w"][b, q0:q0 + qn].numpy(),
-                           q=li["q"][b, q0:q0 + qn].float().numpy(), swa=li["swa"][b, w0:w1].float().numpy()))
+                           q=li["q"][b, q0:q0 + qn].float().numpy(), swa=swa[w0:w1]))
     need = set(wl.new_rows)
     for L in layers:
         if L["mode"] in (group.FULL, group.REINDEX):

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libcsa2.so")
 FULL, REINDEX, REINDEX_POOL, REUSE = 0, 1, 2, 3
 WS_INDEX, WS_ATTN, WS_GROUP, WS_STACK = 1, 2, 3, 4
 GROUP_INPUTS_READY, GROUP_SERIAL = 1, 2
+FMT_BF16, FMT_FP8, FMT_MXFP4 = 0, 1, 2
 ENTRY_BYTES = 288
 
 _c_i32, _c_i64, _c_f32, _c_p = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
@@ -31,19 +32,20 @@ class Csa2Error(RuntimeError):
 class IndexArgs(ctypes.Structure):
     _fields_ = [("mode", _c_i32), ("B", _c_i32), ("Q", _c_i32), ("K", _c_i32), ("N", _c_i64),
                 ("qI", _c_p), ("w", _c_p), ("kI", _c_p), ("n_vis", _c_p), ("idx", _c_p), ("scores", _c_p),
-                ("hsi_blocks", _c_i32), ("hsi_block", _c_i32), ("pool_out", _c_p), ("pool_in", _c_p)]
+                ("hsi_blocks", _c_i32), ("hsi_block", _c_i32), ("pool_out", _c_p), ("pool_in", _c_p),
+                ("k_format", _c_i32)]
 
 
 class AttnArgs(ctypes.Structure):
     _fields_ = [("B", _c_i32), ("Q", _c_i32), ("K", _c_i32), ("W", _c_i32), ("N", _c_i64),
                 ("q", _c_p), ("kv_fp4", _c_p), ("idx", _c_p), ("swa", _c_p),
                 ("swa_rows", _c_i32), ("swa_step", _c_i32), ("scale", _c_f32),
-                ("out", _c_p), ("lse", _c_p)]
+                ("out", _c_p), ("lse", _c_p), ("swa_format", _c_i32), ("swa_scale", _c_p)]
 
 
 class Layer(ctypes.Structure):
     _fields_ = [("mode", _c_i32), ("qI", _c_p), ("w", _c_p), ("q", _c_p), ("swa", _c_p),
-                ("out", _c_p), ("lse", _c_p), ("idx", _c_p), ("scores", _c_p)]
+                ("out", _c_p), ("lse", _c_p), ("idx", _c_p), ("scores", _c_p), ("swa_scale", _c_p)]
 
 
 class GroupArgs(ctypes.Structure):
@@ -51,7 +53,8 @@ class GroupArgs(ctypes.Structure):
                 ("n_vis", _c_p), ("kI", _c_p), ("kv_fp4", _c_p), ("kv_new", _c_p), ("n_new", _c_i64),
                 ("new_rows", _c_p), ("swa_rows", _c_i32), ("swa_step", _c_i32),
                 ("hsi_blocks", _c_i32), ("hsi_block", _c_i32), ("pool", _c_p), ("scale", _c_f32),
-                ("n_layers", _c_i32), ("layers", ctypes.POINTER(Layer)), ("pool_in", _c_p), ("flags", _c_i32)]
+                ("n_layers", _c_i32), ("layers", ctypes.POINTER(Layer)), ("pool_in", _c_p), ("flags", _c_i32),
+                ("swa_format", _c_i32), ("index_k_format", _c_i32)]
 
 
 class StackArgs(ctypes.Structure):
@@ -71,6 +74,8 @@ def load(path=LIB_PATH):
                       f"`python -m fp4_kv_cache_mxfp4_b200.build`")
     lib = ctypes.CDLL(path)
     lib.csa2_quantize_kv_fp4.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_p]
+    lib.csa2_quantize_window_fp8.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_i64, _c_p]
+    lib.csa2_quantize_index_k_mxfp4.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_p]
     lib.csa2_index_score_topk.argtypes = [ctypes.POINTER(IndexArgs), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexArgs), _c_p]
     lib.csa2_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), _c_p, ctypes.c_size_t, _c_p]
@@ -91,7 +96,8 @@ def load(path=LIB_PATH):
     lib.csa2_trace_count.restype = _c_i32
     lib.csa2_kernel_name.argtypes = [_c_i32]
     lib.csa2_kernel_name.restype = ctypes.c_char_p
-    for name in ("csa2_quantize_kv_fp4", "csa2_index_score_topk", "csa2_index_score_topk_noalloc", "csa2_sparse_attn",
+    for name in ("csa2_quantize_kv_fp4", "csa2_quantize_window_fp8", "csa2_quantize_index_k_mxfp4",
+                 "csa2_index_score_topk", "csa2_index_score_topk_noalloc", "csa2_sparse_attn",
                  "csa2_group_decode", "csa2_stack_decode", "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
                  "csa2_trace_end", "csa2_trace_get"):
         getattr(lib, name).restype = _c_i32
@@ -141,13 +147,31 @@ def csa2_quantize_kv_fp4(x, kv_fp4, dst_rows=None, row_offset=0, stream=None):
                                        row_offset, _stream(stream)), "csa2_quantize_kv_fp4")
 
 
+def csa2_quantize_window_fp8(x, codes, scales, dst_rows=None, row_offset=0, stream=None):
+    """x bf16 [n, >=512], codes uint8 [rows, 512], scales float32 [rows],
+    dst_rows optional int64 [n]."""
+    n = x.shape[0]
+    _check(load().csa2_quantize_window_fp8(_ptr(x), n, x.stride(0) if n else 512, _ptr(codes), _ptr(scales),
+                                           _ptr(dst_rows), row_offset, _stream(stream)), "csa2_quantize_window_fp8")
+
+
+def csa2_quantize_index_k_mxfp4(x, out, dst_rows=None, row_offset=0, stream=None):
+    """x bf16 [n, >=128], out uint8 [rows, 68], dst_rows optional int64 [n]."""
+    n = x.shape[0]
+    _check(load().csa2_quantize_index_k_mxfp4(_ptr(x), n, x.stride(0) if n else 128, _ptr(out), _ptr(dst_rows),
+                                              row_offset, _stream(stream)), "csa2_quantize_index_k_mxfp4")
+
+
 def index_args(mode, qI, w, kI, n_vis, idx, scores=None, hsi_blocks=0, hsi_block=8, pool_out=None, pool_in=None):
     """Build csa2_index_args from tensors: qI [B,Q,32,128], w [B,Q,32],
-    kI [B,N,128], n_vis int32 [B,Q], idx int32 [B,Q,K]."""
+    kI bf16 [B,N,128] (or uint8 [B,N,68] MXFP4 entries), n_vis int32 [B,Q],
+    idx int32 [B,Q,K]."""
     B, Q = qI.shape[0], qI.shape[1]
+    mx = kI.dtype == torch.uint8
     a = IndexArgs(mode=mode, B=B, Q=Q, K=idx.shape[-1], N=kI.shape[1],
                   qI=_ptr(qI), w=_ptr(w), kI=_ptr(kI), n_vis=_ptr(n_vis), idx=_ptr(idx), scores=_ptr(scores),
-                  hsi_blocks=hsi_blocks, hsi_block=hsi_block, pool_out=_ptr(pool_out), pool_in=_ptr(pool_in))
+                  hsi_blocks=hsi_blocks, hsi_block=hsi_block, pool_out=_ptr(pool_out), pool_in=_ptr(pool_in),
+                  k_format=FMT_MXFP4 if mx else FMT_BF16)
     a._tensors = (qI, w, kI, n_vis, idx, scores, pool_out, pool_in)     # the struct holds raw pointers
     return a
 
@@ -170,15 +194,17 @@ def noalloc_scratch_bytes():
     return int(load().csa2_noalloc_scratch_bytes())
 
 
-def attn_args(q, kv_fp4, idx, swa, out, lse=None, W=128, swa_step=0, scale=0.0):
+def attn_args(q, kv_fp4, idx, swa, out, lse=None, W=128, swa_step=0, scale=0.0, swa_scale=None):
     """q [B,Q,64,512], kv_fp4 uint8 [B,N,288], idx int32 [B,Q,K], swa bf16
-    [B,rows,512], out bf16 [B,Q,64,512], lse f32 [B,Q,64]."""
+    [B,rows,512] (or uint8 E4M3 codes [B,rows,512] with swa_scale float32
+    [B,rows]), out bf16 [B,Q,64,512], lse f32 [B,Q,64]."""
     B, Q = q.shape[0], q.shape[1]
     a = AttnArgs(B=B, Q=Q, K=idx.shape[-1] if idx is not None else 0, W=W, N=kv_fp4.shape[1],
                  q=_ptr(q), kv_fp4=_ptr(kv_fp4), idx=_ptr(idx), swa=_ptr(swa),
                  swa_rows=swa.shape[1] if swa is not None else 0, swa_step=swa_step, scale=scale,
-                 out=_ptr(out), lse=_ptr(lse))
-    a._tensors = (q, kv_fp4, idx, swa, out, lse)     # the struct holds raw pointers
+                 out=_ptr(out), lse=_ptr(lse), swa_format=FMT_FP8 if swa_scale is not None else FMT_BF16,
+                 swa_scale=_ptr(swa_scale))
+    a._tensors = (q, kv_fp4, idx, swa, out, lse, swa_scale)     # the struct holds raw pointers
     return a
 
 
@@ -188,21 +214,24 @@ def csa2_sparse_attn(args, ws, stream=None):
 
 
 def group_args(B, Q, K, W, N, n_vis, kI, kv_fp4, layers, kv_new=None, new_rows=None, swa_rows=128, swa_step=0,
-               hsi_blocks=0, hsi_block=8, pool=None, scale=0.0, pool_in=None, flags=0):
+               hsi_blocks=0, hsi_block=8, pool=None, scale=0.0, pool_in=None, flags=0, swa_format=0):
     """``layers`` is a list of dicts with keys mode, qI, w, q, swa, out, lse,
     idx, scores (tensors or None).  ``pool_in`` is an HSI pool built by an
     earlier group; ``flags`` a combination of GROUP_INPUTS_READY and
-    GROUP_SERIAL.  The returned struct keeps its layer array alive."""
+    GROUP_SERIAL; ``swa_format`` FMT_FP8 when every layer's swa holds E4M3
+    codes with a ``swa_scale`` tensor.  The returned struct keeps its layer
+    array alive."""
     arr = (Layer * len(layers))()
     for i, L in enumerate(layers):
         arr[i] = Layer(mode=L["mode"], qI=_ptr(L.get("qI")), w=_ptr(L.get("w")), q=_ptr(L["q"]),
                        swa=_ptr(L["swa"]), out=_ptr(L["out"]), lse=_ptr(L.get("lse")),
-                       idx=_ptr(L.get("idx")), scores=_ptr(L.get("scores")))
+                       idx=_ptr(L.get("idx")), scores=_ptr(L.get("scores")), swa_scale=_ptr(L.get("swa_scale")))
     g = GroupArgs(B=B, Q=Q, K=K, W=W, N=N, n_vis=_ptr(n_vis), kI=_ptr(kI), kv_fp4=_ptr(kv_fp4),
                   kv_new=_ptr(kv_new), n_new=0 if kv_new is None else kv_new.shape[0], new_rows=_ptr(new_rows),
                   swa_rows=swa_rows, swa_step=swa_step, hsi_blocks=hsi_blocks, hsi_block=hsi_block,
                   pool=_ptr(pool), scale=scale, n_layers=len(layers),
-                  layers=ctypes.cast(arr, ctypes.POINTER(Layer)), pool_in=_ptr(pool_in), flags=flags)
+                  layers=ctypes.cast(arr, ctypes.POINTER(Layer)), pool_in=_ptr(pool_in), flags=flags,
+                  swa_format=swa_format, index_k_format=FMT_MXFP4 if kI.dtype == torch.uint8 else FMT_BF16)
     g._layer_array = arr
     # the structs hold raw pointers: keep every tensor alive with them
     g._tensors = (n_vis, kI, kv_fp4, kv_new, new_rows, pool, pool_in, [dict(L) for L in layers])

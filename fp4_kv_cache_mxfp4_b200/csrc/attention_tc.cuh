@@ -68,17 +68,14 @@ struct TcAttnParams {
                              // memory and write the final output (no partials)
   int early_inputs;          // 1: q and the window rows are complete at launch (the predecessor is a
                              // kernel of this library): load them before waiting on it
+  int swa_fp8;               // 1: window rows are E4M3 codes [B][swa_rows][512] with one fp32 scale per row
+  const uint8_t* swa8;
+  const float* swa_scale;    // [B][swa_rows]
   float* opart;              // split: [BQ][slices][64][512]
   float* ml;                 // split: [BQ][slices][64][2]
   __nv_bfloat16* out;        // per query: [BQ][64][512]
   float* lse;                // per query, optional: [BQ][64]
 };
-
-// byte offset of the 16-byte unit u (0..7) of row r in a K-major operand
-// chunk of 128-byte rows with the 128-byte swizzle
-__device__ __forceinline__ uint32_t sw128_off(int r, int u) {
-  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4));
-}
 
 // Shared-memory descriptor of an MN-major operand in the 128-byte-swizzle
 // canonical layout: 64-element (128 B) rows along M, 8-row swizzle atoms
@@ -94,31 +91,21 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mnmajor(uint32_t smem_addr, 
   return d;
 }
 
-// Eight E2M1 codes (one 32-bit word of nibbles, code k in bits 4k..4k+3)
-// to eight bf16 values (out[j] = codes 2j, 2j+1), times a bf16 scale.
-// The magnitude (3 bits) selects the high and the low byte of the bf16
-// pattern from two 8-byte tables held in registers (byte_perm); the sign
-// bit is placed separately.  Products E2M1 x E4M3 are exact in bf16.
-//   magnitude code:  0    1     2     3     4     5     6     7
-//   value:           0    0.5   1     1.5   2     3     4     6
-//   bf16:            0000 3F00  3F80  3FC0  4000  4040  4080  40C0
-__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, __nv_bfloat162 scale, uint32_t (&out)[4]) {
-  const uint32_t m = w & 0x77777777u;
-  const uint32_t lo_a = __byte_perm(0xC0800000u, 0xC0804000u, m);
-  const uint32_t hi_a = __byte_perm(0x3F3F3F00u, 0x40404040u, m);
-  const uint32_t lo_b = __byte_perm(0xC0800000u, 0xC0804000u, m >> 16);
-  const uint32_t hi_b = __byte_perm(0x3F3F3F00u, 0x40404040u, m >> 16);
-  uint32_t o[4];
-  o[0] = __byte_perm(lo_a, hi_a, 0x5140) | ((w << 12) & 0x8000u) | ((w << 24) & 0x80000000u);
-  o[1] = __byte_perm(lo_a, hi_a, 0x7362) | ((w << 4) & 0x8000u) | ((w << 16) & 0x80000000u);
-  o[2] = __byte_perm(lo_b, hi_b, 0x5140) | ((w >> 4) & 0x8000u) | ((w << 8) & 0x80000000u);
-  o[3] = __byte_perm(lo_b, hi_b, 0x7362) | ((w >> 12) & 0x8000u) | (w & 0x80000000u);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&o[j]);
-    x = __hmul2(x, scale);
-    out[j] = *reinterpret_cast<uint32_t*>(&x);
-  }
+// Four E4M3 codes (bytes of w) to four bf16 values, exactly.  Placing the
+// code's exponent and mantissa bits at the bottom of a bf16 exponent field
+// gives E4M3(c) * 2^-120 for normal and subnormal codes alike (both formats
+// have a hidden bit and gradual underflow); one multiply by 2^120 restores
+// the value.  lo = codes 0, 1; hi = codes 2, 3.
+__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t a = __byte_perm(w, 0u, 0x4140);     // bytes 0, 1 -> bits 0-7, 16-23
+  const uint32_t c = __byte_perm(w, 0u, 0x4342);     // bytes 2, 3
+  const uint32_t ma = ((a & 0x007F007Fu) << 4) | ((a & 0x00800080u) << 8);
+  const uint32_t mc = ((c & 0x007F007Fu) << 4) | ((c & 0x00800080u) << 8);
+  const __nv_bfloat162 k = __floats2bfloat162_rn(1.329227995784916e36f, 1.329227995784916e36f);   // 2^120
+  __nv_bfloat162 x = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&ma), k);
+  __nv_bfloat162 y = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&mc), k);
+  lo = *reinterpret_cast<uint32_t*>(&x);
+  hi = *reinterpret_cast<uint32_t*>(&y);
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -232,6 +219,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   float* ref_s = reinterpret_cast<float*>(misc + 2624);              // [64] running reference max (log2 units)
   float* sum_s = reinterpret_cast<float*>(misc + 2880);              // [64] running sum of P
   float* fac_s = reinterpret_cast<float*>(misc + 3136);              // [64] rescale factor of this slice
+  float* wsc_s = reinterpret_cast<float*>(misc + 3392);              // [128] FP8 window: row scale per key
 
   const int bq = blockIdx.y;
   const int b = bq / p.Q, qi = bq % p.Q;
@@ -298,11 +286,40 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // ---- operands: window rows by TMA; FP4 rows loaded by the threads
     //      (read-only path, 16 nibble bytes + 2 scales per item) and
     //      dequantised in registers
-    if (tid == 0 && window) {
+    if (tid == 0 && window && !p.swa_fp8) {
       const uint64_t pol = l2_policy_evict_last();
       mbar_arrive_expect_tx(&bars[4], kTcKeyTileBytes);
       const int32_t y = b * p.swa_rows + qi * p.swa_step + key0;
       for (int c = 0; c < 8; ++c) tma_load_2d(kt + c * 16384, &tmap_swa, &bars[4], 64 * c, y, pol);
+    }
+    if (window && p.swa_fp8) {
+      // FP8 window rows: warp w loads rows 8w..8w+7 (512 codes, 16 per lane,
+      // one coalesced load per row), expands E4M3 to bf16 exactly and
+      // stores the key tile; the row scale multiplies the row's logits and
+      // its softmax weights later (wsc_s)
+      const int64_t row0 = static_cast<int64_t>(b) * p.swa_rows + qi * p.swa_step + key0;
+      if (tid < kTcAttnKeys) wsc_s[tid] = (tid < nkeys) ? p.swa_scale[row0 + tid] : 0.0f;
+      uint4 raw[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = 8 * warp + j;
+        raw[j] = (r < nkeys) ? __ldg(reinterpret_cast<const uint4*>(p.swa8 + (row0 + r) * 512) + lane)
+                             : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = 8 * warp + j;
+        uint32_t o[8];
+        e4m3x4_to_bf16(raw[j].x, o[0], o[1]);
+        e4m3x4_to_bf16(raw[j].y, o[2], o[3]);
+        e4m3x4_to_bf16(raw[j].z, o[4], o[5]);
+        e4m3x4_to_bf16(raw[j].w, o[6], o[7]);
+        // channels 16 lane .. 16 lane + 15 = chunk lane/4, units 2(lane%4), +1
+        uint8_t* chunk = kt + (lane >> 2) * 16384;
+        *reinterpret_cast<uint4*>(chunk + sw128_off(r, 2 * (lane & 3))) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(chunk + sw128_off(r, 2 * (lane & 3) + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+      fence_async_smem();
     }
     if (!window) {
       // Gather: warp w loads keys 8w..8w+7, one 288-byte row per load (lane
@@ -362,7 +379,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // ---- MMA 1: S^T = K . Q^T  (M = 128 keys, N = 64 heads, K = 512 dims)
     if (warp == 1 && lane == 0) {
       bool ok = mbar_wait(&bars[0], 0, kErrWaitOperand, abort_flag);
-      if (ok && window) ok = mbar_wait(&bars[4], ph_win, kErrWaitOperand, abort_flag);
+      if (ok && window && !p.swa_fp8) ok = mbar_wait(&bars[4], ph_win, kErrWaitOperand, abort_flag);
       if (ok) {
         tc_fence_after();
         constexpr uint32_t idesc = umma_idesc_bf16_f32(128, 64);
@@ -391,11 +408,13 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const bool kv_ok = valid_s[key] != 0;
+        // an FP8 window key's logits carry its row scale
+        const float ls = p.scale_log2 * ((window && p.swa_fp8) ? wsc_s[key] : 1.0f);
         uint32_t r[16];
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 16 * hg, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) sv[j] = kv_ok ? __uint_as_float(r[j]) * p.scale_log2 : -INFINITY;
+        for (int j = 0; j < 16; ++j) sv[j] = kv_ok ? __uint_as_float(r[j]) * ls : -INFINITY;
       }
       {
         const float m = warp_reduce_heads16<true>(sv, lane);
@@ -414,13 +433,32 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         lj[j] = exp2f(sv[j] - ((nref == -INFINITY) ? 0.0f : nref));
       }
       uint32_t pk[8];
+      if (window && p.swa_fp8) {
+        // MMA 2 multiplies the weight by the key's unscaled codes: fold the
+        // row scale into the weight it sees, and sum the weights that this
+        // rounded product stands for (weight = bf16(P s) / s), so that the
+        // output stays a normalised combination of the rows
+        const float rs = wsc_s[key];
+        const float inv = (rs != 0.0f) ? 1.0f / rs : 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const __nv_bfloat162 v2 = __floats2bfloat162_rn(lj[2 * j], lj[2 * j + 1]);
-        pk[j] = *reinterpret_cast<const uint32_t*>(&v2);
-        const float2 f = __bfloat1622float2(v2);        // the sum uses the rounded weights MMA 2 sees
-        lj[2 * j] = f.x;
-        lj[2 * j + 1] = f.y;
+        for (int j = 0; j < 8; ++j) {
+          const __nv_bfloat162 v2 = __floats2bfloat162_rn(lj[2 * j] * rs, lj[2 * j + 1] * rs);
+          pk[j] = *reinterpret_cast<const uint32_t*>(&v2);
+          if (rs != 0.0f) {
+            const float2 f = __bfloat1622float2(v2);
+            lj[2 * j] = f.x * inv;
+            lj[2 * j + 1] = f.y * inv;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const __nv_bfloat162 v2 = __floats2bfloat162_rn(lj[2 * j], lj[2 * j + 1]);
+          pk[j] = *reinterpret_cast<const uint32_t*>(&v2);
+          const float2 f = __bfloat1622float2(v2);      // the sum uses the rounded weights MMA 2 sees
+          lj[2 * j] = f.x;
+          lj[2 * j + 1] = f.y;
+        }
       }
       *reinterpret_cast<uint4*>(pt + sw128_off(key, 2 * hg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       *reinterpret_cast<uint4*>(pt + sw128_off(key, 2 * hg + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);

@@ -15,7 +15,8 @@ namespace csa2 {
 // Host-side launch tracing: when on, every kernel launch is bracketed by two
 // pre-created CUDA events recorded on the launch stream.
 // ---------------------------------------------------------------------------
-enum KernelId : int { kKQuantize = 0, kKIndexScan = 1, kKTopk = 2, kKAttnSlice = 3, kKAttnCombine = 4, kKCount = 5 };
+enum KernelId : int { kKQuantize = 0, kKIndexScan = 1, kKTopk = 2, kKAttnSlice = 3, kKAttnCombine = 4,
+                      kKQuantizeWindow = 5, kKQuantizeIndexK = 6, kKCount = 7 };
 
 struct LaunchTrace {
   bool on = false;
@@ -197,6 +198,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Untiled bulk copy global -> shared (both 16-byte aligned, size a multiple
+// of 16), completion on an mbarrier, streamed past L2 (evict first).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(l2_policy_evict_first())
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation MMA
 // ---------------------------------------------------------------------------
@@ -311,6 +321,39 @@ __device__ __forceinline__ void warp_hist_add(uint32_t* hist, uint32_t bin, bool
   if (!active) return;
   const uint32_t peers = __match_any_sync(live, bin);
   if ((threadIdx.x & 31) == static_cast<uint32_t>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+}
+
+// byte offset of the 16-byte unit u (0..7) of row r in a K-major operand
+// chunk of 128-byte rows with the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw128_off(int r, int u) {
+  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4));
+}
+
+// Eight E2M1 codes (one 32-bit word of nibbles, code k in bits 4k..4k+3)
+// to eight bf16 values (out[j] = codes 2j, 2j+1), times a bf16 scale.
+// The magnitude (3 bits) selects the high and the low byte of the bf16
+// pattern from two 8-byte tables held in registers (byte_perm); the sign
+// bit is placed separately.  Products E2M1 x E4M3 are exact in bf16.
+//   magnitude code:  0    1     2     3     4     5     6     7
+//   value:           0    0.5   1     1.5   2     3     4     6
+//   bf16:            0000 3F00  3F80  3FC0  4000  4040  4080  40C0
+__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, __nv_bfloat162 scale, uint32_t (&out)[4]) {
+  const uint32_t m = w & 0x77777777u;
+  const uint32_t lo_a = __byte_perm(0xC0800000u, 0xC0804000u, m);
+  const uint32_t hi_a = __byte_perm(0x3F3F3F00u, 0x40404040u, m);
+  const uint32_t lo_b = __byte_perm(0xC0800000u, 0xC0804000u, m >> 16);
+  const uint32_t hi_b = __byte_perm(0x3F3F3F00u, 0x40404040u, m >> 16);
+  uint32_t o[4];
+  o[0] = __byte_perm(lo_a, hi_a, 0x5140) | ((w << 12) & 0x8000u) | ((w << 24) & 0x80000000u);
+  o[1] = __byte_perm(lo_a, hi_a, 0x7362) | ((w << 4) & 0x8000u) | ((w << 16) & 0x80000000u);
+  o[2] = __byte_perm(lo_b, hi_b, 0x5140) | ((w >> 4) & 0x8000u) | ((w << 8) & 0x80000000u);
+  o[3] = __byte_perm(lo_b, hi_b, 0x7362) | ((w >> 12) & 0x8000u) | (w & 0x80000000u);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&o[j]);
+    x = __hmul2(x, scale);
+    out[j] = *reinterpret_cast<uint32_t*>(&x);
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

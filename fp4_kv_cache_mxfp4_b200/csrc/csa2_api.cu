@@ -44,37 +44,49 @@ cudaError_t set_smem_attrs(F* f, int dyn_bytes) {
   return cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
 }
 
-template <int QG, bool HSI>
+template <int QG, bool HSI, bool KF4>
 cudaError_t set_scan_attr_one() {
-  return set_smem_attrs(index_scan_kernel<QG, HSI>, kMaxDynSmem);
+  return set_smem_attrs(index_scan_kernel<QG, HSI, KF4>, kMaxDynSmem);
 }
-cudaError_t set_scan_attrs() {
+template <bool KF4>
+cudaError_t set_scan_attrs_k() {
   cudaError_t e = cudaSuccess;
-  cudaError_t r[8] = {set_scan_attr_one<1, false>(), set_scan_attr_one<1, true>(), set_scan_attr_one<2, false>(),
-                      set_scan_attr_one<2, true>(), set_scan_attr_one<4, false>(), set_scan_attr_one<4, true>(),
-                      set_scan_attr_one<8, false>(), set_scan_attr_one<8, true>()};
+  cudaError_t r[8] = {set_scan_attr_one<1, false, KF4>(), set_scan_attr_one<1, true, KF4>(),
+                      set_scan_attr_one<2, false, KF4>(), set_scan_attr_one<2, true, KF4>(),
+                      set_scan_attr_one<4, false, KF4>(), set_scan_attr_one<4, true, KF4>(),
+                      set_scan_attr_one<8, false, KF4>(), set_scan_attr_one<8, true, KF4>()};
   for (cudaError_t x : r) if (x != cudaSuccess) e = x;
   return e;
 }
+cudaError_t set_scan_attrs() {
+  const cudaError_t a = set_scan_attrs_k<false>(), b = set_scan_attrs_k<true>();
+  return a != cudaSuccess ? a : b;
+}
 inline int scan_qg(int qg) { return qg <= 1 ? 1 : qg <= 2 ? 2 : qg <= 4 ? 4 : 8; }
 
-template <int QG, bool HSI>
+template <int QG, bool HSI, bool KF4>
 cudaError_t launch_scan_t(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk, const CUtensorMap& tq,
                           const ScanParams& sp) {
-  return launch_ex(index_scan_kernel<QG, HSI>, dim3(grid), dim3(kScanThreads), smem, st, 0, tk, tq, sp);
+  return launch_ex(index_scan_kernel<QG, HSI, KF4>, dim3(grid), dim3(kScanThreads), smem, st, 0, tk, tq, sp);
 }
-cudaError_t launch_scan(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
-                        const CUtensorMap& tq, const ScanParams& sp) {
+template <bool KF4>
+cudaError_t launch_scan_k(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
+                          const CUtensorMap& tq, const ScanParams& sp) {
   switch (QG * 2 + (hsi ? 1 : 0)) {
-    case 2: return launch_scan_t<1, false>(grid, smem, st, tk, tq, sp);
-    case 3: return launch_scan_t<1, true>(grid, smem, st, tk, tq, sp);
-    case 4: return launch_scan_t<2, false>(grid, smem, st, tk, tq, sp);
-    case 5: return launch_scan_t<2, true>(grid, smem, st, tk, tq, sp);
-    case 8: return launch_scan_t<4, false>(grid, smem, st, tk, tq, sp);
-    case 9: return launch_scan_t<4, true>(grid, smem, st, tk, tq, sp);
-    case 16: return launch_scan_t<8, false>(grid, smem, st, tk, tq, sp);
-    default: return launch_scan_t<8, true>(grid, smem, st, tk, tq, sp);
+    case 2: return launch_scan_t<1, false, KF4>(grid, smem, st, tk, tq, sp);
+    case 3: return launch_scan_t<1, true, KF4>(grid, smem, st, tk, tq, sp);
+    case 4: return launch_scan_t<2, false, KF4>(grid, smem, st, tk, tq, sp);
+    case 5: return launch_scan_t<2, true, KF4>(grid, smem, st, tk, tq, sp);
+    case 8: return launch_scan_t<4, false, KF4>(grid, smem, st, tk, tq, sp);
+    case 9: return launch_scan_t<4, true, KF4>(grid, smem, st, tk, tq, sp);
+    case 16: return launch_scan_t<8, false, KF4>(grid, smem, st, tk, tq, sp);
+    default: return launch_scan_t<8, true, KF4>(grid, smem, st, tk, tq, sp);
   }
+}
+cudaError_t launch_scan(int QG, bool hsi, bool kf4, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
+                        const CUtensorMap& tq, const ScanParams& sp) {
+  return kf4 ? launch_scan_k<true>(QG, hsi, grid, smem, st, tk, tq, sp)
+             : launch_scan_k<false>(QG, hsi, grid, smem, st, tk, tq, sp);
 }
 
 // Largest top-K cluster this GPU can place: 16 (non-portable) when at least
@@ -125,7 +137,9 @@ csa2_status device_info(DeviceInfo** out) {
         set_smem_attrs(topk_select_kernel, static_cast<int>(topk_smem_bytes())) != cudaSuccess ||
         set_smem_attrs(sparse_attn_tc_kernel, static_cast<int>(kTcAttnSmem)) != cudaSuccess ||
         set_smem_attrs(sparse_attn_combine_kernel, 0) != cudaSuccess ||
-        set_smem_attrs(quantize_kv_fp4_kernel, 0) != cudaSuccess)
+        set_smem_attrs(quantize_kv_fp4_kernel, 0) != cudaSuccess ||
+        set_smem_attrs(quantize_window_fp8_kernel, 0) != cudaSuccess ||
+        set_smem_attrs(quantize_index_k_mxfp4_kernel, 0) != cudaSuccess)
       return CSA2_ERR_CUDA;
     d.topk_max_cluster = topk_cluster_limit();
     if (!g_encode) {
@@ -187,6 +201,8 @@ csa2_status validate_index(const csa2_index_args* a) {
   }
   if (hsi && !a->pool_out) return CSA2_ERR_ARG;
   if (a->mode == CSA2_REINDEX_POOL && !a->pool_in) return CSA2_ERR_ARG;
+  if (a->k_format != CSA2_FMT_BF16 && a->k_format != CSA2_FMT_MXFP4) return CSA2_ERR_ARG;
+  if (a->k_format == CSA2_FMT_MXFP4 && (a->N & 3)) return CSA2_ERR_SHAPE;   // 16-byte aligned raw tiles
   if (!aligned16(a->qI) || !aligned16(a->w) || !aligned16(a->kI) || !aligned16(a->n_vis) || !aligned16(a->idx) ||
       (a->scores && !aligned16(a->scores)) || (hsi && !aligned16(a->pool_out)) ||
       (a->mode == CSA2_REINDEX_POOL && !aligned16(a->pool_in)))
@@ -283,19 +299,32 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   while (cols < scan_acc_bufs(QG) * n_mma) cols <<= 1;
   sp.tmem_cols = cols;
   sp.early_q = early_q ? 1 : 0;
-  const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi);
+  const bool kf4 = a->k_format == CSA2_FMT_MXFP4;
+  int raw = 0;
+  if (kf4) {
+    // MXFP4 index-K: up to 8 raw tiles (8.5 KB each) in flight, beside at
+    // least two bf16 stages
+    sp.k4 = static_cast<const uint8_t*>(a->kI);
+    const int room = kMaxDynSmem - 1024 - static_cast<int>(scan_smem_layout(2, QG, P.hb, P.hsi, 0).total);
+    raw = std::min(8, room / (kRawStageBytes + 16));
+    if (raw < 2) return CSA2_ERR_SHAPE;
+  }
+  sp.raw_stages = raw;
+  const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi, raw);
   // three 32 KB stages per SM measured fastest (fewer bytes in flight per
   // stream keep DRAM pages open longer; 2, 4 and 6 stages were slower)
-  sp.stages = std::min(kScanStages, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / kStageBytes));
+  sp.stages = std::min(kScanStages, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / (kStageBytes + 16)));
   if (sp.stages < 2) return CSA2_ERR_SHAPE;
-  const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi);
+  const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi, raw);
   CUtensorMap tk, tq;
-  if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : kTileRows)) return CSA2_ERR_CUDA;
   if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, n_mma)) return CSA2_ERR_CUDA;
+  if (kf4) tk = tq;                                 // not read: index-K arrives by bulk copies
+  else if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : kTileRows))
+    return CSA2_ERR_CUDA;
 
   const unsigned grid = static_cast<unsigned>(sp.groups * sp.ctas_per_group);
   trace_pre(kKIndexScan, st);
-  const cudaError_t es = launch_scan(QG, P.hsi, grid, L.total + 1024, st, tk, tq, sp);
+  const cudaError_t es = launch_scan(QG, P.hsi, kf4, grid, L.total + 1024, st, tk, tq, sp);
   trace_post(st);
   if (es != cudaSuccess) return CSA2_ERR_CUDA;
 
@@ -345,10 +374,13 @@ csa2_status validate_attn(const csa2_attn_args* a) {
       a->W < 0 || a->W > CSA2_MAX_W ||
       a->K + a->W < 1 || a->N < 1 || a->swa_step < 0)
     return CSA2_ERR_SHAPE;
+  if (a->swa_format != CSA2_FMT_BF16 && a->swa_format != CSA2_FMT_FP8) return CSA2_ERR_ARG;
   if (!a->q || !a->out || (a->K > 0 && (!a->kv_fp4 || !a->idx)) || (a->W > 0 && !a->swa)) return CSA2_ERR_ARG;
+  if (a->W > 0 && a->swa_format == CSA2_FMT_FP8 && !a->swa_scale) return CSA2_ERR_ARG;
   if (a->W > 0 && static_cast<int64_t>(a->Q - 1) * a->swa_step + a->W > a->swa_rows) return CSA2_ERR_SHAPE;
   if (!aligned16(a->q) || !aligned16(a->out) || (a->kv_fp4 && !aligned16(a->kv_fp4)) || (a->idx && !aligned16(a->idx)) ||
-      (a->swa && !aligned16(a->swa)) || (a->lse && !aligned16(a->lse)))
+      (a->swa && !aligned16(a->swa)) || (a->lse && !aligned16(a->lse)) ||
+      (a->swa_scale && (reinterpret_cast<uintptr_t>(a->swa_scale) & 3)))
     return CSA2_ERR_ALIGN;
   return CSA2_OK;
 }
@@ -417,9 +449,12 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st, bool ea
   t.ml = (per_query || cluster) ? nullptr : ml;
   t.out = static_cast<__nv_bfloat16*>(a->out);
   t.lse = a->lse;
+  t.swa_fp8 = (a->W > 0 && a->swa_format == CSA2_FMT_FP8) ? 1 : 0;
+  t.swa8 = static_cast<const uint8_t*>(a->swa);
+  t.swa_scale = a->swa_scale;
   CUtensorMap tq, tw;
   if (!make_map_bf16_512(&tq, a->q, bq * 64, 64)) return CSA2_ERR_CUDA;
-  if (a->W > 0) {
+  if (a->W > 0 && !t.swa_fp8) {
     if (!make_map_bf16_512(&tw, a->swa, static_cast<uint64_t>(a->B) * a->swa_rows, kTcAttnKeys)) return CSA2_ERR_CUDA;
   } else {
     tw = tq;                                    // no window slices: never used
@@ -454,6 +489,7 @@ csa2_index_args layer_index_args(const csa2_group_args* g, const csa2_layer& L, 
   a.mode = L.mode; a.B = g->B; a.Q = g->Q; a.K = g->K; a.N = g->N;
   a.qI = L.qI; a.w = L.w; a.kI = g->kI; a.n_vis = g->n_vis;
   a.idx = L.idx; a.scores = L.scores;
+  a.k_format = g->index_k_format;
   a.hsi_blocks = (L.mode == CSA2_FULL || L.mode == CSA2_REINDEX_POOL) ? g->hsi_blocks : 0;
   a.hsi_block = g->hsi_block;
   a.pool_out = (L.mode == CSA2_FULL && g->hsi_blocks > 0) ? g->pool : nullptr;
@@ -468,6 +504,7 @@ csa2_attn_args layer_attn_args(const csa2_group_args* g, const csa2_layer& L, co
   a.q = L.q; a.kv_fp4 = g->kv_fp4; a.idx = idx; a.swa = L.swa;
   a.swa_rows = g->swa_rows; a.swa_step = g->swa_step; a.scale = g->scale;
   a.out = L.out; a.lse = L.lse;
+  a.swa_format = g->swa_format; a.swa_scale = L.swa_scale;
   return a;
 }
 
@@ -643,6 +680,36 @@ csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x, void* k
              ? CSA2_OK : CSA2_ERR_CUDA;
 }
 
+csa2_status csa2_quantize_window_fp8(const void* x, int64_t n, int64_t ld_x, void* codes, float* scales,
+                                     const int64_t* dst_rows, int64_t row_offset, void* stream) {
+  if (n < 0 || ld_x < 512 || (ld_x & 7) || row_offset < 0) return CSA2_ERR_SHAPE;
+  if (n == 0) return CSA2_OK;
+  if (!x || !codes || !scales) return CSA2_ERR_ARG;
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3) ||
+      (dst_rows && (reinterpret_cast<uintptr_t>(dst_rows) & 7)))
+    return CSA2_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  const csa2_status s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  return launch_quantize_window(x, n, ld_x, codes, scales, dst_rows, row_offset, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
+csa2_status csa2_quantize_index_k_mxfp4(const void* x, int64_t n, int64_t ld_x, void* out, const int64_t* dst_rows,
+                                        int64_t row_offset, void* stream) {
+  if (n < 0 || ld_x < 128 || (ld_x & 3) || row_offset < 0) return CSA2_ERR_SHAPE;
+  if (n == 0) return CSA2_OK;
+  if (!x || !out) return CSA2_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 7) || (reinterpret_cast<uintptr_t>(out) & 3) ||
+      (dst_rows && (reinterpret_cast<uintptr_t>(dst_rows) & 7)))
+    return CSA2_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  const csa2_status s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  return launch_quantize_index_k(x, n, ld_x, out, dst_rows, row_offset, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
 csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws, size_t ws_bytes, void* stream) {
   csa2_status s = validate_index(a);
   if (s != CSA2_OK) return s;
@@ -768,7 +835,7 @@ const char* csa2_status_string(int32_t s) {
   }
 }
 
-int32_t csa2_version(void) { return 101; }
+int32_t csa2_version(void) { return 103; }
 
 csa2_status csa2_trace_begin(int32_t max_launches) {
   if (max_launches < 1 || max_launches > (1 << 20)) return CSA2_ERR_SHAPE;
@@ -822,6 +889,8 @@ const char* csa2_kernel_name(int32_t kernel) {
     case kKTopk: return "topk_select_kernel";
     case kKAttnSlice: return "sparse_attn_tc_kernel";
     case kKAttnCombine: return "sparse_attn_combine_kernel";
+    case kKQuantizeWindow: return "quantize_window_fp8_kernel";
+    case kKQuantizeIndexK: return "quantize_index_k_mxfp4_kernel";
     default: return "unknown";
   }
 }

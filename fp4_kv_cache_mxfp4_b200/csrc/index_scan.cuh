@@ -21,6 +21,14 @@
 // Pool mode (Reindex restricted to the HSI pool) gathers the tile as 16
 // blocks of 8 contiguous index-K rows with one 1 KB TMA box per block half.
 //
+// MXFP4 index-K (68-byte entries: 64 bytes of E2M1 nibbles, 4 E8M0 block
+// scales; "DeepSeek V4.1-Flash 技术报告深度解析" §3.4 FP4 indexer K): the
+// producer streams raw tiles (128 entries, 8.5 KB, one bulk copy; pool mode
+// one 544-byte copy per block) into a ring of its own, and the epilogue
+// warps, one tile ahead of the MMA, expand each tile into the bf16 stage
+// (E2M1 x 2^e is exact in bf16) before handling their accumulators.  The
+// MMA and the score arithmetic are those of the bf16 path.
+//
 // HBM roofline: 256 B of index-K per entry per (row, layer) + 4 B of score
 // write; index-Q, w and histograms are negligible.
 #pragma once
@@ -34,6 +42,7 @@ constexpr int kScanThreads = 64 + kScanEpiThreads;
 constexpr int kTileRows = 128;                     // entries per MMA tile (M)
 constexpr int kStageBytes = kTileRows * 128 * 2;   // 32 KB: two 128x64 swizzled boxes
 constexpr int kAccBufs = 4;                        // TMEM accumulator slots (barriers)
+constexpr int kRawStageBytes = kTileRows * 68;     // MXFP4 index-K: one raw tile of 68-byte entries
 
 // accumulators in flight: as many as fit the 512 TMEM columns, at most 4
 __host__ __device__ constexpr int scan_acc_bufs(int QG) { return 32 * QG * 4 <= 512 ? 4 : 2; }
@@ -64,28 +73,32 @@ struct ScanParams {
   uint32_t tmem_cols;
   int early_q;            // 1: index-Q and w are complete at launch (load them before waiting on
                           // the predecessor); 0: they may be the predecessor's results
+  const uint8_t* k4;      // MXFP4 index-K: [B*N][68] entries (N a multiple of 4)
+  int raw_stages;         // MXFP4 index-K: raw tiles in flight
 };
 
 struct ScanSmem {
   // offsets inside the dynamic shared memory block
-  uint32_t stage0, qi0, w0, hist0, bhist0, bar0, total;
+  uint32_t stage0, raw0, qi0, w0, hist0, bhist0, bar0, total;
 };
 
-__host__ __device__ inline ScanSmem scan_smem_layout(int stages, int QG, int hb, int hsi) {
+// raw_stages: MXFP4 index-K raw tiles (0 for bf16 index-K)
+__host__ __device__ inline ScanSmem scan_smem_layout(int stages, int QG, int hb, int hsi, int raw_stages = 0) {
   ScanSmem L;
   uint32_t off = 0;
   L.stage0 = off; off += stages * kStageBytes;
+  L.raw0 = off;   off += raw_stages * kRawStageBytes;
   L.qi0 = off;    off += 2 * (32 * QG) * 128;          // two 64-dim halves of [32*QG x 64] bf16
   L.w0 = off;     off += QG * 32 * 4;
   L.hist0 = off;  off += QG * (1u << hb) * 4;
   L.bhist0 = off; off += hsi ? QG * (1u << hb) * 4 : 0;
   off = (off + 15) & ~15u;
-  L.bar0 = off;   off += (2 * stages + 2 * kAccBufs + 2) * 8 + 16 + 64;   // barriers, TMEM slot, flags, scratch
+  L.bar0 = off;   off += (2 * stages + 2 * kAccBufs + 2 * raw_stages + 2) * 8 + 16 + 64;   // barriers, TMEM slot, flags
   L.total = off;
   return L;
 }
 
-template <int QG, bool HSI>
+template <int QG, bool HSI, bool KF4>
 __global__ void __launch_bounds__(kScanThreads, 1)
 index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_q,
@@ -93,12 +106,15 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the swizzle atoms need 1024-byte alignment of every operand tile
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const ScanSmem L = scan_smem_layout(p.stages, QG, p.hb, HSI);
+  const int R = KF4 ? p.raw_stages : 0;
+  const ScanSmem L = scan_smem_layout(p.stages, QG, p.hb, HSI, R);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L.bar0);
   uint64_t* empty_bar = full_bar + p.stages;
   uint64_t* tfull_bar = empty_bar + p.stages;
   uint64_t* tempty_bar = tfull_bar + kAccBufs;
-  uint64_t* q_bar = tempty_bar + kAccBufs;
+  uint64_t* rfull_bar = tempty_bar + kAccBufs;     // MXFP4: raw tile landed
+  uint64_t* rempty_bar = rfull_bar + R;            // MXFP4: raw tile expanded
+  uint64_t* q_bar = rempty_bar + R;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* w_s = reinterpret_cast<float*>(smem + L.w0);
@@ -116,13 +132,16 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int nbins = 1 << p.hb;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    // with MXFP4 index-K a bf16 stage is full once every epilogue thread has
+    // written its part of the tile
+    for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], KF4 ? kScanEpiThreads : 1); mbar_init(&empty_bar[s], 1); }
+    for (int r = 0; r < R; ++r) { mbar_init(&rfull_bar[r], 1); mbar_init(&rempty_bar[r], kScanEpiThreads); }
     for (int a = 0; a < scan_acc_bufs(QG); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 128); }
     mbar_init(q_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmap_k); tma_prefetch_desc(&tmap_q); }
+  if (warp == 0 && lane == 0) { if (!KF4) tma_prefetch_desc(&tmap_k); tma_prefetch_desc(&tmap_q); }
   if (warp == 1) { tmem_alloc(tmem_slot, p.tmem_cols); tmem_relinquish(); }
   for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) hist_s[i] = 0;
   if (HSI) for (int i = threadIdx.x; i < QG * nbins; i += blockDim.x) bhist_s[i] = 0;
@@ -174,7 +193,36 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
       // first ring of index-K tiles is in flight and the predecessor is done
       const bool q_late = !p.early_q && !p.pool_mode;
       if (!q_late) load_q();
-      for (int i = 0; i < ntiles; ++i) {
+      if constexpr (KF4) {
+        // raw MXFP4 tiles: one bulk copy per tile (its valid rows), or one
+        // per pool block of 8 entries
+        for (int i = 0; i < ntiles; ++i) {
+          const int r = i % R;
+          if (q_late && i == min(R, ntiles)) { pdl_wait(); load_q(); }
+          if (!mbar_wait(&rempty_bar[r], ((i / R) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag)) break;
+          uint8_t* dst = smem + L.raw0 + r * kRawStageBytes;
+          const int tile = tile_lo + i;
+          if (!p.pool_mode) {
+            const int64_t row0 = static_cast<int64_t>(tile) * kTileRows;
+            const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(kTileRows), p.N - row0));
+            mbar_arrive_expect_tx(&rfull_bar[r], rows * 68u);
+            bulk_load(dst, p.k4 + (static_cast<int64_t>(b) * p.N + row0) * 68, rows * 68u, &rfull_bar[r]);
+          } else {
+            const int32_t* pool = p.pool + static_cast<int64_t>(bq0) * p.pool_blocks;
+            mbar_arrive_expect_tx(&rfull_bar[r], (kTileRows / 8) * 544u);
+#pragma unroll 1
+            for (int j = 0; j < kTileRows / 8; ++j) {
+              const int slot = tile * (kTileRows / 8) + j;
+              int blk = (slot < p.pool_blocks) ? pool[slot] : -1;
+              if (blk < 0) blk = 0;                  // padding slot: load any block, scores masked
+              bulk_load(dst + j * 544, p.k4 + (static_cast<int64_t>(b) * p.N + static_cast<int64_t>(blk) * 8) * 68,
+                        544u, &rfull_bar[r]);
+            }
+          }
+        }
+        if (q_late && ntiles <= R) { pdl_wait(); load_q(); }
+      }
+      for (int i = 0; !KF4 && i < ntiles; ++i) {
         const int s = i % p.stages;
         const uint32_t ph = (i / p.stages) & 1;
         if (q_late && i == min(p.stages, ntiles)) { pdl_wait(); load_q(); }
@@ -199,7 +247,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
         }
       }
-      if (q_late && ntiles <= p.stages) { pdl_wait(); load_q(); }
+      if (!KF4 && q_late && ntiles <= p.stages) { pdl_wait(); load_q(); }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -245,11 +293,12 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     float wr[WREG];
 #pragma unroll
     for (int h = 0; h < WREG; ++h) wr[h] = (QG <= 2) ? w_s[h] : 0.0f;
-    for (int i = set; i < ntiles; i += 2) {
+    // one tile's accumulator -> scores, histograms (false: a wait gave up)
+    auto epi_tile = [&](int i) -> bool {
       const int a = i % ACC;
       // tcgen05.ld is warp-collective: leave the loop as a whole warp
       const bool ok = mbar_wait(&tfull_bar[a], (i / ACC) & 1, kErrWaitTmemFull, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!__all_sync(0xffffffffu, ok)) return false;
       tc_fence_after();
       const int tile = tile_lo + i;
       const int64_t e = static_cast<int64_t>(tile) * kTileRows + row;   // score slot
@@ -314,6 +363,48 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
             warp_hist_add(bhist_s + q * nbins, okey(m) >> (32 - p.hb), writer && m != -INFINITY);
           }
         }
+      }
+      return true;
+    };
+    if constexpr (!KF4) {
+      for (int i = set; i < ntiles; i += 2)
+        if (!epi_tile(i)) break;
+    } else {
+      // expand raw tile t into its bf16 stage (every epilogue thread: half a
+      // row), then handle accumulator t - 1 when it belongs to this set
+      const int et = threadIdx.x - 64;
+      const int crow = et >> 1, chalf = et & 1;
+      for (int t = 0; t <= ntiles; ++t) {
+        if (t < ntiles) {
+          const int r = t % R, st = t % p.stages;
+          bool okc = mbar_wait(&rfull_bar[r], (t / R) & 1, kErrWaitTmaFull, abort_flag);
+          okc = okc && mbar_wait(&empty_bar[st], ((t / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag);
+          if (!__all_sync(0xffffffffu, okc)) break;
+          const uint8_t* src = smem + L.raw0 + r * kRawStageBytes + crow * 68;
+          uint32_t wv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) wv[k] = *reinterpret_cast<const uint32_t*>(src + 32 * chalf + 4 * k);
+          const uint32_t c0 = src[64 + 2 * chalf], c1 = src[65 + 2 * chalf];
+          // 2^(code - 127) as bf16: exponent field = code; code 0 is 2^-127,
+          // the subnormal 0x0040
+          const uint32_t b0 = c0 ? (c0 << 7) : 0x40u, b1 = c1 ? (c1 << 7) : 0x40u;
+          const uint32_t p0 = b0 | (b0 << 16), p1 = b1 | (b1 << 16);
+          const __nv_bfloat162 S0 = *reinterpret_cast<const __nv_bfloat162*>(&p0);
+          const __nv_bfloat162 S1 = *reinterpret_cast<const __nv_bfloat162*>(&p1);
+          uint8_t* box = smem + L.stage0 + st * kStageBytes + chalf * (kStageBytes / 2);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            uint32_t o[4];
+            e2m1x8_to_bf16(wv[k], k < 4 ? S0 : S1, o);       // channels 64 half + 8k .. + 7
+            *reinterpret_cast<uint4*>(box + sw128_off(crow, k)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive(&full_bar[st]);
+          mbar_arrive(&rempty_bar[r]);
+        }
+        const int i = t - 1;
+        if (i >= 0 && (i & 1) == set)
+          if (!epi_tile(i)) break;
       }
     }
     // flush the CTA's histograms into the global ones

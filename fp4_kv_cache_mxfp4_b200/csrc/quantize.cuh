@@ -103,4 +103,131 @@ inline cudaError_t launch_quantize(const void* x, int64_t n, int64_t ld_x, void*
   return e;
 }
 
+// ---------------------------------------------------------------------------
+// FP8 window rows ("DeepSeek V4.1-Flash 技术报告深度解析" §3.4: the SWA KV cache
+// stays FP8): one E4M3 code per channel and one fp32 scale per 512-channel
+// row, s = amax / 448, code = E4M3(x / s) (round to nearest even,
+// saturating; a zero row gives signed zeros).  One warp per row, 16
+// channels per lane; the warp reduces amax, then writes its 512 codes with
+// one coalesced 16-byte store per lane.
+// HBM roofline: 1024 B read + 516 B written per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+quantize_window_fp8_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t ld_x,
+                           uint8_t* __restrict__ codes, float* __restrict__ scales,
+                           const int64_t* __restrict__ dst_rows, int64_t row_offset) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (row >= n) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x + row * ld_x + lane * 16);
+  uint4 raw[2];
+  raw[0] = __ldg(src);
+  raw[1] = __ldg(src + 1);
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(raw);
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 f = __bfloat1622float2(h2[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = __fdiv_rn(amax, 448.0f);
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = v[4 * k + j];
+      // a zero scale keeps the sign of x: cvt of a signed zero keeps it
+      const float y = (s != 0.0f) ? __fdiv_rn(a, s) : copysignf(0.0f, a);
+      word |= e4m3_rn_sat(y) << (8 * j);
+    }
+    w[k] = word;
+  }
+  const int64_t dst = dst_rows ? dst_rows[row] : row_offset + row;
+  *reinterpret_cast<uint4*>(codes + dst * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  if (lane == 0) scales[dst] = s;
+}
+
+inline cudaError_t launch_quantize_window(const void* x, int64_t n, int64_t ld_x, void* codes, float* scales,
+                                          const int64_t* dst_rows, int64_t row_offset, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int warps = 8;
+  const int64_t blocks = (n + warps - 1) / warps;
+  trace_pre(kKQuantizeWindow, st);
+  const cudaError_t e = launch_ex(quantize_window_fp8_kernel, dim3(static_cast<unsigned>(blocks)), dim3(warps * 32), 0,
+                                  st, 0, static_cast<const __nv_bfloat16*>(x), n, ld_x, static_cast<uint8_t*>(codes),
+                                  scales, dst_rows, row_offset);
+  trace_post(st);
+  return e;
+}
+
+// ---------------------------------------------------------------------------
+// MXFP4 index-K entries ("DeepSeek V4.1-Flash 技术报告深度解析" §3.4: FP4
+// indexer Q/K in the OCP MXFP4 format): per block of 32 channels a shared
+// scale 2^e, e = floor(log2(amax)) - 2 clamped to [-127, 127] (-127 for an
+// all-zero block), codes E2M1(x / 2^e) (round to nearest even, saturate at
+// 6, sign kept); entry = 64 nibble bytes (channel 2i low nibble of byte i)
+// + 4 scale bytes e + 127 = 68 B.  One warp per entry, 4 channels per lane,
+// 8 lanes per block.
+// HBM roofline: 256 B read + 68 B written per entry.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+quantize_index_k_mxfp4_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t ld_x,
+                              uint8_t* __restrict__ out, const int64_t* __restrict__ dst_rows,
+                              int64_t row_offset) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (row >= n) return;
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(x + row * ld_x + lane * 4));
+  const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  const float v[4] = {f0.x, f0.y, f1.x, f1.y};
+  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int e = -127;
+  if (amax > 0.0f) {
+    int E;
+    frexpf(amax, &E);                                  // amax = m 2^E, m in [0.5, 1)
+    e = max(-127, min(127, E - 1 - 2));
+  }
+  uint32_t nib = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float a = ldexpf(v[2 * i], -e), b = ldexpf(v[2 * i + 1], -e);   // exact: powers of two
+    uint32_t byte = e2m1x2_rn_sat(fabsf(a), fabsf(b));
+    byte |= (__float_as_uint(a) >> 31) << 3;
+    byte |= (__float_as_uint(b) >> 31) << 7;
+    nib |= byte << (8 * i);
+  }
+  const int64_t dst = dst_rows ? dst_rows[row] : row_offset + row;
+  uint8_t* entry = out + dst * 68;
+  *reinterpret_cast<uint16_t*>(entry + 2 * lane) = static_cast<uint16_t>(nib);
+  if ((lane & 7) == 0) entry[64 + (lane >> 3)] = static_cast<uint8_t>(e + 127);
+}
+
+inline cudaError_t launch_quantize_index_k(const void* x, int64_t n, int64_t ld_x, void* out, const int64_t* dst_rows,
+                                           int64_t row_offset, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int warps = 8;
+  const int64_t blocks = (n + warps - 1) / warps;
+  trace_pre(kKQuantizeIndexK, st);
+  const cudaError_t e = launch_ex(quantize_index_k_mxfp4_kernel, dim3(static_cast<unsigned>(blocks)), dim3(warps * 32),
+                                  0, st, 0, static_cast<const __nv_bfloat16*>(x), n, ld_x, static_cast<uint8_t*>(out),
+                                  dst_rows, row_offset);
+  trace_post(st);
+  return e;
+}
+
 }  // namespace csa2

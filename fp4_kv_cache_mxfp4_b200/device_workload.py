@@ -28,8 +28,9 @@ def with_seed_shift(wl, shift):
 
 
 def _stage_cache(cw, csa2, d):
-    """FP4 main KV of every row but the step's new entries, index-K, the
-    new entries and their absolute destination rows."""
+    """FP4 main KV of every row but the step's new entries, index-K (bf16,
+    or quantised on the device to MXFP4 entries), the new entries and their
+    absolute destination rows."""
     B, N = cw.B, cw.N
     kv = torch.empty(B, N, 288, dtype=torch.uint8, device=d)
     for b in range(B):
@@ -37,7 +38,12 @@ def _stage_cache(cw, csa2, d):
             n = min(workloads.KV_CHUNK, N - cw.n_new - r0)
             x = workloads.main_kv_rows(cw, b, r0, n).to(d)
             csa2.csa2_quantize_kv_fp4(x, kv[b], row_offset=r0)
-    kI = torch.stack([workloads.index_k(cw, b) for b in range(B)]).to(d)
+    if cw.index_k_format == csa2.FMT_MXFP4:
+        kI = torch.empty(B, N, 68, dtype=torch.uint8, device=d)
+        for b in range(B):
+            csa2.csa2_quantize_index_k_mxfp4(workloads.index_k(cw, b).to(d), kI[b])
+    else:
+        kI = torch.stack([workloads.index_k(cw, b) for b in range(B)]).to(d)
     new = torch.cat([workloads.main_kv_rows(cw, b, N - cw.n_new, cw.n_new) for b in range(B)]).to(d)
     new_rows = torch.tensor([b * N + r for b in range(B) for r in cw.new_rows], dtype=torch.int64, device=d)
     return dict(kv=kv, kI=kI, new=new, new_rows=new_rows)
@@ -52,8 +58,15 @@ def make_device_workload(wl, csa2, seed_shift=0):
     layers = []
     for l, mode in enumerate(wl.modes):
         li = workloads.layer_inputs(wl, l)
-        layers.append(dict(mode=mode, qI=li["qI"].to(d), w=li["w"].to(d), q=li["q"].to(d), swa=li["swa"].to(d),
-                           out=torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=d),
+        swa, swa_scale = li["swa"].to(d), None
+        if wl.window_format == csa2.FMT_FP8:
+            codes = torch.empty(B, wl.swa_rows, 512, dtype=torch.uint8, device=d)
+            swa_scale = torch.empty(B, wl.swa_rows, device=d)
+            for b in range(B):
+                csa2.csa2_quantize_window_fp8(swa[b], codes[b], swa_scale[b])
+            swa = codes
+        layers.append(dict(mode=mode, qI=li["qI"].to(d), w=li["w"].to(d), q=li["q"].to(d), swa=swa,
+                           swa_scale=swa_scale, out=torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=d),
                            lse=torch.empty(B, Q, 64, device=d),
                            idx=torch.empty(B, Q, K, dtype=torch.int32, device=d) if mode != workloads.REUSE else None))
     n_vis = workloads.n_vis_tensor(wl).to(d)
@@ -68,7 +81,7 @@ def make_device_workload(wl, csa2, seed_shift=0):
         ga = csa2.group_args(B, Q, K, wl.W, wl.N, n_vis, C["kI"], C["kv"], Ls,
                              kv_new=C["new"] if quantise else None, new_rows=C["new_rows"] if quantise else None,
                              swa_rows=wl.swa_rows, swa_step=wl.swa_step, hsi_blocks=wl.hsi_blocks,
-                             hsi_block=wl.hsi_block, pool=own_pool, pool_in=pool)
+                             hsi_block=wl.hsi_block, pool=own_pool, pool_in=pool, swa_format=wl.window_format)
         groups.append(dict(g=ga, cache=C, layers=Ls, pool=own_pool, pool_in=pool))
         if own_pool is not None:
             pool = own_pool

@@ -52,6 +52,8 @@ class Workload:
     groups: List[int] = field(default_factory=list)  # layers per sharing group (default: one group)
     cache_per_group: bool = False  # each group has its own main KV and index-K (encoder), else one
                                    # cache for all groups (decoder)
+    index_k_format: int = 0        # 0: bf16 index-K; 2: 68-byte MXFP4 entries
+    window_format: int = 0         # 0: bf16 window rows; 1: E4M3 codes + one f32 scale per row
 
     def __post_init__(self):
         if not self.groups:
@@ -115,6 +117,10 @@ WORKLOADS = {
                 prefill=True, swa_step=1,
                 desc="The encoder's 18 CSA2 layers as 3 groups (Full + 5 Reuse), each group with its own "
                      "cache of 32,768 entries (64K tokens at r=2), 5 query positions per row, batch 4"),
+    8: Workload("group4_decode_ctx128k_b4_mxfp4ik_fp8win", 2, B=4, Q=1, N=131072, r=1,
+                modes=[FULL, REINDEX, REINDEX, REUSE], n_new=1, index_k_format=2, window_format=1,
+                desc="The decoder group of workload 2 (same draws) with the pages' other precisions: index-K "
+                     "as 68-byte MXFP4 entries and FP8 window rows"),
     5: Workload("prefill_t1024_prefix64k_r2", 5, B=1, Q=1024, N=32768 + 512, r=2, modes=[FULL],
                 n_new=512, prefill=True, swa_step=1,
                 desc="Prefill chunk of 1024 tokens after a 64K-token prefix at r=2, causal: the prefill "

@@ -73,6 +73,12 @@ typedef enum csa2_status {
     CSA2_ERR_ARCH      = 7   /* current device is not sm_100                 */
 } csa2_status;
 
+/* Storage formats of the window rows (attention) and of index-K. */
+#define CSA2_FMT_BF16     0     /* bf16 values                                  */
+#define CSA2_FMT_FP8      1     /* window rows: E4M3 codes + one f32 scale per row ([eogee] §3.4) */
+#define CSA2_FMT_MXFP4    2     /* index-K: 68-byte OCP MXFP4 entries ([eogee] §3.4) */
+#define CSA2_INDEX_K_MXFP4_BYTES 68   /* 64 B of E2M1 nibbles + 4 E8M0 scales        */
+
 /* Static layer modes, [eogee] §3.2 and §3.3. */
 typedef enum csa2_mode {
     CSA2_FULL         = 0,  /* score every visible entry                       */
@@ -109,6 +115,49 @@ csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x,
                                  int64_t row_offset, void* stream);
 
 /* ------------------------------------------------------------------------
+ * csa2_quantize_window_fp8 -- [eogee] §3.4: the quantisation-sensitive SWA
+ * KV cache stays in FP8.  The page names the precision only; this library's
+ * format is one E4M3 code per channel and one f32 scale per 512-channel row:
+ *     s = fp32(amax / 448)                (round to nearest even)
+ *     code_i = E4M3(fp32(x_i / s))        (round to nearest even, saturate
+ *                                          448; sign kept; s == 0 gives
+ *                                          signed zeros)
+ * Dequantised value = E4M3(code) * s; a row costs 516 B against 1024 B of bf16.
+ *
+ *   x         bf16 [n][ld_x] rows (ld_x >= 512, a multiple of 8)
+ *   codes     u8 [rows][512] E4M3 codes
+ *   scales    f32 [rows]
+ *   dst_rows / row_offset  as in csa2_quantize_kv_fp4
+ * Errors: ARG, SHAPE, ALIGN (codes 16-byte, scales 4-byte aligned), CUDA.
+ * ---------------------------------------------------------------------- */
+csa2_status csa2_quantize_window_fp8(const void* x, int64_t n, int64_t ld_x,
+                                     void* codes, float* scales,
+                                     const int64_t* dst_rows, int64_t row_offset,
+                                     void* stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_quantize_index_k_mxfp4 -- [eogee] §3.4: the indexer's Q/K were
+ * already trained with FP4 quantisation, in the OCP MXFP4 family the page
+ * names.  Index-K entries of 128 channels become 68 bytes, the size that
+ * closes the pages' 890 B/token accounting ([ainewsway] "KV 快取為何成為
+ * 瓶頸": 3 encoder caches at r=2 and one decoder cache, 288 B main-KV and
+ * 68 B index-K entries): per block of 32 channels
+ *     e = floor(log2(amax)) - 2   (clamped to [-127, 127]; -127 for a zero block)
+ *     q_i = E2M1(x_i / 2^e)       (round to nearest even, saturate 6, sign kept)
+ * Entry: byte i (0..63) holds channel 2i in its low nibble and 2i+1 in its
+ * high nibble; byte 64+k holds e + 127 for channels 32k..32k+31.
+ * Dequantised value E2M1(q) * 2^e, exact in bf16.
+ *
+ *   x       bf16 [n][ld_x] (ld_x >= 128, a multiple of 4; 8-byte aligned)
+ *   out     u8 entries of 68 bytes (4-byte aligned)
+ *   dst_rows / row_offset  as in csa2_quantize_kv_fp4
+ * Errors: ARG, SHAPE, ALIGN, CUDA.
+ * ---------------------------------------------------------------------- */
+csa2_status csa2_quantize_index_k_mxfp4(const void* x, int64_t n, int64_t ld_x,
+                                        void* out, const int64_t* dst_rows,
+                                        int64_t row_offset, void* stream);
+
+/* ------------------------------------------------------------------------
  * csa2_index_score_topk -- [eogee] §3.2 lightweight indexer + top-K,
  * §3.3 Hierarchical Sparse Indexer.
  *
@@ -128,6 +177,11 @@ csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x,
  *   block ids per query, ascending, -1 padding ignored); positions at or
  *   beyond n_vis do not score.  The selected entries come out in pool order
  *   (ascending positions for an ascending pool).
+ *
+ * k_format CSA2_FMT_MXFP4: kI holds 68-byte MXFP4 entries [B][N][68]
+ *   (csa2_quantize_index_k_mxfp4; N a multiple of 4) and the scores use the
+ *   dequantised index-K, E2M1 x 2^e, which bf16 holds exactly; index-Q stays
+ *   bf16.
  * ---------------------------------------------------------------------- */
 typedef struct csa2_index_args {
     int32_t        mode;        /* CSA2_FULL, CSA2_REINDEX or CSA2_REINDEX_POOL  */
@@ -145,6 +199,7 @@ typedef struct csa2_index_args {
     int32_t        hsi_block;   /* positions per block (CSA2_HSI_BLOCK)          */
     int32_t*       pool_out;    /* FULL with hsi_blocks > 0: out int32 [B][Q][hsi_blocks] */
     const int32_t* pool_in;     /* REINDEX_POOL: in int32 [B][Q][hsi_blocks]     */
+    int32_t        k_format;    /* CSA2_FMT_BF16 or CSA2_FMT_MXFP4               */
 } csa2_index_args;
 
 csa2_status csa2_index_score_topk(const csa2_index_args* a, void* ws,
@@ -201,7 +256,8 @@ size_t csa2_noalloc_scratch_bytes(void);
  * A query with no key at all gets out = 0 and lse = -inf.
  *
  * idx entries must be -1 or in [0, N); the window rows read must lie inside
- * [0, swa_rows).
+ * [0, swa_rows).  With swa_format CSA2_FMT_FP8 a window key is the
+ * dequantised row E4M3(code) * s (csa2_quantize_window_fp8).
  *
  * With fewer than 128 queries per call (B*Q) the keys of a query are split
  * into 128-key slices over several CTAs: up to 8 slices (K + W <= 1024)
@@ -226,6 +282,9 @@ typedef struct csa2_attn_args {
     float          scale;       /* logit scale; <= 0 means 1/sqrt(512)           */
     void*          out;         /* out bf16 [B][Q][64][512]                      */
     float*         lse;         /* optional out f32 [B][Q][64]                   */
+    int32_t        swa_format;  /* CSA2_FMT_BF16 (swa is bf16) or CSA2_FMT_FP8   */
+    const float*   swa_scale;   /* CSA2_FMT_FP8: f32 [B][swa_rows]; swa is then
+                                   u8 [B][swa_rows][512] E4M3 codes              */
 } csa2_attn_args;
 
 csa2_status csa2_sparse_attn(const csa2_attn_args* a, void* ws,
@@ -271,6 +330,7 @@ typedef struct csa2_layer {
     float*         lse;         /* optional out f32 [B][Q][64]                   */
     int32_t*       idx;         /* indexing modes: out int32 [B][Q][K]           */
     float*         scores;      /* optional out f32 [B][Q][K]                    */
+    const float*   swa_scale;   /* group swa_format CSA2_FMT_FP8: f32 [B][swa_rows] */
 } csa2_layer;
 
 typedef struct csa2_group_args {
@@ -292,6 +352,8 @@ typedef struct csa2_group_args {
                                    an earlier call, read by REINDEX_POOL layers
                                    that come before any FULL layer of this call */
     int32_t          flags;     /* CSA2_GROUP_* bits                             */
+    int32_t          swa_format;/* the layers' window rows: CSA2_FMT_BF16 or _FP8 */
+    int32_t          index_k_format; /* kI: CSA2_FMT_BF16 or CSA2_FMT_MXFP4      */
 } csa2_group_args;
 
 #define CSA2_GROUP_INPUTS_READY 1
@@ -371,6 +433,8 @@ int32_t csa2_version(void);
 #define CSA2_KERNEL_TOPK         2
 #define CSA2_KERNEL_ATTN_SLICE   3
 #define CSA2_KERNEL_ATTN_COMBINE 4
+#define CSA2_KERNEL_QUANTIZE_WINDOW 5
+#define CSA2_KERNEL_QUANTIZE_INDEX_K 6
 csa2_status csa2_trace_begin(int32_t max_launches);
 csa2_status csa2_trace_stop(void);
 csa2_status csa2_trace_end(void);

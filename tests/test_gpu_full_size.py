@@ -16,7 +16,7 @@ import torch
 
 from fp4_kv_cache_mxfp4_b200 import csa2, workloads
 from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload, run_step
-from oracle import attention, fp4, indexer
+from oracle import attention, fp4, fp8, indexer, mxfp4
 from parity import check_attention, check_topk, f32
 
 pytestmark = pytest.mark.gpu
@@ -42,7 +42,24 @@ def _attn_oracle(kv_host_b, sel, q, win):
     return attention.sparse_mqa(q, deq, local, win)
 
 
-@pytest.mark.parametrize("w", [1, 2, 3, 4, 6, 7], ids=lambda w: workloads.WORKLOADS[w].name)
+def _index_k_for_oracle(wl, cw, b):
+    """The index-K the scores are defined on: the bf16 draws, or their MXFP4
+    entries dequantised (the pages' FP4 index-K)."""
+    k = f32(workloads.index_k(cw, b))
+    if wl.index_k_format == 2:
+        return mxfp4.dequantize_index_k_mxfp4(mxfp4.quantize_index_k_mxfp4(k))
+    return k
+
+
+def _window_for_oracle(wl, swa_b):
+    """A layer's window rows of one batch row as the attention sees them."""
+    x = f32(swa_b)
+    if wl.window_format == 1:
+        return fp8.dequantize_window_fp8(*fp8.quantize_window_fp8(x))
+    return x
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 4, 6, 7, 8], ids=lambda w: workloads.WORKLOADS[w].name)
 def test_full_size_sampled(w):
     """One step of a full-size workload (a stack of groups for 6 and 7)
     through the library call the bench times."""
@@ -69,6 +86,15 @@ def test_full_size_sampled(w):
                 np.testing.assert_array_equal(got, fp4.quantize_kv_fp4(f32(workloads.main_kv_rows(cw, b, r, 1)))[0],
                                               err_msg=f"entry {r} of cache {c} row {b}")
 
+    # MXFP4 index-K entries: 64 sampled rows per cache row, bit-exact
+    if wl.index_k_format == 2:
+        for c in range(n_caches):
+            cw = wl.cache_of_group(c)
+            for b in range(B):
+                rows = rng.integers(0, N, 64)
+                want = mxfp4.quantize_index_k_mxfp4(f32(workloads.index_k(cw, b))[rows])
+                np.testing.assert_array_equal(T["caches"][c]["kI"][b][torch.as_tensor(rows, device="cuda")].cpu().numpy(), want)
+
     samples = _samples(wl)
     kv_host = {(c, b): T["caches"][c]["kv"][b].cpu().numpy() for c in range(n_caches) for b in range(B)}
     n_vis = np.asarray(wl.n_vis)
@@ -87,7 +113,8 @@ def test_full_size_sampled(w):
             if mode != workloads.REUSE:
                 last_idx = L["idx"].cpu().numpy()
             for b in range(B):
-                kI = f32(workloads.index_k(cw, b)) if mode != workloads.REUSE else None
+                kI = _index_k_for_oracle(wl, cw, b) if mode != workloads.REUSE else None
+                win_b = _window_for_oracle(wl, li["swa"][b])
                 for (bb, q) in samples:
                     if bb != b:
                         continue
@@ -106,7 +133,7 @@ def test_full_size_sampled(w):
                     elif mode == workloads.REINDEX_POOL:
                         pos, ps = indexer.pool_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, pool[b, q], nv)
                         check_topk(last_idx[b, q], ps, wl.K, positions=pos, what=what)
-                    win = f32(li["swa"][b])[q * wl.swa_step: q * wl.swa_step + wl.W]
+                    win = win_b[q * wl.swa_step: q * wl.swa_step + wl.W]
                     o, lse = _attn_oracle(kv_host[(c, b)], last_idx[b, q], f32(li["q"][b, q]), win)
                     check_attention(L["out"][b, q], o, what=what)
                     np.testing.assert_allclose(L["lse"][b, q].cpu().numpy(), lse, rtol=1e-3, atol=1e-3)
