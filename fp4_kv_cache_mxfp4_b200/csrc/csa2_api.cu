@@ -67,7 +67,8 @@ inline int scan_qg(int qg) { return qg <= 1 ? 1 : qg <= 2 ? 2 : qg <= 4 ? 4 : 8;
 template <int QG, bool HSI, bool KF4>
 cudaError_t launch_scan_t(unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk, const CUtensorMap& tq,
                           const ScanParams& sp) {
-  return launch_ex(index_scan_kernel<QG, HSI, KF4>, dim3(grid), dim3(kScanThreads), smem, st, 0, tk, tq, sp);
+  return launch_ex(index_scan_kernel<QG, HSI, KF4>, dim3(grid), dim3(KF4 ? kScanThreadsF4 : kScanThreads), smem, st, 0,
+                   tk, tq, sp);
 }
 template <bool KF4>
 cudaError_t launch_scan_k(int QG, bool hsi, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
@@ -303,7 +304,7 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   int raw = 0;
   if (kf4) {
     // MXFP4 index-K: up to 8 raw tiles (8.5 KB each) in flight, beside at
-    // least two bf16 stages
+    // least two bf16 stages (three where they fit)
     sp.k4 = static_cast<const uint8_t*>(a->kI);
     const int room = kMaxDynSmem - 1024 - static_cast<int>(scan_smem_layout(2, QG, P.hb, P.hsi, 0).total);
     raw = std::min(8, room / (kRawStageBytes + 16));

@@ -10,13 +10,15 @@
 // epilogue thread then owns one entry: it reads its 32*QG head values from
 // TMEM and reduces them to QG scores (ReLU, weight, sum).
 //
-// Warp roles (320 threads):
+// Warp roles (320 threads; 448 with MXFP4 index-K):
 //   warp 0      TMA producer: streams index-K tiles into an S-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer
 //   warps 2..9  epilogue, two sets of four warps taking alternate tiles
 //               (each set covers the 128 TMEM lanes): TMEM -> scores, the
 //               score histogram used for the top-K threshold and, with HSI,
 //               the block max over 8 positions with its own histogram
+//   warps 10..13  MXFP4 index-K only: expand each raw tile into the bf16
+//               stage the MMA reads, one entry per thread
 // After the last tile every CTA adds its histograms to the global ones.
 // Pool mode (Reindex restricted to the HSI pool) gathers the tile as 16
 // blocks of 8 contiguous index-K rows with one 1 KB TMA box per block half.
@@ -24,10 +26,10 @@
 // MXFP4 index-K (68-byte entries: 64 bytes of E2M1 nibbles, 4 E8M0 block
 // scales; "DeepSeek V4.1-Flash 技术报告深度解析" §3.4 FP4 indexer K): the
 // producer streams raw tiles (128 entries, 8.5 KB, one bulk copy; pool mode
-// one 544-byte copy per block) into a ring of its own, and the epilogue
-// warps, one tile ahead of the MMA, expand each tile into the bf16 stage
-// (E2M1 x 2^e is exact in bf16) before handling their accumulators.  The
-// MMA and the score arithmetic are those of the bf16 path.
+// one 544-byte copy per block) into a ring of its own, and four extra warps
+// expand each tile into the bf16 stage (E2M1 x 2^e is exact in bf16) while
+// the epilogue warps handle earlier accumulators.  The MMA and the score
+// arithmetic are those of the bf16 path.
 //
 // HBM roofline: 256 B of index-K per entry per (row, layer) + 4 B of score
 // write; index-Q, w and histograms are negligible.
@@ -39,6 +41,8 @@ namespace csa2 {
 constexpr int kScanEpiWarps = 8;
 constexpr int kScanEpiThreads = kScanEpiWarps * 32;
 constexpr int kScanThreads = 64 + kScanEpiThreads;
+constexpr int kScanCvtWarps = 4;                   // MXFP4 index-K: warps expanding raw tiles, one row per thread
+constexpr int kScanThreadsF4 = kScanThreads + kScanCvtWarps * 32;
 constexpr int kTileRows = 128;                     // entries per MMA tile (M)
 constexpr int kStageBytes = kTileRows * 128 * 2;   // 32 KB: two 128x64 swizzled boxes
 constexpr int kAccBufs = 4;                        // TMEM accumulator slots (barriers)
@@ -99,7 +103,7 @@ __host__ __device__ inline ScanSmem scan_smem_layout(int stages, int QG, int hb,
 }
 
 template <int QG, bool HSI, bool KF4>
-__global__ void __launch_bounds__(kScanThreads, 1)
+__global__ void __launch_bounds__(KF4 ? kScanThreadsF4 : kScanThreads, 1)
 index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_q,
                   ScanParams p) {
@@ -134,9 +138,11 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   if (threadIdx.x == 0) {
     // with MXFP4 index-K a bf16 stage is full once every epilogue thread has
     // written its part of the tile
-    for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], KF4 ? kScanEpiThreads : 1); mbar_init(&empty_bar[s], 1); }
-    for (int r = 0; r < R; ++r) { mbar_init(&rfull_bar[r], 1); mbar_init(&rempty_bar[r], kScanEpiThreads); }
-    for (int a = 0; a < scan_acc_bufs(QG); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 128); }
+    // arrivals from several warps come one per warp (lane 0, after a warp
+    // barrier), not one per thread
+    for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], KF4 ? kScanCvtWarps : 1); mbar_init(&empty_bar[s], 1); }
+    for (int r = 0; r < R; ++r) { mbar_init(&rfull_bar[r], 1); mbar_init(&rempty_bar[r], kScanCvtWarps); }
+    for (int a = 0; a < scan_acc_bufs(QG); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
     mbar_init(q_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -276,6 +282,46 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
         umma_commit(&tfull_bar[a]);
       }
     }
+  } else if (KF4 && warp >= 2 + kScanEpiWarps) {
+    // ------------------------------------------------------------ expansion
+    // thread c expands entry c of each raw tile: 64 nibble bytes and four
+    // block scales -> 128 bf16 values, E2M1 x 2^e (exact), written as row c
+    // of the two 64-dim boxes of the bf16 stage in the MMA's swizzled layout
+    const int crow = threadIdx.x - 64 - kScanEpiThreads;
+    for (int t = 0; t < ntiles; ++t) {
+      const int r = t % R, st = t % p.stages;
+      bool okc = mbar_wait(&rfull_bar[r], (t / R) & 1, kErrWaitTmaFull, abort_flag);
+      okc = okc && mbar_wait(&empty_bar[st], ((t / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag);
+      if (!__all_sync(0xffffffffu, okc)) break;
+      const uint8_t* src = smem + L.raw0 + r * kRawStageBytes + crow * 68;
+      uint32_t wv[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) wv[k] = *reinterpret_cast<const uint32_t*>(src + 4 * k);
+      const uint32_t scw = *reinterpret_cast<const uint32_t*>(src + 64);
+      uint8_t* stage = smem + L.stage0 + st * kStageBytes;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        // 2^(code - 127) as bf16: exponent field = code; code 0 is 2^-127,
+        // the subnormal 0x0040
+        const uint32_t c = (scw >> (8 * blk)) & 0xFFu;
+        const uint32_t bits = c ? (c << 7) : 0x40u;
+        const uint32_t pair = bits | (bits << 16);
+        const __nv_bfloat162 S = *reinterpret_cast<const __nv_bfloat162*>(&pair);
+        uint8_t* box = stage + (blk >> 1) * (kStageBytes / 2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t o[4];
+          e2m1x8_to_bf16(wv[4 * blk + k], S, o);        // channels 32 blk + 8k .. + 7
+          *reinterpret_cast<uint4*>(box + sw128_off(crow, 4 * (blk & 1) + k)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full_bar[st]);
+        mbar_arrive(&rempty_bar[r]);
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     pdl_wait();                                   // before w and the first score store
@@ -324,7 +370,8 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
           // every head value of the tile is in registers: hand the
           // accumulator back to the MMA issuer before the reductions
           tc_fence_before();
-          mbar_arrive(&tempty_bar[a]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[a]);
         }
 #pragma unroll
         for (int j = 0; j < QB; ++j) {
@@ -366,47 +413,8 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
       }
       return true;
     };
-    if constexpr (!KF4) {
-      for (int i = set; i < ntiles; i += 2)
-        if (!epi_tile(i)) break;
-    } else {
-      // expand raw tile t into its bf16 stage (every epilogue thread: half a
-      // row), then handle accumulator t - 1 when it belongs to this set
-      const int et = threadIdx.x - 64;
-      const int crow = et >> 1, chalf = et & 1;
-      for (int t = 0; t <= ntiles; ++t) {
-        if (t < ntiles) {
-          const int r = t % R, st = t % p.stages;
-          bool okc = mbar_wait(&rfull_bar[r], (t / R) & 1, kErrWaitTmaFull, abort_flag);
-          okc = okc && mbar_wait(&empty_bar[st], ((t / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag);
-          if (!__all_sync(0xffffffffu, okc)) break;
-          const uint8_t* src = smem + L.raw0 + r * kRawStageBytes + crow * 68;
-          uint32_t wv[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) wv[k] = *reinterpret_cast<const uint32_t*>(src + 32 * chalf + 4 * k);
-          const uint32_t c0 = src[64 + 2 * chalf], c1 = src[65 + 2 * chalf];
-          // 2^(code - 127) as bf16: exponent field = code; code 0 is 2^-127,
-          // the subnormal 0x0040
-          const uint32_t b0 = c0 ? (c0 << 7) : 0x40u, b1 = c1 ? (c1 << 7) : 0x40u;
-          const uint32_t p0 = b0 | (b0 << 16), p1 = b1 | (b1 << 16);
-          const __nv_bfloat162 S0 = *reinterpret_cast<const __nv_bfloat162*>(&p0);
-          const __nv_bfloat162 S1 = *reinterpret_cast<const __nv_bfloat162*>(&p1);
-          uint8_t* box = smem + L.stage0 + st * kStageBytes + chalf * (kStageBytes / 2);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            uint32_t o[4];
-            e2m1x8_to_bf16(wv[k], k < 4 ? S0 : S1, o);       // channels 64 half + 8k .. + 7
-            *reinterpret_cast<uint4*>(box + sw128_off(crow, k)) = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_arrive(&full_bar[st]);
-          mbar_arrive(&rempty_bar[r]);
-        }
-        const int i = t - 1;
-        if (i >= 0 && (i & 1) == set)
-          if (!epi_tile(i)) break;
-      }
-    }
+    for (int i = set; i < ntiles; i += 2)
+      if (!epi_tile(i)) break;
     // flush the CTA's histograms into the global ones
     named_bar_sync(1, kScanEpiThreads);
     const int et = threadIdx.x - 64;
