@@ -32,4 +32,4 @@ library routines (ml_dtypes / torch float8, torch SDPA), brute force on tiny
 inputs or closed forms.
 """
 
-from . import fp4, fp8, mxfp4, indexer, attention, group  # noqa: F401
+from . import fp4, fp8, mxfp4, compress, indexer, attention, group  # noqa: F401
