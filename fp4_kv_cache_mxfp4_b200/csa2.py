@@ -57,6 +57,12 @@ class GroupArgs(ctypes.Structure):
                 ("swa_format", _c_i32), ("index_k_format", _c_i32)]
 
 
+class CompressArgs(ctypes.Structure):
+    _fields_ = [("x", _c_p), ("n_entries", _c_i64), ("ld_x", _c_i64), ("r", _c_i32), ("w", _c_p),
+                ("w_stride", _c_i64), ("cos", _c_p), ("sin", _c_p), ("kv_fp4", _c_p), ("dst_rows", _c_p),
+                ("row_offset", _c_i64)]
+
+
 class StackArgs(ctypes.Structure):
     _fields_ = [("n_groups", _c_i32), ("groups", ctypes.POINTER(GroupArgs))]
 
@@ -76,6 +82,7 @@ def load(path=LIB_PATH):
     lib.csa2_quantize_kv_fp4.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_p]
     lib.csa2_quantize_window_fp8.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_i64, _c_p]
     lib.csa2_quantize_index_k_mxfp4.argtypes = [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_p]
+    lib.csa2_compress_rope_quantize_kv_fp4.argtypes = [ctypes.POINTER(CompressArgs), _c_p]
     lib.csa2_index_score_topk.argtypes = [ctypes.POINTER(IndexArgs), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_index_score_topk_noalloc.argtypes = [ctypes.POINTER(IndexArgs), _c_p]
     lib.csa2_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), _c_p, ctypes.c_size_t, _c_p]
@@ -97,6 +104,7 @@ def load(path=LIB_PATH):
     lib.csa2_kernel_name.argtypes = [_c_i32]
     lib.csa2_kernel_name.restype = ctypes.c_char_p
     for name in ("csa2_quantize_kv_fp4", "csa2_quantize_window_fp8", "csa2_quantize_index_k_mxfp4",
+                 "csa2_compress_rope_quantize_kv_fp4",
                  "csa2_index_score_topk", "csa2_index_score_topk_noalloc", "csa2_sparse_attn",
                  "csa2_group_decode", "csa2_stack_decode", "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
                  "csa2_trace_end", "csa2_trace_get"):
@@ -160,6 +168,17 @@ def csa2_quantize_index_k_mxfp4(x, out, dst_rows=None, row_offset=0, stream=None
     n = x.shape[0]
     _check(load().csa2_quantize_index_k_mxfp4(_ptr(x), n, x.stride(0) if n else 128, _ptr(out), _ptr(dst_rows),
                                               row_offset, _stream(stream)), "csa2_quantize_index_k_mxfp4")
+
+
+def csa2_compress_rope_quantize_kv_fp4(x, r, w, cos, sin, kv_fp4, dst_rows=None, row_offset=0, stream=None):
+    """x bf16 [n*r, >=512] tokens, w float32 [1 or n, r, 512] weights, cos/sin
+    float32 [n, 32], kv_fp4 uint8 [rows, 288], dst_rows optional int64 [n]."""
+    n = x.shape[0] // r
+    a = CompressArgs(x=_ptr(x), n_entries=n, ld_x=x.stride(0) if n else 512, r=r, w=_ptr(w),
+                     w_stride=0 if w.shape[0] == 1 else r * 512, cos=_ptr(cos), sin=_ptr(sin), kv_fp4=_ptr(kv_fp4),
+                     dst_rows=_ptr(dst_rows), row_offset=row_offset)
+    _check(load().csa2_compress_rope_quantize_kv_fp4(ctypes.byref(a), _stream(stream)),
+           "csa2_compress_rope_quantize_kv_fp4")
 
 
 def index_args(mode, qI, w, kI, n_vis, idx, scores=None, hsi_blocks=0, hsi_block=8, pool_out=None, pool_in=None):

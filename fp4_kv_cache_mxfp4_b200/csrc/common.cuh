@@ -16,7 +16,7 @@ namespace csa2 {
 // pre-created CUDA events recorded on the launch stream.
 // ---------------------------------------------------------------------------
 enum KernelId : int { kKQuantize = 0, kKIndexScan = 1, kKTopk = 2, kKAttnSlice = 3, kKAttnCombine = 4,
-                      kKQuantizeWindow = 5, kKQuantizeIndexK = 6, kKCount = 7 };
+                      kKQuantizeWindow = 5, kKQuantizeIndexK = 6, kKCompressRope = 7, kKCount = 8 };
 
 struct LaunchTrace {
   bool on = false;

@@ -140,7 +140,8 @@ csa2_status device_info(DeviceInfo** out) {
         set_smem_attrs(sparse_attn_combine_kernel, 0) != cudaSuccess ||
         set_smem_attrs(quantize_kv_fp4_kernel, 0) != cudaSuccess ||
         set_smem_attrs(quantize_window_fp8_kernel, 0) != cudaSuccess ||
-        set_smem_attrs(quantize_index_k_mxfp4_kernel, 0) != cudaSuccess)
+        set_smem_attrs(quantize_index_k_mxfp4_kernel, 0) != cudaSuccess ||
+        set_smem_attrs(compress_rope_quantize_kernel, 0) != cudaSuccess)
       return CSA2_ERR_CUDA;
     d.topk_max_cluster = topk_cluster_limit();
     if (!g_encode) {
@@ -696,6 +697,25 @@ csa2_status csa2_quantize_window_fp8(const void* x, int64_t n, int64_t ld_x, voi
                  cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }
 
+csa2_status csa2_compress_rope_quantize_kv_fp4(const csa2_compress_args* a, void* stream) {
+  if (!a) return CSA2_ERR_ARG;
+  if (a->n_entries < 0 || a->ld_x < 512 || (a->ld_x & 7) || a->r < 1 || a->r > 16 || a->row_offset < 0 ||
+      (a->w_stride != 0 && a->w_stride != static_cast<int64_t>(a->r) * 512))
+    return CSA2_ERR_SHAPE;
+  if (a->n_entries == 0) return CSA2_OK;
+  if (!a->x || !a->w || !a->cos || !a->sin || !a->kv_fp4) return CSA2_ERR_ARG;
+  if (!aligned16(a->x) || !aligned16(a->w) || !aligned16(a->kv_fp4) ||
+      (reinterpret_cast<uintptr_t>(a->cos) & 3) || (reinterpret_cast<uintptr_t>(a->sin) & 3) ||
+      (a->dst_rows && (reinterpret_cast<uintptr_t>(a->dst_rows) & 7)))
+    return CSA2_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  const csa2_status s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  return launch_compress_rope_quantize(a->x, a->n_entries, a->ld_x, a->r, a->w, a->w_stride, a->cos, a->sin, a->kv_fp4,
+                                       a->dst_rows, a->row_offset, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
 csa2_status csa2_quantize_index_k_mxfp4(const void* x, int64_t n, int64_t ld_x, void* out, const int64_t* dst_rows,
                                         int64_t row_offset, void* stream) {
   if (n < 0 || ld_x < 128 || (ld_x & 3) || row_offset < 0) return CSA2_ERR_SHAPE;
@@ -836,7 +856,7 @@ const char* csa2_status_string(int32_t s) {
   }
 }
 
-int32_t csa2_version(void) { return 103; }
+int32_t csa2_version(void) { return 104; }
 
 csa2_status csa2_trace_begin(int32_t max_launches) {
   if (max_launches < 1 || max_launches > (1 << 20)) return CSA2_ERR_SHAPE;
@@ -892,6 +912,7 @@ const char* csa2_kernel_name(int32_t kernel) {
     case kKAttnCombine: return "sparse_attn_combine_kernel";
     case kKQuantizeWindow: return "quantize_window_fp8_kernel";
     case kKQuantizeIndexK: return "quantize_index_k_mxfp4_kernel";
+    case kKCompressRope: return "compress_rope_quantize_kernel";
     default: return "unknown";
   }
 }

@@ -40,6 +40,31 @@ __device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
   return out & 0xFF;
 }
 
+// One block of 16 channels (fp32 values) to its 8 nibble bytes and E4M3
+// scale code: sf = amax / 6, s = E4M3(sf), q = E2M1(x / s), sign kept.
+__device__ __forceinline__ void fp4_block16(const float (&v)[16], uint2& nib, uint32_t& s_code) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float sf = __fdiv_rn(amax, 6.0f);
+  s_code = e4m3_rn_sat(sf);
+  const float s = e4m3_code_to_float(s_code);
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a = v[2 * i], b = v[2 * i + 1];
+    const float ya = (s != 0.0f) ? __fdiv_rn(a, s) : 0.0f;
+    const float yb = (s != 0.0f) ? __fdiv_rn(b, s) : 0.0f;
+    uint32_t byte = e2m1x2_rn_sat(fabsf(ya), fabsf(yb));
+    // sign bits come from the inputs (x and x/s share their sign, and a
+    // zero scale keeps the sign of x)
+    byte |= (__float_as_uint(a) >> 31) << 3;
+    byte |= (__float_as_uint(b) >> 31) << 7;
+    packed[i >> 2] |= byte << (8 * (i & 3));
+  }
+  nib = make_uint2(packed[0], packed[1]);
+}
+
 __global__ void __launch_bounds__(256)
 quantize_kv_fp4_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t ld_x,
                        uint8_t* __restrict__ kv, const int64_t* __restrict__ dst_rows,
@@ -62,31 +87,12 @@ quantize_kv_fp4_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t l
     v[2 * i] = f.x;
     v[2 * i + 1] = f.y;
   }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-
-  const float sf = __fdiv_rn(amax, 6.0f);
-  const uint32_t s_code = e4m3_rn_sat(sf);
-  const float s = e4m3_code_to_float(s_code);
-
-  uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float a = v[2 * i], b = v[2 * i + 1];
-    const float ya = (s != 0.0f) ? __fdiv_rn(a, s) : 0.0f;
-    const float yb = (s != 0.0f) ? __fdiv_rn(b, s) : 0.0f;
-    uint32_t byte = e2m1x2_rn_sat(fabsf(ya), fabsf(yb));
-    // sign bits come from the inputs (x and x/s share their sign, and a
-    // zero scale keeps the sign of x)
-    byte |= (__float_as_uint(a) >> 31) << 3;
-    byte |= (__float_as_uint(b) >> 31) << 7;
-    packed[i >> 2] |= byte << (8 * (i & 3));
-  }
-
+  uint2 nib;
+  uint32_t s_code;
+  fp4_block16(v, nib, s_code);
   const int64_t dst = dst_rows ? dst_rows[row] : row_offset + row;
   uint8_t* out = kv + dst * 288;
-  *reinterpret_cast<uint2*>(out + lane * 8) = make_uint2(packed[0], packed[1]);
+  *reinterpret_cast<uint2*>(out + lane * 8) = nib;
   out[256 + lane] = static_cast<uint8_t>(s_code);
 }
 
@@ -226,6 +232,83 @@ inline cudaError_t launch_quantize_index_k(const void* x, int64_t n, int64_t ld_
   const cudaError_t e = launch_ex(quantize_index_k_mxfp4_kernel, dim3(static_cast<unsigned>(blocks)), dim3(warps * 32),
                                   0, st, 0, static_cast<const __nv_bfloat16*>(x), n, ld_x, static_cast<uint8_t*>(out),
                                   dst_rows, row_offset);
+  trace_post(st);
+  return e;
+}
+
+// ---------------------------------------------------------------------------
+// New main-KV entries compressed, rotated and quantised in one pass
+// ("DeepSeek V4.1-Flash 技术报告深度解析" §3.2 compression of r tokens per
+// entry without overlap, §3.4 quantisation after RoPE): entry e =
+// sum_j w[e][j] * x[e r + j] channel by channel (float32, one rounding per
+// operation, j ascending), then channels 448..511 rotated in adjacent pairs
+// by the caller's cos/sin (a cos - b sin, a sin + b cos), then the FP4 block
+// quantiser on the float32 result.  One warp per entry, 16 channels (one
+// scale block) per lane.
+// HBM roofline: r * 1024 B of tokens + 288 B written per entry (+ weights
+// and angles, shared or 256 B per entry).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+compress_rope_quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t ld_x, int r,
+                              const float* __restrict__ w, int64_t w_stride, const float* __restrict__ cosv,
+                              const float* __restrict__ sinv, uint8_t* __restrict__ kv,
+                              const int64_t* __restrict__ dst_rows, int64_t row_offset) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (e >= n) return;
+  float v[16] = {};                                   // every element is set at j = 0
+  const float* we = w + e * w_stride;
+#pragma unroll 1
+  for (int j = 0; j < r; ++j) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (e * r + j) * ld_x + lane * 16);
+    const uint4 raw0 = __ldg(src), raw1 = __ldg(src + 1);
+    const uint32_t rw[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
+    const float4* wj = reinterpret_cast<const float4*>(we + j * 512 + lane * 16);
+    float wv[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 t = __ldg(wj + k);
+      wv[4 * k] = t.x; wv[4 * k + 1] = t.y; wv[4 * k + 2] = t.z; wv[4 * k + 3] = t.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[i]));
+      const float p0 = __fmul_rn(wv[2 * i], f.x), p1 = __fmul_rn(wv[2 * i + 1], f.y);
+      v[2 * i] = (j == 0) ? p0 : __fadd_rn(v[2 * i], p0);
+      v[2 * i + 1] = (j == 0) ? p1 : __fadd_rn(v[2 * i + 1], p1);
+    }
+  }
+  if (lane >= 28) {                                   // channels 448..511: pairs 8 (lane - 28) ..
+    const int p0 = 8 * (lane - 28);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float c = __ldg(cosv + e * 32 + p0 + k), sn = __ldg(sinv + e * 32 + p0 + k);
+      const float a = v[2 * k], b = v[2 * k + 1];
+      v[2 * k] = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, sn));
+      v[2 * k + 1] = __fadd_rn(__fmul_rn(a, sn), __fmul_rn(b, c));
+    }
+  }
+  uint2 nib;
+  uint32_t s_code;
+  fp4_block16(v, nib, s_code);
+  const int64_t dst = dst_rows ? dst_rows[e] : row_offset + e;
+  uint8_t* out = kv + dst * 288;
+  *reinterpret_cast<uint2*>(out + lane * 8) = nib;
+  out[256 + lane] = static_cast<uint8_t>(s_code);
+}
+
+inline cudaError_t launch_compress_rope_quantize(const void* x, int64_t n, int64_t ld_x, int r, const float* w,
+                                                 int64_t w_stride, const float* cosv, const float* sinv, void* kv,
+                                                 const int64_t* dst_rows, int64_t row_offset, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int warps = 8;
+  const int64_t blocks = (n + warps - 1) / warps;
+  trace_pre(kKCompressRope, st);
+  const cudaError_t e = launch_ex(compress_rope_quantize_kernel, dim3(static_cast<unsigned>(blocks)),
+                                  dim3(warps * 32), 0, st, 0, static_cast<const __nv_bfloat16*>(x), n, ld_x, r, w,
+                                  w_stride, cosv, sinv, static_cast<uint8_t*>(kv), dst_rows, row_offset);
   trace_post(st);
   return e;
 }

@@ -115,6 +115,39 @@ csa2_status csa2_quantize_kv_fp4(const void* x, int64_t n, int64_t ld_x,
                                  int64_t row_offset, void* stream);
 
 /* ------------------------------------------------------------------------
+ * csa2_compress_rope_quantize_kv_fp4 -- new main-KV entries made, rotated
+ * and quantised in one pass.  [eogee] §3.2: CSA2 compresses every r tokens
+ * into one entry (r = 2 in the encoder, 1 in the decoder), with no overlap
+ * between neighbouring entries and no absolute position encoding in the
+ * compression; §3.4: the entry is quantised after RoPE.  The pages give
+ * neither the compressor's form nor the rotation layout; this call takes:
+ *     entry e = sum_{j<r} w[e][j] (.) x[e*r + j]         (channel by channel)
+ *     channels 448 + 2i, 449 + 2i (i < 32, the 64-dim RoPE slice) rotated:
+ *         (a, b) -> (a cos[e][i] - b sin[e][i], a sin[e][i] + b cos[e][i])
+ *     then the FP4 quantiser of csa2_quantize_kv_fp4 on the result.
+ * Every step is IEEE float32 with one rounding per operation, in the order
+ * written (no fused multiply-add), with no bf16 rounding before the
+ * quantiser; the angles (cos, sin) are the caller's, so the frequencies
+ * (YaRN or other) are the model's choice.
+ * ---------------------------------------------------------------------- */
+typedef struct csa2_compress_args {
+    const void*    x;           /* bf16 [n_entries * r][ld_x] token vectors      */
+    int64_t        n_entries;   /* entries to make, >= 0                         */
+    int64_t        ld_x;        /* >= 512, a multiple of 8                       */
+    int32_t        r;           /* tokens per entry, 1..16                       */
+    const float*   w;           /* f32 weights [.][r][512]                       */
+    int64_t        w_stride;    /* floats between entries' weights: 0 (shared)
+                                   or r * 512                                    */
+    const float*   cos;         /* f32 [n_entries][32]                           */
+    const float*   sin;         /* f32 [n_entries][32]                           */
+    void*          kv_fp4;      /* u8 cache rows of CSA2_ENTRY_BYTES bytes       */
+    const int64_t* dst_rows;    /* optional int64 [n_entries]: destination rows  */
+    int64_t        row_offset;  /* first destination row when dst_rows is NULL   */
+} csa2_compress_args;
+
+csa2_status csa2_compress_rope_quantize_kv_fp4(const csa2_compress_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
  * csa2_quantize_window_fp8 -- [eogee] §3.4: the quantisation-sensitive SWA
  * KV cache stays in FP8.  The page names the precision only; this library's
  * format is one E4M3 code per channel and one f32 scale per 512-channel row:
@@ -435,6 +468,7 @@ int32_t csa2_version(void);
 #define CSA2_KERNEL_ATTN_COMBINE 4
 #define CSA2_KERNEL_QUANTIZE_WINDOW 5
 #define CSA2_KERNEL_QUANTIZE_INDEX_K 6
+#define CSA2_KERNEL_COMPRESS_ROPE   7
 csa2_status csa2_trace_begin(int32_t max_launches);
 csa2_status csa2_trace_stop(void);
 csa2_status csa2_trace_end(void);

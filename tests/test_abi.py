@@ -42,7 +42,7 @@ def test_every_declared_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert csa2.version() == 103
+    assert csa2.version() == 104
     assert csa2.status_string(0) == "ok"
     assert "workspace" in csa2.status_string(4)
     assert csa2.status_string(99) == "unknown status"
@@ -55,6 +55,7 @@ def _c_layout():
         "csa2_layer": [f for f, _ in csa2.Layer._fields_],
         "csa2_group_args": [f for f, _ in csa2.GroupArgs._fields_],
         "csa2_stack_args": [f for f, _ in csa2.StackArgs._fields_],
+        "csa2_compress_args": [f for f, _ in csa2.CompressArgs._fields_],
     }
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "csa2.h"', "int main(void) {"]
     for s, fs in fields.items():
@@ -74,7 +75,7 @@ def test_struct_layouts_match_the_header():
     c = _c_layout()
     for cname, py in [("csa2_index_args", csa2.IndexArgs), ("csa2_attn_args", csa2.AttnArgs),
                       ("csa2_layer", csa2.Layer), ("csa2_group_args", csa2.GroupArgs),
-                      ("csa2_stack_args", csa2.StackArgs)]:
+                      ("csa2_stack_args", csa2.StackArgs), ("csa2_compress_args", csa2.CompressArgs)]:
         assert int(c[cname]) == ctypes.sizeof(py), cname
         for f, _ in py._fields_:
             assert int(c[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
@@ -279,3 +280,19 @@ def test_workspace_sizes_for_prefill_shapes(L):
     assert 0 < L.csa2_workspace_size(ctypes.byref(small), csa2.WS_ATTN) <= 256
     many = _attn(B=1, Q=127, K=1024, W=128, swa_step=1, swa_rows=128 + 126)      # 9 slices
     assert L.csa2_workspace_size(ctypes.byref(many), csa2.WS_ATTN) >= 127 * 9 * 64 * 512 * 4
+
+
+def test_compress_validation(L):
+    def args(**kw):
+        a = csa2.CompressArgs(x=FAKE, n_entries=4, ld_x=512, r=2, w=FAKE, w_stride=0, cos=FAKE, sin=FAKE,
+                              kv_fp4=FAKE, dst_rows=None, row_offset=0)
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return L.csa2_compress_rope_quantize_kv_fp4(ctypes.byref(a), None)
+    assert L.csa2_compress_rope_quantize_kv_fp4(None, None) == 1
+    assert args(r=0) == 2 and args(r=17) == 2 and args(ld_x=500) == 2 and args(w_stride=7) == 2
+    assert args(n_entries=-1) == 2 and args(row_offset=-1) == 2
+    assert args(cos=None) == 1 and args(w=None) == 1 and args(kv_fp4=None) == 1
+    assert args(x=FAKE + 8) == 3 and args(sin=FAKE + 2) == 3
+    assert args(n_entries=0, x=None) == 0
+
