@@ -560,8 +560,11 @@ csa2_status check_group(const csa2_group_args* g, size_t* iz, size_t* iw, size_t
 }
 
 // Enqueue one validated group on `st` (workspace already large enough).
+// first_early: the first layer's inputs were complete before the call
+// (false for a group of a stack after the first: its first layer follows
+// the previous group's last layer in model order)
 csa2_status run_group(const csa2_group_args* g, size_t iz, size_t iw, const DeviceInfo& dev, void* ws,
-                      cudaStream_t st) {
+                      cudaStream_t st, bool first_early = true) {
   struct SerialScope {                             // CSA2_GROUP_SERIAL: plain stream order for this call
     bool prev;
     explicit SerialScope(bool on) : prev(g_serial_launch) { if (on) g_serial_launch = true; }
@@ -581,7 +584,7 @@ csa2_status run_group(const csa2_group_args* g, size_t iz, size_t iw, const Devi
     const csa2_layer& L = g->layers[i];
     // the first layer's inputs precede the call; a later layer's are, in a
     // model, the previous layer's results unless the caller says otherwise
-    const bool early = inputs_ready || i == 0;
+    const bool early = inputs_ready || (i == 0 && first_early);
     if (L.mode != CSA2_REUSE) {
       const csa2_index_args a = layer_index_args(g, L, cur_pool);
       const csa2_status s = run_index(&a, dev, zws, dws, st, g->kv_fp4, early);
@@ -794,7 +797,7 @@ csa2_status csa2_stack_decode(const csa2_stack_args* sa, void* ws, size_t ws_byt
   for (int i = 0; i < sa->n_groups; ++i) {
     size_t iz = 0, iw = 0, n = 0;
     check_group(&sa->groups[i], &iz, &iw, &n);
-    s = run_group(&sa->groups[i], iz, iw, *dev, ws, static_cast<cudaStream_t>(stream));
+    s = run_group(&sa->groups[i], iz, iw, *dev, ws, static_cast<cudaStream_t>(stream), i == 0);
     if (s != CSA2_OK) return s;
   }
   return CSA2_OK;
@@ -856,7 +859,7 @@ const char* csa2_status_string(int32_t s) {
   }
 }
 
-int32_t csa2_version(void) { return 104; }
+int32_t csa2_version(void) { return 105; }
 
 csa2_status csa2_trace_begin(int32_t max_launches) {
   if (max_launches < 1 || max_launches > (1 << 20)) return CSA2_ERR_SHAPE;

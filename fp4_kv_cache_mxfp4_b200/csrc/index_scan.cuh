@@ -288,9 +288,10 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // block scales -> 128 bf16 values, E2M1 x 2^e (exact), written as row c
     // of the two 64-dim boxes of the bf16 stage in the MMA's swizzled layout
     const int crow = threadIdx.x - 64 - kScanEpiThreads;
+    const int Rc = R > 0 ? R : 1;                  // R >= 2 here (this role exists with MXFP4 index-K only)
     for (int t = 0; t < ntiles; ++t) {
-      const int r = t % R, st = t % p.stages;
-      bool okc = mbar_wait(&rfull_bar[r], (t / R) & 1, kErrWaitTmaFull, abort_flag);
+      const int r = t % Rc, st = t % p.stages;
+      bool okc = mbar_wait(&rfull_bar[r], (t / Rc) & 1, kErrWaitTmaFull, abort_flag);
       okc = okc && mbar_wait(&empty_bar[st], ((t / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag);
       if (!__all_sync(0xffffffffu, okc)) break;
       const uint8_t* src = smem + L.raw0 + r * kRawStageBytes + crow * 68;

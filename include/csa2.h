@@ -401,11 +401,15 @@ csa2_status csa2_group_decode(const csa2_group_args* g, void* ws,
  * the decoder's 20 layers are 5 groups of 4, the first Full + 3 Reuse, the
  * others Reindex + 3 Reuse; the encoder's 18 are 3 groups of Full + 5
  * Reuse).  Equivalent to calling csa2_group_decode for groups[0..n_groups)
- * in order with one workspace: each group's pool_in may point at an earlier
- * group's pool (the decoder's first Full layer builds the pool that every
- * later Reindex layer re-scores, [eogee] §3.3).  The workspace is the
- * largest any single group needs (csa2_workspace_size(&stack_args,
- * CSA2_WS_STACK)); flags of the groups apply to their own kernels.
+ * in order with one workspace, except that a group after the first is a
+ * model-order successor of the one before it: its first layer's inputs are
+ * read only after the previous group's last kernel has finished (unless
+ * that group's flags hold CSA2_GROUP_INPUTS_READY).  Each group's pool_in
+ * may point at an earlier group's pool (the decoder's first Full layer
+ * builds the pool that every later Reindex layer re-scores, [eogee] §3.3).
+ * The workspace is the largest any single group needs
+ * (csa2_workspace_size(&stack_args, CSA2_WS_STACK)); flags of the groups
+ * apply to their own kernels.
  * Errors: those of csa2_group_decode, checked for every group before
  * anything is enqueued; ARG when n_groups is outside 1..64.
  * ---------------------------------------------------------------------- */

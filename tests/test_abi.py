@@ -42,7 +42,7 @@ def test_every_declared_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert csa2.version() == 104
+    assert csa2.version() == 105
     assert csa2.status_string(0) == "ok"
     assert "workspace" in csa2.status_string(4)
     assert csa2.status_string(99) == "unknown status"
