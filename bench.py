@@ -360,7 +360,10 @@ def oracle_row_setup(wl, b):
         swa = li["swa"][b].float().numpy()
         if wl.window_format == 1:               # FP8 window rows, dequantised
             swa = fp8.dequantize_window_fp8(*fp8.quantize_window_fp8(swa))
-        layers.append(dict(mode=mode, qI=li["qI"][b, q0:q0 + qn].float().numpy(), w=li["w"][b, q0:q0 + qn].numpy(),
+        qI = li["qI"][b, q0:q0 + qn].float().numpy()
+        if wl.index_k_format == 2:              # index-Q quantised like the FP4 index-K
+            qI = mxfp4.fake_quantize(qI)
+        layers.append(dict(mode=mode, qI=qI, w=li["w"][b, q0:q0 + qn].numpy(),
                            q=li["q"][b, q0:q0 + qn].float().numpy(), swa=swa[w0:w1]))
     need = set(wl.new_rows)
     for L in layers:

@@ -159,6 +159,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int er
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+#ifdef CSA2_WAIT_BACKOFF_NS
+    __nanosleep(CSA2_WAIT_BACKOFF_NS);
+#endif
     if (*abort) return false;
     if (global_ns() - t0 > kWaitLimitNs) {
       record_error(err);
@@ -354,6 +357,87 @@ __device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, __nv_bfloat162 scale,
     x = __hmul2(x, scale);
     out[j] = *reinterpret_cast<uint32_t*>(&x);
   }
+}
+
+// Two magnitudes to E2M1 (round to nearest even, saturate at 6): `lo` lands
+// in bits 0-3, `hi` in bits 4-7.
+__device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+      "cvt.u32.u8 %0, b;\n\t}"
+      : "=r"(out) : "f"(hi), "f"(lo));
+  return out & 0xFF;
+}
+
+// ---------------------------------------------------------------- block-scaled FP4 MMA
+// Shared-memory descriptor for a K-major operand in the 64-byte-swizzle
+// canonical layout: rows of 64 B (128 packed E2M1 values), groups of 8 rows
+// 512 B apart, the 16-byte chunk c of row r stored at chunk c ^ ((r >> 1) & 3).
+// Layout type 4 = 64-byte swizzle; the other fields as for 128-byte swizzle.
+__device__ __forceinline__ uint64_t umma_desc_sw64_kmajor(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(512 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
+  return d;
+}
+// byte offset of 16-byte chunk c of row r in a 64-byte-swizzled tile
+__host__ __device__ __forceinline__ uint32_t sw64_off(int r, int c) {
+  return static_cast<uint32_t>(r) * 64u + static_cast<uint32_t>((c ^ ((r >> 1) & 3)) * 16);
+}
+
+// Descriptor of a 32-row x 16-byte block-scale chunk (no swizzle, rows
+// contiguous, 8-row core matrices 128 B apart) for tcgen05.cp.
+__device__ __forceinline__ uint64_t umma_desc_sf_chunk(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Block-scale chunk of 128 operand rows x 4 scale bytes (512 B), the
+// arrangement the MMA reads from tensor memory after one
+// tcgen05.cp.32x128b.warpx4: 16-byte line m0 holds rows m0, m0+32, m0+64,
+// m0+96 (4 bytes each: the scales of K blocks 0..3).  Byte offset of the
+// scale of row r (0..127), K block k.
+__host__ __device__ __forceinline__ uint32_t sf_chunk_off(int r, int k) {
+  return static_cast<uint32_t>(16 * (r & 31) + 4 * (r >> 5) + k);
+}
+
+// Copy one 512-byte scale chunk into 4 tensor-memory columns at taddr; the
+// 32 lines land in lanes 0..31 and are repeated in every lane quarter.
+__device__ __forceinline__ void tmem_cp_sf_chunk(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor, kind::mxf4 (E2M1 A and B, UE8M0 scales per 32
+// values, f32 accumulator, both K-major, K = 64 per instruction), shape
+// M x N; sf_id selects the scale byte of each 32-bit scale column (the
+// instruction uses bytes sf_id and sf_id + 1).
+__host__ __device__ constexpr uint32_t umma_idesc_mxf4(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4)                                // B scale byte
+       | (1u << 7)                                   // A format: E2M1
+       | (1u << 10)                                  // B format: E2M1
+       | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
+       | (1u << 23)                                  // scale format: UE8M0
+       | (static_cast<uint32_t>(M >> 4) << 24)       // M / 16
+       | (sf_id << 29);                              // A scale byte
+}
+
+// D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T, block-scaled E2M1,
+// issued by a single thread; tsfa / tsfb: tensor-memory scale columns.
+__device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

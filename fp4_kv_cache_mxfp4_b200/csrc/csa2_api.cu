@@ -54,7 +54,11 @@ cudaError_t set_scan_attrs_k() {
   cudaError_t r[8] = {set_scan_attr_one<1, false, KF4>(), set_scan_attr_one<1, true, KF4>(),
                       set_scan_attr_one<2, false, KF4>(), set_scan_attr_one<2, true, KF4>(),
                       set_scan_attr_one<4, false, KF4>(), set_scan_attr_one<4, true, KF4>(),
-                      set_scan_attr_one<8, false, KF4>(), set_scan_attr_one<8, true, KF4>()};
+                      cudaSuccess, cudaSuccess};
+  if constexpr (!KF4) {                      // MXFP4 index-K groups at most 4 queries
+    r[6] = set_scan_attr_one<8, false, KF4>();
+    r[7] = set_scan_attr_one<8, true, KF4>();
+  }
   for (cudaError_t x : r) if (x != cudaSuccess) e = x;
   return e;
 }
@@ -80,8 +84,10 @@ cudaError_t launch_scan_k(int QG, bool hsi, unsigned grid, size_t smem, cudaStre
     case 5: return launch_scan_t<2, true, KF4>(grid, smem, st, tk, tq, sp);
     case 8: return launch_scan_t<4, false, KF4>(grid, smem, st, tk, tq, sp);
     case 9: return launch_scan_t<4, true, KF4>(grid, smem, st, tk, tq, sp);
-    case 16: return launch_scan_t<8, false, KF4>(grid, smem, st, tk, tq, sp);
-    default: return launch_scan_t<8, true, KF4>(grid, smem, st, tk, tq, sp);
+    default:
+      if constexpr (KF4) return cudaErrorInvalidValue;   // plan_index caps MXFP4 groups at 4 queries
+      else return QG * 2 == 16 ? launch_scan_t<8, false, KF4>(grid, smem, st, tk, tq, sp)
+                               : launch_scan_t<8, true, KF4>(grid, smem, st, tk, tq, sp);
   }
 }
 cudaError_t launch_scan(int QG, bool hsi, bool kf4, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
@@ -217,7 +223,7 @@ IndexPlan plan_index(const csa2_index_args* a) {
   P.pool = a->mode == CSA2_REINDEX_POOL;
   P.hsi = a->mode == CSA2_FULL && a->hsi_blocks > 0;
   P.BQ = a->B * a->Q;
-  P.qg = P.pool ? 1 : std::min(a->Q, 8);
+  P.qg = P.pool ? 1 : std::min(a->Q, a->k_format == CSA2_FMT_MXFP4 ? kF4MaxQG : 8);
   // score histogram bits: 4096 bins per query for 1-2 queries per MMA group,
   // 2048 for 4-8 (1024 with HSI, whose block histogram needs the room too)
   P.hb = (P.qg <= 2) ? 12 : (P.hsi ? 10 : 11);
@@ -297,27 +303,28 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.ctas_per_group = scan_ctas_per_group(sp.groups, sp.tiles_per_group, dev.sms);
   const int QG = scan_qg(P.qg);
   const uint32_t n_mma = 32u * QG;
-  uint32_t cols = 32;
-  while (cols < scan_acc_bufs(QG) * n_mma) cols <<= 1;
-  sp.tmem_cols = cols;
   sp.early_q = early_q ? 1 : 0;
   const bool kf4 = a->k_format == CSA2_FMT_MXFP4;
+  const int smem_room = kMaxDynSmem - 1024;
   int raw = 0;
   if (kf4) {
-    // MXFP4 index-K: up to 8 raw tiles (8.5 KB each) in flight, beside at
-    // least two bf16 stages (three where they fit)
+    // MXFP4 index-K: up to kF4RawStages raw tiles (8.5 KB each) in flight
+    // and 4 repacked stages (9 KB each) for the MMA
     sp.k4 = static_cast<const uint8_t*>(a->kI);
-    const int room = kMaxDynSmem - 1024 - static_cast<int>(scan_smem_layout(2, QG, P.hb, P.hsi, 0).total);
-    raw = std::min(8, room / (kRawStageBytes + 16));
-    if (raw < 2) return CSA2_ERR_SHAPE;
+    sp.stages = 4;
+    raw = kF4RawStages;
+    while (raw > 2 && static_cast<int>(scan_smem_layout(sp.stages, QG, P.hb, P.hsi, raw).total) > smem_room) --raw;
+  } else {
+    // three 32 KB stages per SM measured fastest (fewer bytes in flight per
+    // stream keep DRAM pages open longer; 2, 4 and 6 stages were slower)
+    const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi, 0);
+    sp.stages = std::min(kScanStages, static_cast<int>((smem_room - L0.total) / (kStageBytes + 16)));
+    if (sp.stages < 2) return CSA2_ERR_SHAPE;
   }
   sp.raw_stages = raw;
-  const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi, raw);
-  // three 32 KB stages per SM measured fastest (fewer bytes in flight per
-  // stream keep DRAM pages open longer; 2, 4 and 6 stages were slower)
-  sp.stages = std::min(kScanStages, static_cast<int>((kMaxDynSmem - 1024 - L0.total) / (kStageBytes + 16)));
-  if (sp.stages < 2) return CSA2_ERR_SHAPE;
   const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi, raw);
+  if (static_cast<int>(L.total) > smem_room) return CSA2_ERR_SHAPE;
+  sp.tmem_cols = scan_tmem_cols(QG, kf4, sp.stages);
   CUtensorMap tk, tq;
   if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, n_mma)) return CSA2_ERR_CUDA;
   if (kf4) tk = tq;                                 // not read: index-K arrives by bulk copies

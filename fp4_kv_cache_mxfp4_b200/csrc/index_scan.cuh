@@ -17,22 +17,35 @@
 //               (each set covers the 128 TMEM lanes): TMEM -> scores, the
 //               score histogram used for the top-K threshold and, with HSI,
 //               the block max over 8 positions with its own histogram
-//   warps 10..13  MXFP4 index-K only: expand each raw tile into the bf16
-//               stage the MMA reads, one entry per thread
+//   warps 10..13  MXFP4 index-K only: quantise the index-Q tile, then
+//               repack each raw tile into the stage the MMA reads, one
+//               entry per thread
 // After the last tile every CTA adds its histograms to the global ones.
 // Pool mode (Reindex restricted to the HSI pool) gathers the tile as 16
 // blocks of 8 contiguous index-K rows with one 1 KB TMA box per block half.
 //
 // MXFP4 index-K (68-byte entries: 64 bytes of E2M1 nibbles, 4 E8M0 block
-// scales; "DeepSeek V4.1-Flash 技术报告深度解析" §3.4 FP4 indexer K): the
-// producer streams raw tiles (128 entries, 8.5 KB, one bulk copy; pool mode
-// one 544-byte copy per block) into a ring of its own, and four extra warps
-// expand each tile into the bf16 stage (E2M1 x 2^e is exact in bf16) while
-// the epilogue warps handle earlier accumulators.  The MMA and the score
-// arithmetic are those of the bf16 path.
+// scales; "DeepSeek V4.1-Flash 技术报告深度解析" §3.4, where the indexer's
+// Q and K are both FP4): the contraction runs on the block-scaled FP4 tensor
+// path (tcgen05.mma kind::mxf4, E2M1 x E2M1 with one UE8M0 scale per 32
+// values, f32 accumulation), so no value is widened.
+//   - index-Q is quantised to the same MXFP4 rule once per CTA by the four
+//     extra warps: E2M1 codes in a 64-byte-swizzled tile (the B operand)
+//     and its scales in the block-scale chunk layout, copied once into
+//     tensor memory;
+//   - the producer streams raw tiles (128 entries, 8.5 KB, one bulk copy;
+//     pool mode one 544-byte copy per block of 8) into a ring of its own;
+//   - the extra warps repack each raw tile: the 64 nibble bytes of entry c
+//     become row c of a 64-byte-swizzled 128 x 128 E2M1 tile (the A
+//     operand) and its 4 scale bytes go to the tile's scale chunk, which
+//     the MMA issuer copies into tensor memory (tcgen05.cp) before the two
+//     K = 64 MMAs of the tile.
+// E2M1 x E2M1 x 2^(ea + eb) products are exact and the sum is f32, as in
+// the bf16 path: the score is that of the dequantised Q and K.
 //
-// HBM roofline: 256 B of index-K per entry per (row, layer) + 4 B of score
-// write; index-Q, w and histograms are negligible.
+// HBM roofline: 256 B (bf16) or 68 B (MXFP4) of index-K per entry per
+// (row, layer) + 4 B of score write; index-Q, w and histograms are
+// negligible.
 #pragma once
 #include "common.cuh"
 
@@ -47,9 +60,29 @@ constexpr int kTileRows = 128;                     // entries per MMA tile (M)
 constexpr int kStageBytes = kTileRows * 128 * 2;   // 32 KB: two 128x64 swizzled boxes
 constexpr int kAccBufs = 4;                        // TMEM accumulator slots (barriers)
 constexpr int kRawStageBytes = kTileRows * 68;     // MXFP4 index-K: one raw tile of 68-byte entries
+constexpr int kF4NibBytes = kTileRows * 64;        // MXFP4: repacked E2M1 tile, 128 rows x 64 B
+constexpr int kF4StageBytes = kF4NibBytes + 1024;  // + its 512-byte scale chunk, padded to the swizzle alignment
+constexpr int kF4MaxQG = 4;                        // MXFP4: queries per MMA group (TMEM room for scales)
+#ifndef CSA2_F4_RAW_STAGES
+#define CSA2_F4_RAW_STAGES 8
+#endif
+constexpr int kF4RawStages = CSA2_F4_RAW_STAGES;   // MXFP4: raw tiles in flight per CTA (at most)
 
-// accumulators in flight: as many as fit the 512 TMEM columns, at most 4
-__host__ __device__ constexpr int scan_acc_bufs(int QG) { return 32 * QG * 4 <= 512 ? 4 : 2; }
+// accumulators in flight: as many as fit the 512 TMEM columns (less the
+// block-scale columns of the MXFP4 path), at most 4
+__host__ __device__ constexpr int scan_acc_bufs(int QG, bool kf4 = false) {
+  return 32 * QG * 4 + (kf4 ? 64 : 0) <= 512 ? 4 : 2;
+}
+// MXFP4: 512-byte scale chunks (128 rows each) of the index-Q tile
+__host__ __device__ constexpr int scan_q_chunks(int QG) { return (32 * QG + 127) / 128; }
+// tensor-memory columns: accumulators, then (MXFP4) 4 scale columns per
+// stage and per index-Q chunk; a power of two >= 32
+__host__ __device__ inline uint32_t scan_tmem_cols(int QG, bool kf4, int stages) {
+  uint32_t need = static_cast<uint32_t>(scan_acc_bufs(QG, kf4) * 32 * QG + (kf4 ? 4 * (stages + scan_q_chunks(QG)) : 0));
+  uint32_t cols = 32;
+  while (cols < need) cols <<= 1;
+  return cols;
+}
 
 struct ScanParams {
   int pool_mode;          // 0: scan [0, n_vis) of each row; 1: scan the pool of each (b,q)
@@ -83,16 +116,21 @@ struct ScanParams {
 
 struct ScanSmem {
   // offsets inside the dynamic shared memory block
-  uint32_t stage0, raw0, qi0, w0, hist0, bhist0, bar0, total;
+  uint32_t stage0, raw0, qi0, q40, sfb0, w0, hist0, bhist0, bar0, total;
 };
 
-// raw_stages: MXFP4 index-K raw tiles (0 for bf16 index-K)
+// raw_stages: MXFP4 index-K raw tiles (0 for bf16 index-K, which also
+// selects the bf16 stage size)
 __host__ __device__ inline ScanSmem scan_smem_layout(int stages, int QG, int hb, int hsi, int raw_stages = 0) {
   ScanSmem L;
+  const bool kf4 = raw_stages > 0;
   uint32_t off = 0;
-  L.stage0 = off; off += stages * kStageBytes;
+  L.stage0 = off; off += stages * (kf4 ? kF4StageBytes : kStageBytes);
   L.raw0 = off;   off += raw_stages * kRawStageBytes;
+  off = (off + 1023) & ~1023u;                          // swizzled operand tiles start on 1 KB
   L.qi0 = off;    off += 2 * (32 * QG) * 128;          // two 64-dim halves of [32*QG x 64] bf16
+  L.q40 = off;    off += kf4 ? (32 * QG) * 64 : 0;     // MXFP4 index-Q, [32*QG x 64 B] swizzled
+  L.sfb0 = off;   off += kf4 ? scan_q_chunks(QG) * 512 : 0;
   L.w0 = off;     off += QG * 32 * 4;
   L.hist0 = off;  off += QG * (1u << hb) * 4;
   L.bhist0 = off; off += hsi ? QG * (1u << hb) * 4 : 0;
@@ -119,6 +157,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   uint64_t* rfull_bar = tempty_bar + kAccBufs;     // MXFP4: raw tile landed
   uint64_t* rempty_bar = rfull_bar + R;            // MXFP4: raw tile expanded
   uint64_t* q_bar = rempty_bar + R;
+  uint64_t* q4_bar = q_bar + 1;                    // MXFP4: index-Q quantised
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* w_s = reinterpret_cast<float*>(smem + L.w0);
@@ -136,14 +175,14 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int nbins = 1 << p.hb;
 
   if (threadIdx.x == 0) {
-    // with MXFP4 index-K a bf16 stage is full once every epilogue thread has
-    // written its part of the tile
-    // arrivals from several warps come one per warp (lane 0, after a warp
-    // barrier), not one per thread
+    // with MXFP4 index-K a stage is full once every repacking warp has
+    // written its part of the tile; arrivals from several warps come one
+    // per warp (lane 0, after a warp barrier), not one per thread
     for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], KF4 ? kScanCvtWarps : 1); mbar_init(&empty_bar[s], 1); }
     for (int r = 0; r < R; ++r) { mbar_init(&rfull_bar[r], 1); mbar_init(&rempty_bar[r], kScanCvtWarps); }
-    for (int a = 0; a < scan_acc_bufs(QG); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
+    for (int a = 0; a < scan_acc_bufs(QG, KF4); ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
     mbar_init(q_bar, 1);
+    mbar_init(q4_bar, kScanCvtWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -180,7 +219,8 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   constexpr uint32_t n_mma = 32u * QG;
-  constexpr int ACC = scan_acc_bufs(QG);
+  constexpr int ACC = scan_acc_bufs(QG, KF4);
+  static_assert(!KF4 || QG <= kF4MaxQG, "MXFP4 index-K: at most 4 queries per MMA group");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -257,7 +297,37 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && ntiles > 0) {
+    if (KF4 && lane == 0 && ntiles > 0) {
+      // block-scaled FP4: per tile, its scale chunk into this stage's 4
+      // scale columns, then two K = 64 MMAs (scale bytes 0-1, then 2-3)
+      const uint32_t sfa_col = tmem_base + ACC * n_mma;
+      const uint32_t sfb_col = sfa_col + 4 * p.stages;
+      const uint32_t q4_addr = smem_u32(smem + L.q40);
+      bool ok = mbar_wait(q4_bar, 0, kErrWaitOperand, abort_flag);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < scan_q_chunks(QG); ++c)
+          tmem_cp_sf_chunk(sfb_col + 4 * c, umma_desc_sf_chunk(smem_u32(smem + L.sfb0 + 512 * c)));
+      }
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int s = i % p.stages;
+        const int a = i % ACC;
+        if (!mbar_wait(&tempty_bar[a], ((i / ACC) & 1) ^ 1, kErrWaitTmemEmpty, abort_flag)) break;
+        if (!mbar_wait(&full_bar[s], (i / p.stages) & 1, kErrWaitTmaFull, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t st_addr = smem_u32(smem + L.stage0 + s * kF4StageBytes);
+        const uint32_t d_tmem = tmem_base + a * n_mma;
+        tmem_cp_sf_chunk(sfa_col + 4 * s, umma_desc_sf_chunk(st_addr + kF4NibBytes));
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          umma_mxf4(d_tmem, umma_desc_sw64_kmajor(st_addr + 32 * ks), umma_desc_sw64_kmajor(q4_addr + 32 * ks),
+                    umma_idesc_mxf4(128, n_mma, 2u * ks), sfa_col + 4 * s, sfb_col, ks > 0 ? 1u : 0u);
+        umma_commit(&empty_bar[s]);
+        umma_commit(&tfull_bar[a]);
+      }
+    }
+    if (!KF4 && lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc = umma_idesc_bf16_f32(128, n_mma);
       const uint32_t qi_addr = smem_u32(smem + L.qi0);
       constexpr uint32_t qbox = n_mma * 128;
@@ -283,39 +353,80 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
       }
     }
   } else if (KF4 && warp >= 2 + kScanEpiWarps) {
-    // ------------------------------------------------------------ expansion
-    // thread c expands entry c of each raw tile: 64 nibble bytes and four
-    // block scales -> 128 bf16 values, E2M1 x 2^e (exact), written as row c
-    // of the two 64-dim boxes of the bf16 stage in the MMA's swizzled layout
-    const int crow = threadIdx.x - 64 - kScanEpiThreads;
+    // ------------------------------------------------------------ MXFP4 repacking
+    const int crow = threadIdx.x - 64 - kScanEpiThreads;      // 0..127
     const int Rc = R > 0 ? R : 1;                  // R >= 2 here (this role exists with MXFP4 index-K only)
+    // index-Q to MXFP4 (the index-K rule: e = floor(log2 amax) - 2 per 32
+    // values, q = E2M1(x / 2^e)), one (head row, 32-value block) per thread
+    auto quantize_q = [&]() {
+      if (mbar_wait(q_bar, 0, kErrWaitOperand, abort_flag)) {
+        constexpr uint32_t qbox = n_mma * 128;
+        const uint8_t* qi = smem + L.qi0;
+        uint8_t* q4 = smem + L.q40;
+        uint8_t* sfb = smem + L.sfb0;
+        for (int item = crow; item < static_cast<int>(n_mma) * 4; item += kScanCvtWarps * 32) {
+          const int rr = item >> 2, k = item & 3;
+          const uint8_t* box = qi + (k >> 1) * qbox;
+          float v[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 u = *reinterpret_cast<const uint4*>(box + sw128_off(rr, 4 * (k & 1) + c));
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[j]));
+              v[8 * c + 2 * j] = f.x;
+              v[8 * c + 2 * j + 1] = f.y;
+            }
+          }
+          float amax = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+          // floor(log2 amax) from the bits (a bf16 value: normal, subnormal or 0)
+          const uint32_t ab = __float_as_uint(amax);
+          const int fl = ab >= 0x00800000u ? static_cast<int>(ab >> 23) - 127 : (31 - __clz(ab)) - 149;
+          const int e = ab ? max(-127, min(127, fl - 2)) : -127;
+          // 2^-e is a normal float (e <= 125 for bf16 inputs); x * 2^-e is
+          // exact unless it underflows, where E2M1 gives 0 either way
+          const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+          uint32_t packed[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float a = v[2 * j] * inv, b = v[2 * j + 1] * inv;
+            uint32_t byte = e2m1x2_rn_sat(fabsf(a), fabsf(b));
+            byte |= (__float_as_uint(a) >> 31) << 3;
+            byte |= (__float_as_uint(b) >> 31) << 7;
+            packed[j >> 2] |= byte << (8 * (j & 3));
+          }
+          *reinterpret_cast<uint4*>(q4 + sw64_off(rr, k)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          sfb[(rr >> 7) * 512 + sf_chunk_off(rr & 127, k)] = static_cast<uint8_t>(e + 127);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q4_bar);
+    };
+    // index-Q first when it is there from the start; otherwise (it may
+    // arrive only once the previous kernel has finished) the first ring of
+    // stages is repacked before it is needed
+    bool q_done = false;
+    if (ntiles > 0 && (p.early_q || p.pool_mode)) { quantize_q(); q_done = true; }
     for (int t = 0; t < ntiles; ++t) {
+      if (!q_done && t == min(p.stages, ntiles)) { quantize_q(); q_done = true; }
       const int r = t % Rc, st = t % p.stages;
       bool okc = mbar_wait(&rfull_bar[r], (t / Rc) & 1, kErrWaitTmaFull, abort_flag);
       okc = okc && mbar_wait(&empty_bar[st], ((t / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag);
       if (!__all_sync(0xffffffffu, okc)) break;
-      const uint8_t* src = smem + L.raw0 + r * kRawStageBytes + crow * 68;
-      uint32_t wv[16];
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(smem + L.raw0 + r * kRawStageBytes + crow * 68);
+      uint32_t wv[17];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) wv[k] = *reinterpret_cast<const uint32_t*>(src + 4 * k);
-      const uint32_t scw = *reinterpret_cast<const uint32_t*>(src + 64);
-      uint8_t* stage = smem + L.stage0 + st * kStageBytes;
+      for (int k = 0; k < 17; ++k) wv[k] = src[k];
+      uint8_t* stage = smem + L.stage0 + st * kF4StageBytes;
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        // 2^(code - 127) as bf16: exponent field = code; code 0 is 2^-127,
-        // the subnormal 0x0040
-        const uint32_t c = (scw >> (8 * blk)) & 0xFFu;
-        const uint32_t bits = c ? (c << 7) : 0x40u;
-        const uint32_t pair = bits | (bits << 16);
-        const __nv_bfloat162 S = *reinterpret_cast<const __nv_bfloat162*>(&pair);
-        uint8_t* box = stage + (blk >> 1) * (kStageBytes / 2);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t o[4];
-          e2m1x8_to_bf16(wv[4 * blk + k], S, o);        // channels 32 blk + 8k .. + 7
-          *reinterpret_cast<uint4*>(box + sw128_off(crow, 4 * (blk & 1) + k)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      }
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(stage + sw64_off(crow, c)) = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+      // the entry's scale bytes are its 4 K blocks in order: one word
+      *reinterpret_cast<uint32_t*>(stage + kF4NibBytes + sf_chunk_off(crow, 0)) = wv[16];
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
@@ -323,6 +434,7 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
         mbar_arrive(&rempty_bar[r]);
       }
     }
+    if (!q_done && ntiles > 0) quantize_q();       // with no tiles nothing loads index-Q
   } else {
     // ------------------------------------------------------------ epilogue
     pdl_wait();                                   // before w and the first score store

@@ -29,17 +29,6 @@ __device__ __forceinline__ uint32_t e4m3_rn_sat(float v) {
   return out & 0xFF;
 }
 
-// Two magnitudes to E2M1 (round to nearest even, saturate at 6): `lo` lands
-// in bits 0-3, `hi` in bits 4-7.
-__device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
-      "cvt.u32.u8 %0, b;\n\t}"
-      : "=r"(out) : "f"(hi), "f"(lo));
-  return out & 0xFF;
-}
-
 // One block of 16 channels (fp32 values) to its 8 nibble bytes and E4M3
 // scale code: sf = amax / 6, s = E4M3(sf), q = E2M1(x / s), sign kept.
 __device__ __forceinline__ void fp4_block16(const float (&v)[16], uint2& nib, uint32_t& s_code) {

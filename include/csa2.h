@@ -212,9 +212,12 @@ csa2_status csa2_quantize_index_k_mxfp4(const void* x, int64_t n, int64_t ld_x,
  *   (ascending positions for an ascending pool).
  *
  * k_format CSA2_FMT_MXFP4: kI holds 68-byte MXFP4 entries [B][N][68]
- *   (csa2_quantize_index_k_mxfp4; N a multiple of 4) and the scores use the
- *   dequantised index-K, E2M1 x 2^e, which bf16 holds exactly; index-Q stays
- *   bf16.
+ *   (csa2_quantize_index_k_mxfp4; N a multiple of 4).  The page has the
+ *   indexer's Q and K both in FP4, so index-Q (given in bf16) is quantised
+ *   by the same rule inside the call (each head row of 128 dims, blocks of
+ *   32: e = floor(log2 amax) - 2, q = E2M1(x / 2^e)) and the scores are
+ *   those of the dequantised Q and K, computed on the block-scaled FP4
+ *   tensor cores with fp32 accumulation.
  * ---------------------------------------------------------------------- */
 typedef struct csa2_index_args {
     int32_t        mode;        /* CSA2_FULL, CSA2_REINDEX or CSA2_REINDEX_POOL  */

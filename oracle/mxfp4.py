@@ -24,6 +24,12 @@ E2M1 values and 4 B of scales.  OCP MXFP4 proper is exactly that: one
 
 x / X is a power-of-two scaling, exact in float32 for every bf16 input.
 
+Index-Q: the same page says the indexer's Q and K are both FP4 (quantisation
+aware training), so when index-K is MXFP4 the scores are those of index-Q
+quantised by the same rule (per head row of 128 dims, blocks of 32) and
+dequantised (``fake_quantize``); index-Q is never stored, so only its values
+matter.
+
 Parity: pinned (tests/test_oracle_mxfp4.py) against hand-worked blocks,
 the ml_dtypes float4_e2m1fn conversion of x / X and its float8_e8m0fnu
 decoding of the scale bytes, the exponent rule computed by frexp, and the
@@ -76,3 +82,14 @@ def dequantize_index_k_mxfp4(packed):
     e = packed[:, D_INDEX // 2:].astype(np.float64) - 127.0
     vals = e2m1_value(codes).reshape(n, N_BLOCKS, BLOCK)
     return (vals * np.exp2(e)[..., None]).reshape(n, D_INDEX)
+
+
+def fake_quantize(x):
+    """Rows of 128 values (float32, bf16-representable; any leading shape)
+    through the MXFP4 rule and back: float64 of the same shape.  Used for
+    index-Q, whose scores with an MXFP4 index-K are defined on these values."""
+    x = np.asarray(x, dtype=np.float32)
+    shape = x.shape
+    assert shape[-1] == D_INDEX
+    rows = x.reshape(-1, D_INDEX)
+    return dequantize_index_k_mxfp4(quantize_index_k_mxfp4(rows)).reshape(shape)

@@ -51,6 +51,13 @@ def _index_k_for_oracle(wl, cw, b):
     return k
 
 
+def _index_q_for_oracle(wl, qI):
+    """A query's index-Q as the scores see it: bf16, or MXFP4-quantised when
+    index-K is MXFP4 (the page's FP4 indexer Q and K)."""
+    q = f32(qI)
+    return mxfp4.fake_quantize(q) if wl.index_k_format == 2 else q
+
+
 def _window_for_oracle(wl, swa_b):
     """A layer's window rows of one batch row as the attention sees them."""
     x = f32(swa_b)
@@ -121,7 +128,7 @@ def test_full_size_sampled(w):
                     what = f"{wl.name} group {g} layer {l} b{b} q{q}"
                     nv = int(n_vis[q])
                     if mode in (workloads.FULL, workloads.REINDEX):
-                        s = indexer.index_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, nv)
+                        s = indexer.index_scores(_index_q_for_oracle(wl, li["qI"][b, q]), f32(li["w"][b, q]), kI, nv)
                         check_topk(last_idx[b, q], s, wl.K, what=what)
                         if mode == workloads.FULL and wl.hsi_blocks:
                             bs = indexer.block_scores(s, 8)
@@ -131,7 +138,7 @@ def test_full_size_sampled(w):
                             check_topk(np.concatenate([v[np.argsort(-bs[v], kind="stable")], gp[gp < 0]]), bs,
                                        wl.hsi_blocks, what=what + " pool")
                     elif mode == workloads.REINDEX_POOL:
-                        pos, ps = indexer.pool_scores(f32(li["qI"][b, q]), f32(li["w"][b, q]), kI, pool[b, q], nv)
+                        pos, ps = indexer.pool_scores(_index_q_for_oracle(wl, li["qI"][b, q]), f32(li["w"][b, q]), kI, pool[b, q], nv)
                         check_topk(last_idx[b, q], ps, wl.K, positions=pos, what=what)
                     win = win_b[q * wl.swa_step: q * wl.swa_step + wl.W]
                     o, lse = _attn_oracle(kv_host[(c, b)], last_idx[b, q], f32(li["q"][b, q]), win)

@@ -4,8 +4,9 @@
 * csa2_quantize_index_k_mxfp4: entries bit-exact against oracle.mxfp4;
 * csa2_index_score_topk on those entries (oracle-made bytes): the top-K under
   the band rule of tests/parity.py against the oracle's scores on the
-  dequantised index-K, in Full scans (one to many queries, ragged tails,
-  fewer visible entries than K), with the HSI pool, and pool re-scores.
+  dequantised index-K and the MXFP4-quantised index-Q (the page's FP4
+  indexer Q and K), in Full scans (one to many queries, ragged tails, fewer
+  visible entries than K), with the HSI pool, and pool re-scores.
 """
 
 import numpy as np
@@ -87,7 +88,7 @@ def test_scan_topk_against_dequantised_oracle(B, Q, N, seed, vis):
     idx, sc, _ = _run(0, qI, w, k4, n_vis, K)
     for b in range(B):
         for q in range(Q):
-            s = indexer.index_scores(f32(qI[b, q]), f32(w[b, q]), kdeq[b], int(n_vis[b, q]))
+            s = indexer.index_scores(mxfp4.fake_quantize(f32(qI[b, q])), f32(w[b, q]), kdeq[b], int(n_vis[b, q]))
             sel = check_topk(idx[b, q], s, K, what=f"b{b} q{q}")
             assert np.all(np.diff(sel) > 0)
             np.testing.assert_allclose(sc[b, q, :len(sel)], s[sel], rtol=2e-3, atol=2e-3)
@@ -100,7 +101,7 @@ def test_hsi_pool_and_pool_rescore():
     n_vis = np.array([[N], [N - 13]])
     idx, _, pool = _run(0, qI, w, k4, n_vis, 512, hsi_blocks=400)
     for b in range(B):
-        s = indexer.index_scores(f32(qI[b, 0]), f32(w[b, 0]), kdeq[b], int(n_vis[b, 0]))
+        s = indexer.index_scores(mxfp4.fake_quantize(f32(qI[b, 0])), f32(w[b, 0]), kdeq[b], int(n_vis[b, 0]))
         check_topk(idx[b, 0], s, 512, what=f"full b{b}")
         bs = indexer.block_scores(s, 8)
         v = pool[b, 0][pool[b, 0] >= 0]
@@ -109,7 +110,8 @@ def test_hsi_pool_and_pool_rescore():
                    what=f"pool b{b}")
     idx2, _, _ = _run(2, qI2, w, k4, n_vis, 300, hsi_blocks=400, pool_in=pool)
     for b in range(B):
-        pos, ps = indexer.pool_scores(f32(qI2[b, 0]), f32(w[b, 0]), kdeq[b], pool[b, 0], int(n_vis[b, 0]))
+        pos, ps = indexer.pool_scores(mxfp4.fake_quantize(f32(qI2[b, 0])), f32(w[b, 0]), kdeq[b], pool[b, 0],
+                                      int(n_vis[b, 0]))
         check_topk(idx2[b, 0], ps, 300, positions=pos, what=f"pool rescore b{b}")
 
 
@@ -118,3 +120,27 @@ def test_n_not_a_multiple_of_four_is_refused():
     with pytest.raises(csa2.Csa2Error) as e:
         _run(0, qI, w, np.ascontiguousarray(k4[:, :999]), np.array([[999]]), 64)
     assert e.value.status == 2
+
+
+def test_scores_exact_on_grid_values():
+    """Index-Q and index-K already on their MXFP4 grids with small exponents:
+    every product and partial sum is exact in f32, so the scores the kernel
+    returns equal the oracle's float64 scores exactly, and the selection is
+    compared index for index (ties to the lower position)."""
+    B, Q, N, K = 1, 2, 4000, 256
+    rng = np.random.default_rng(12)
+    kc = rng.integers(0, 16, (N, 128)).astype(np.uint8)
+    qc = rng.integers(0, 16, (B, Q, 32, 128)).astype(np.uint8)
+    kx = mxfp4.e2m1_value(kc) * 0.5
+    qx = mxfp4.e2m1_value(qc) * 0.25
+    k4 = mxfp4.quantize_index_k_mxfp4(kx.astype(np.float32))[None]
+    kdeq = mxfp4.dequantize_index_k_mxfp4(k4[0])
+    qI = torch.from_numpy(qx.astype(np.float32)).to(torch.bfloat16)
+    w = torch.from_numpy(rng.integers(0, 4, (B, Q, 32)).astype(np.float32))
+    n_vis = np.array([[N, N - 777]])
+    idx, sc, _ = _run(0, qI, w, k4, n_vis, K)
+    for q in range(Q):
+        s = indexer.index_scores(mxfp4.fake_quantize(f32(qI[0, q])), f32(w[0, q]), kdeq, int(n_vis[0, q]))
+        want, _ = indexer.topk(s, K)
+        np.testing.assert_array_equal(np.sort(idx[0, q]), np.sort(want))
+        np.testing.assert_array_equal(sc[0, q][np.argsort(idx[0, q])], s[np.sort(want)])

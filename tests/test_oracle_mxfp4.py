@@ -107,3 +107,25 @@ def test_entry_bytes_close_the_890_accounting():
     main = 3 * 288 / 2 + 288
     index = 3 * mxfp4.ENTRY_BYTES / 2 + mxfp4.ENTRY_BYTES
     assert main + index == 890
+
+
+def test_fake_quantize_is_idempotent_and_keeps_grid_values():
+    """Index-Q goes through the same rule: values already on a block's grid
+    (E2M1 x 2^e with the block maximum at 4 or 6 times 2^e) are fixed
+    points, and quantising twice equals quantising once (the block maximum
+    after quantisation is 4 or 6 times 2^e, so the exponent is kept)."""
+    rng = np.random.default_rng(11)
+    x = torch.from_numpy(rng.normal(0, 1, (300, 128)).astype(np.float32) *
+                         np.exp2(rng.integers(-30, 30, (300, 1))).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    once = mxfp4.fake_quantize(x)
+    twice = mxfp4.fake_quantize(once.astype(np.float32))
+    np.testing.assert_array_equal(once, twice)
+    # grid values: codes times 2^e, with the largest magnitude 6 * 2^e
+    e = rng.integers(-20, 20, (50, 4, 1))
+    codes = rng.integers(0, 16, (50, 4, 32)).astype(np.uint8)
+    codes[:, :, 0] = 7
+    grid = (mxfp4.e2m1_value(codes) * np.exp2(e)).reshape(50, 128)
+    np.testing.assert_array_equal(mxfp4.fake_quantize(grid.astype(np.float32)), grid)
+    # any leading shape: [B, Q, 32 heads, 128]
+    q = x[:64].reshape(2, 1, 32, 128)
+    np.testing.assert_array_equal(mxfp4.fake_quantize(q).reshape(64, 128), once[:64])
