@@ -159,9 +159,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int er
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-#ifdef CSA2_WAIT_BACKOFF_NS
-    __nanosleep(CSA2_WAIT_BACKOFF_NS);
-#endif
     if (*abort) return false;
     if (global_ns() - t0 > kWaitLimitNs) {
       record_error(err);

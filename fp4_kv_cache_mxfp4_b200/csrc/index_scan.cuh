@@ -510,8 +510,17 @@ index_scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
           if (!valid) s = -INFINITY;
           const bool in_range = e < p.n_elems && q < qn;
           if (in_range) p.scores[static_cast<int64_t>(bq0 + q) * p.ld + e] = s;
-          if (tile % p.hist_every == 0)                 // uniform over the warp
-            warp_hist_add(hist_s + q * nbins, okey(s) >> (32 - p.hb), in_range && valid);
+          if (tile % p.hist_every == 0) {               // uniform over the warp
+            // decode scores rarely share a bin: one shared atomic per
+            // score; with query blocks (prefill, many near-equal scores)
+            // the warp's increments of a bin are combined first
+            const uint32_t bin = okey(s) >> (32 - p.hb);
+            if (QG <= 2) {
+              if (in_range && valid) atomicAdd(&hist_s[q * nbins + bin], 1u);
+            } else {
+              warp_hist_add(hist_s + q * nbins, bin, in_range && valid);
+            }
+          }
           if (HSI) {
             float m = s;
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
