@@ -69,15 +69,17 @@ inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size
   return e;
 }
 
+// External records: under stream capture they become event-record nodes of
+// the graph (so a replayed graph times its kernels), not capture edges.
 inline void trace_pre(int kid, cudaStream_t st) {
   if (g_trace.on && g_trace.n < g_trace.max) {
     g_trace.kid[g_trace.n] = kid;
-    cudaEventRecord(g_trace.ev[2 * g_trace.n], st);
+    cudaEventRecordWithFlags(g_trace.ev[2 * g_trace.n], st, cudaEventRecordExternal);
   }
 }
 inline void trace_post(cudaStream_t st) {
   if (g_trace.on && g_trace.n < g_trace.max) {
-    cudaEventRecord(g_trace.ev[2 * g_trace.n + 1], st);
+    cudaEventRecordWithFlags(g_trace.ev[2 * g_trace.n + 1], st, cudaEventRecordExternal);
     ++g_trace.n;
   }
 }

@@ -465,8 +465,12 @@ int32_t csa2_version(void);
  * recorded; csa2_trace_get(i, &kernel, &ms) waits for launch i and returns
  * its kernel id and event-measured duration in milliseconds.
  * csa2_trace_end() destroys the events.  Kernel ids name the library's
- * kernels (csa2_kernel_name).  Tracing state is process-global and not
- * synchronised: enable it only while one thread drives the library.
+ * kernels (csa2_kernel_name).  Calls enqueued while their stream is being
+ * captured into a CUDA graph put the event records into the graph (external
+ * event-record nodes): each replay of the graph re-records them, and
+ * csa2_trace_get then returns the durations of the latest replay.  Tracing
+ * state is process-global and not synchronised: enable it only while one
+ * thread drives the library.
  * ---------------------------------------------------------------------- */
 #define CSA2_KERNEL_QUANTIZE     0
 #define CSA2_KERNEL_INDEX_SCAN   1
