@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 from fp4_kv_cache_mxfp4_b200 import build as _build  # noqa: E402
 from fp4_kv_cache_mxfp4_b200 import workloads  # noqa: E402
-from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload, run_step, set_flags  # noqa: E402
+from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload, run_step, set_flags, set_q_format  # noqa: E402
 
 METRIC = "CSA2 decode queries/s and HBM GB/s vs peak at 128K ctx, FP4 main KV"
 UNIT = "queries/s"
@@ -525,6 +525,17 @@ def run_ours(args, world, rank, local):
     mean_ms = time_steps(graphs["model"].replay, args.steps, flush, st, world)
     ready_ms = time_steps(graphs["inputs_ready"].replay, args.steps, flush, st, world)
     serial_ms = time_steps(graphs["serial"].replay, args.steps, flush, st, world)
+    # the same step with quantised attention Q (each layer's q given as FP4
+    # rows; the FP4 tensor path for the selected entries' logits), model
+    # launch order
+    set_q_format(T, csa2.FMT_NVFP4, csa2)
+    qgraph = capture(call(0))
+    for _ in range(args.warmup):
+        flush.zero_()
+        qgraph.replay()
+    quant_q_ms = time_steps(qgraph.replay, args.steps, flush, st, world)
+    del qgraph
+    set_q_format(T, csa2.FMT_BF16, csa2)
 
     # ---- traced step: every launch of one step bracketed by a pair of CUDA
     #      events on its launch stream, captured as one graph and replayed
@@ -645,6 +656,8 @@ def run_ours(args, world, rank, local):
         "ms_per_step_inputs_ready": ready_ms,
         "value_serial": aggregate_queries_per_s(wl.B * wl.Q, world, serial_ms),
         "ms_per_step_serial": serial_ms,
+        "value_quantised_q": aggregate_queries_per_s(wl.B * wl.Q, world, quant_q_ms),
+        "ms_per_step_quantised_q": quant_q_ms,
         "hbm_gbs_step": step_bytes / (mean_ms * 1e-3) / 1e9,
         "hbm_frac_step": step_bytes / (mean_ms * 1e-3) / 1e9 / hbm,
         "roofline": roofline,

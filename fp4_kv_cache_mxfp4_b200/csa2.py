@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libcsa2.so")
 FULL, REINDEX, REINDEX_POOL, REUSE = 0, 1, 2, 3
 WS_INDEX, WS_ATTN, WS_GROUP, WS_STACK = 1, 2, 3, 4
 GROUP_INPUTS_READY, GROUP_SERIAL = 1, 2
-FMT_BF16, FMT_FP8, FMT_MXFP4 = 0, 1, 2
+FMT_BF16, FMT_FP8, FMT_MXFP4, FMT_NVFP4 = 0, 1, 2, 3
 ENTRY_BYTES = 288
 
 _c_i32, _c_i64, _c_f32, _c_p = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
@@ -40,7 +40,7 @@ class AttnArgs(ctypes.Structure):
     _fields_ = [("B", _c_i32), ("Q", _c_i32), ("K", _c_i32), ("W", _c_i32), ("N", _c_i64),
                 ("q", _c_p), ("kv_fp4", _c_p), ("idx", _c_p), ("swa", _c_p),
                 ("swa_rows", _c_i32), ("swa_step", _c_i32), ("scale", _c_f32),
-                ("out", _c_p), ("lse", _c_p), ("swa_format", _c_i32), ("swa_scale", _c_p)]
+                ("out", _c_p), ("lse", _c_p), ("swa_format", _c_i32), ("swa_scale", _c_p), ("q_format", _c_i32)]
 
 
 class Layer(ctypes.Structure):
@@ -54,7 +54,7 @@ class GroupArgs(ctypes.Structure):
                 ("new_rows", _c_p), ("swa_rows", _c_i32), ("swa_step", _c_i32),
                 ("hsi_blocks", _c_i32), ("hsi_block", _c_i32), ("pool", _c_p), ("scale", _c_f32),
                 ("n_layers", _c_i32), ("layers", ctypes.POINTER(Layer)), ("pool_in", _c_p), ("flags", _c_i32),
-                ("swa_format", _c_i32), ("index_k_format", _c_i32)]
+                ("swa_format", _c_i32), ("index_k_format", _c_i32), ("q_format", _c_i32)]
 
 
 class CompressArgs(ctypes.Structure):
@@ -214,15 +214,16 @@ def noalloc_scratch_bytes():
 
 
 def attn_args(q, kv_fp4, idx, swa, out, lse=None, W=128, swa_step=0, scale=0.0, swa_scale=None):
-    """q [B,Q,64,512], kv_fp4 uint8 [B,N,288], idx int32 [B,Q,K], swa bf16
-    [B,rows,512] (or uint8 E4M3 codes [B,rows,512] with swa_scale float32
-    [B,rows]), out bf16 [B,Q,64,512], lse f32 [B,Q,64]."""
+    """q bf16 [B,Q,64,512] (or uint8 [B,Q,64,288] FP4 rows: quantised Q),
+    kv_fp4 uint8 [B,N,288], idx int32 [B,Q,K], swa bf16 [B,rows,512] (or
+    uint8 E4M3 codes [B,rows,512] with swa_scale float32 [B,rows]), out bf16
+    [B,Q,64,512], lse f32 [B,Q,64]."""
     B, Q = q.shape[0], q.shape[1]
     a = AttnArgs(B=B, Q=Q, K=idx.shape[-1] if idx is not None else 0, W=W, N=kv_fp4.shape[1],
                  q=_ptr(q), kv_fp4=_ptr(kv_fp4), idx=_ptr(idx), swa=_ptr(swa),
                  swa_rows=swa.shape[1] if swa is not None else 0, swa_step=swa_step, scale=scale,
                  out=_ptr(out), lse=_ptr(lse), swa_format=FMT_FP8 if swa_scale is not None else FMT_BF16,
-                 swa_scale=_ptr(swa_scale))
+                 swa_scale=_ptr(swa_scale), q_format=FMT_NVFP4 if q.dtype == torch.uint8 else FMT_BF16)
     a._tensors = (q, kv_fp4, idx, swa, out, lse, swa_scale)     # the struct holds raw pointers
     return a
 
@@ -233,11 +234,12 @@ def csa2_sparse_attn(args, ws, stream=None):
 
 
 def group_args(B, Q, K, W, N, n_vis, kI, kv_fp4, layers, kv_new=None, new_rows=None, swa_rows=128, swa_step=0,
-               hsi_blocks=0, hsi_block=8, pool=None, scale=0.0, pool_in=None, flags=0, swa_format=0):
+               hsi_blocks=0, hsi_block=8, pool=None, scale=0.0, pool_in=None, flags=0, swa_format=0, q_format=0):
     """``layers`` is a list of dicts with keys mode, qI, w, q, swa, out, lse,
     idx, scores (tensors or None).  ``pool_in`` is an HSI pool built by an
     earlier group; ``flags`` a combination of GROUP_INPUTS_READY and
-    GROUP_SERIAL; ``swa_format`` FMT_FP8 when every layer's swa holds E4M3
+    GROUP_SERIAL; ``q_format`` FMT_NVFP4 for quantised attention Q;
+    ``swa_format`` FMT_FP8 when every layer's swa holds E4M3
     codes with a ``swa_scale`` tensor.  The returned struct keeps its layer
     array alive."""
     arr = (Layer * len(layers))()
@@ -250,7 +252,8 @@ def group_args(B, Q, K, W, N, n_vis, kI, kv_fp4, layers, kv_new=None, new_rows=N
                   swa_rows=swa_rows, swa_step=swa_step, hsi_blocks=hsi_blocks, hsi_block=hsi_block,
                   pool=_ptr(pool), scale=scale, n_layers=len(layers),
                   layers=ctypes.cast(arr, ctypes.POINTER(Layer)), pool_in=_ptr(pool_in), flags=flags,
-                  swa_format=swa_format, index_k_format=FMT_MXFP4 if kI.dtype == torch.uint8 else FMT_BF16)
+                  swa_format=swa_format, index_k_format=FMT_MXFP4 if kI.dtype == torch.uint8 else FMT_BF16,
+                  q_format=q_format)
     g._layer_array = arr
     # the structs hold raw pointers: keep every tensor alive with them
     g._tensors = (n_vis, kI, kv_fp4, kv_new, new_rows, pool, pool_in, [dict(L) for L in layers])

@@ -36,9 +36,19 @@
 //                  sparse_attn_combine_kernel merges the slices;
 //     one CTA per query: normalised by the running sum, written as bf16 with
 //                  the log-sum-exp.
-// Accumulators: S^T in TMEM columns [0, 64), O^T tile t in [64 + 64t, 128 + 64t).
+// Quantised Q (q_fp4): Q arrives as FP4 rows in the main-KV entry format
+// (E2M1 values, one E4M3 scale per 16 channels, 288 bytes per head; one
+// bulk copy).  A split-mode CTA of an FP4 slice repacks Q's codes and
+// scales and its gathered entries' codes and scales for the block-scaled
+// FP4 tensor path and runs MMA 1 as 8 instructions (tcgen05 kind::mxf4nvf4,
+// K = 64, a UE4M3 scale per 16 values: exactly the cache's format) while
+// its threads expand the entries to bf16 for MMA 2; every other CTA expands
+// Q to bf16 (exact) and runs MMA 1 on that.
+// Accumulators: S^T in TMEM columns [0, 64), O^T tile t in [64 + 64t, 128 + 64t),
+// block scales of the FP4 MMA 1 in [320, 384).
 #pragma once
 #include "common.cuh"
+#include "quantize.cuh"
 #include "attention.cuh"
 
 namespace csa2 {
@@ -75,6 +85,9 @@ struct TcAttnParams {
   float* ml;                 // split: [BQ][slices][64][2]
   __nv_bfloat16* out;        // per query: [BQ][64][512]
   float* lse;                // per query, optional: [BQ][64]
+  int q_fp4;                 // 1: Q given as FP4 rows (the main-KV entry format, 288 B per head);
+                             // in split mode the FP4 slices run MMA 1 on the block-scaled FP4 path
+  const uint8_t* q4;         // q_fp4: [BQ][64][288]
 };
 
 // Shared-memory descriptor of an MN-major operand in the 128-byte-swizzle
@@ -243,15 +256,67 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   // idx comes from the previous kernel, and the partial outputs overwrite a
   // buffer the previous layer's merge reads: those wait for the predecessor
   if (!p.early_inputs) pdl_wait();
+  uint8_t* qstage = kt + 65536;                         // q_fp4: [64][288] FP4 rows (past the gather's staging)
   if (tid == 0) {                                       // this thread initialised the barrier
-    mbar_arrive_expect_tx(&bars[0], kTcQTileBytes);
-    const uint64_t pol = l2_policy_evict_last();
-    for (int c = 0; c < 8; ++c) tma_load_2d(qt + c * 8192, &tmap_q, &bars[0], 64 * c, bq * 64, pol);
+    if (p.q_fp4) {
+      mbar_arrive_expect_tx(&bars[0], 64 * 288);
+      bulk_load(qstage, p.q4 + static_cast<int64_t>(bq) * 64 * 288, 64 * 288, &bars[0]);
+    } else {
+      mbar_arrive_expect_tx(&bars[0], kTcQTileBytes);
+      const uint64_t pol = l2_policy_evict_last();
+      for (int c = 0; c < 8; ++c) tma_load_2d(qt + c * 8192, &tmap_q, &bars[0], 64 * c, bq * 64, pol);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // ---- quantised Q.  The FP4 path's operands live in the Q region: codes
+  //      [64 heads][256 B] (two 128-byte-swizzled boxes), then 8 scale
+  //      chunks (one per MMA step of 64 dims), then the slice's entries
+  //      repacked the same way ([128 keys][256 B] and 8 scale chunks).
+  const bool fp4_mma = p.q_fp4 && !p.per_query && first_slice < p.kv_slices;
+  uint8_t* q4 = qt;
+  uint8_t* sfq = qt + 16384;
+  uint8_t* k4 = qt + 20480;
+  uint8_t* sfk = qt + 53248;
+  // FP4 Q rows -> the FP4 MMA's operands (to_fp4: codes in two
+  // 128-byte-swizzled boxes, scales in 8 chunks, one per MMA step), or the
+  // values expanded to bf16 (exact) into the bf16 Q tile.  Thread t: head
+  // t / 8, dims 64 (t % 8).. (32 code bytes, 4 scales).  Every thread of
+  // the CTA calls it at the same point (it ends with a CTA barrier).
+  auto unpack_q = [&](bool to_fp4) {
+    const bool okq = mbar_wait(&bars[0], 0, kErrWaitOperand, abort_flag);
+    const int h = tid >> 3, part = tid & 7;
+    const uint8_t* row = qstage + h * 288;
+    const uint4 c0 = okq ? *reinterpret_cast<const uint4*>(row + 32 * part) : make_uint4(0, 0, 0, 0);
+    const uint4 c1 = okq ? *reinterpret_cast<const uint4*>(row + 32 * part + 16) : make_uint4(0, 0, 0, 0);
+    const uint32_t scw = okq ? *reinterpret_cast<const uint32_t*>(row + 256 + 4 * part) : 0u;
+    if (to_fp4) {
+      // dims 64 part.. = box part/4, bytes 32 (part % 4).. of the row: chunks 2 (part % 4), +1
+      uint8_t* box = q4 + (part >> 2) * 8192 + (h >> 3) * 1024 + (h & 7) * 128;
+      const int ch = 2 * (part & 3);
+      *reinterpret_cast<uint4*>(box + ((ch ^ (h & 7)) << 4)) = c0;
+      *reinterpret_cast<uint4*>(box + (((ch + 1) ^ (h & 7)) << 4)) = c1;
+      *reinterpret_cast<uint32_t*>(sfq + part * 512 + sf_chunk_off(h, 0)) = scw;
+    } else {
+      // dims 64 part.. = bf16 box part, 16-byte units 0..7 of row h
+      uint8_t* box = qt + part * 8192;
+      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int wd = 0; wd < 8; ++wd) {
+        const float sv = e4m3_code_to_float((scw >> (8 * (wd >> 1))) & 0xFF);   // 16 values per scale
+        uint32_t o[4];
+        e2m1x8_to_bf16(words[wd], __floats2bfloat162_rn(sv, sv), o);
+        *reinterpret_cast<uint4*>(box + sw128_off(h, wd)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+  };
+  // CTAs of the FP4 MMA unpack Q while their entry rows are on the way
+  if (p.q_fp4 && !fp4_mma) unpack_q(false);
 
   for (int it = 0; it < n_iter; ++it) {
     const int slice = first_slice + it;
@@ -339,6 +404,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (vr != 0 && lane < 18)
           raw[j] = __ldg(reinterpret_cast<const uint4*>(p.kv + (static_cast<int64_t>(b) * p.N + (vr - 1)) * 288) + lane);
       }
+      if (fp4_mma && it == 0) unpack_q(true);            // the row loads are in flight meanwhile
       if (lane < 18) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(stage + (8 * warp + j) * 288 + 16 * lane) = raw[j];
@@ -354,7 +420,43 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         nib[k] = *reinterpret_cast<const uint4*>(stage + r * 288 + c * 16);
         sc[k] = *reinterpret_cast<const uint16_t*>(stage + r * 288 + 256 + 2 * c);
       }
+      if (fp4_mma) {
+        // repack for the FP4 MMA 1: thread (key r, quarter qq) moves dims
+        // 128 qq..128 qq+127 (64 nibble bytes: box qq/2, chunks 4(qq%2)..)
+        // and their 8 scales (MMA steps 2qq, 2qq+1: one word each)
+        const int r = tid & (kTcAttnKeys - 1), qq = tid >> 7;
+        const uint8_t* src = stage + r * 288;
+        uint8_t* box = k4 + (qq >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int ch = 4 * (qq & 1) + u;
+          *reinterpret_cast<uint4*>(box + ((ch ^ (r & 7)) << 4)) = *reinterpret_cast<const uint4*>(src + 64 * qq + 16 * u);
+        }
+        const uint2 scw = *reinterpret_cast<const uint2*>(src + 256 + 8 * qq);
+        *reinterpret_cast<uint32_t*>(sfk + (2 * qq) * 512 + sf_chunk_off(r, 0)) = scw.x;
+        *reinterpret_cast<uint32_t*>(sfk + (2 * qq + 1) * 512 + sf_chunk_off(r, 0)) = scw.y;
+        fence_async_smem();
+      }
       __syncthreads();
+      if (fp4_mma && warp == 1 && lane == 0) {
+        // MMA 1 on the FP4 tensor path, while the threads expand the
+        // entries for MMA 2: scale chunks into tensor memory, then 8 steps
+        tc_fence_after();
+        const uint32_t sfq_col = tmem + 320, sfk_col = tmem + 352;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          tmem_cp_sf_chunk(sfq_col + 4 * j, umma_desc_sf_chunk(smem_u32(sfq + 512 * j)));
+          tmem_cp_sf_chunk(sfk_col + 4 * j, umma_desc_sf_chunk(smem_u32(sfk + 512 * j)));
+        }
+        constexpr uint32_t idesc = umma_idesc_nvf4(128, 64);
+        const uint32_t ka = smem_u32(k4), qa = smem_u32(q4);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          umma_nvf4(tmem, umma_desc_sw128_kmajor(ka + (j >> 2) * 16384 + (j & 3) * 32),
+                    umma_desc_sw128_kmajor(qa + (j >> 2) * 8192 + (j & 3) * 32), idesc, sfk_col + 4 * j,
+                    sfq_col + 4 * j, j > 0 ? 1u : 0u);
+        umma_commit(&bars[1]);
+      }
 #pragma unroll
       for (int k = 0; k < kItems; ++k) {
         const int i = tid + k * kTcAttnThreads;
@@ -376,8 +478,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     }
     __syncthreads();
 
-    // ---- MMA 1: S^T = K . Q^T  (M = 128 keys, N = 64 heads, K = 512 dims)
-    if (warp == 1 && lane == 0) {
+    // ---- MMA 1: S^T = K . Q^T  (M = 128 keys, N = 64 heads, K = 512 dims);
+    //      already issued on the FP4 path for quantised Q
+    if (warp == 1 && lane == 0 && !(fp4_mma && !window)) {
       bool ok = mbar_wait(&bars[0], 0, kErrWaitOperand, abort_flag);
       if (ok && window && !p.swa_fp8) ok = mbar_wait(&bars[4], ph_win, kErrWaitOperand, abort_flag);
       if (ok) {

@@ -439,6 +439,25 @@ __device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t adesc, uint6
       :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb) : "memory");
 }
 
+// Instruction descriptor, kind::mxf4nvf4 with 16-value blocks (E2M1 A and
+// B, one UE4M3 scale per 16 values, f32 accumulator, both K-major, K = 64
+// per instruction: 4 scale bytes per row and instruction), shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_nvf4(int M, int N) {
+  return (1u << 7)                                   // A format: E2M1
+       | (1u << 10)                                  // B format: E2M1
+       | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
+       | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16; scale format 0 = UE4M3
+}
+
+__device__ __forceinline__ void umma_nvf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -384,6 +384,7 @@ csa2_status validate_attn(const csa2_attn_args* a) {
       a->K + a->W < 1 || a->N < 1 || a->swa_step < 0)
     return CSA2_ERR_SHAPE;
   if (a->swa_format != CSA2_FMT_BF16 && a->swa_format != CSA2_FMT_FP8) return CSA2_ERR_ARG;
+  if (a->q_format != CSA2_FMT_BF16 && a->q_format != CSA2_FMT_NVFP4) return CSA2_ERR_ARG;
   if (!a->q || !a->out || (a->K > 0 && (!a->kv_fp4 || !a->idx)) || (a->W > 0 && !a->swa)) return CSA2_ERR_ARG;
   if (a->W > 0 && a->swa_format == CSA2_FMT_FP8 && !a->swa_scale) return CSA2_ERR_ARG;
   if (a->W > 0 && static_cast<int64_t>(a->Q - 1) * a->swa_step + a->W > a->swa_rows) return CSA2_ERR_SHAPE;
@@ -459,10 +460,17 @@ csa2_status run_attn(const csa2_attn_args* a, void* ws, cudaStream_t st, bool ea
   t.out = static_cast<__nv_bfloat16*>(a->out);
   t.lse = a->lse;
   t.swa_fp8 = (a->W > 0 && a->swa_format == CSA2_FMT_FP8) ? 1 : 0;
+  t.q_fp4 = a->q_format == CSA2_FMT_NVFP4 ? 1 : 0;
+  t.q4 = static_cast<const uint8_t*>(a->q);
   t.swa8 = static_cast<const uint8_t*>(a->swa);
   t.swa_scale = a->swa_scale;
   CUtensorMap tq, tw;
-  if (!make_map_bf16_512(&tq, a->q, bq * 64, 64)) return CSA2_ERR_CUDA;
+  if (t.q_fp4) {
+    // Q arrives by one bulk copy of FP4 rows; the map is never read
+    if (!make_map_bf16_512(&tq, a->out, bq * 64, 64)) return CSA2_ERR_CUDA;
+  } else if (!make_map_bf16_512(&tq, a->q, bq * 64, 64)) {
+    return CSA2_ERR_CUDA;
+  }
   if (a->W > 0 && !t.swa_fp8) {
     if (!make_map_bf16_512(&tw, a->swa, static_cast<uint64_t>(a->B) * a->swa_rows, kTcAttnKeys)) return CSA2_ERR_CUDA;
   } else {
@@ -514,6 +522,7 @@ csa2_attn_args layer_attn_args(const csa2_group_args* g, const csa2_layer& L, co
   a.swa_rows = g->swa_rows; a.swa_step = g->swa_step; a.scale = g->scale;
   a.out = L.out; a.lse = L.lse;
   a.swa_format = g->swa_format; a.swa_scale = L.swa_scale;
+  a.q_format = g->q_format;
   return a;
 }
 
@@ -866,7 +875,7 @@ const char* csa2_status_string(int32_t s) {
   }
 }
 
-int32_t csa2_version(void) { return 105; }
+int32_t csa2_version(void) { return 106; }
 
 csa2_status csa2_trace_begin(int32_t max_launches) {
   if (max_launches < 1 || max_launches > (1 << 20)) return CSA2_ERR_SHAPE;

@@ -29,6 +29,32 @@ __device__ __forceinline__ uint32_t e4m3_rn_sat(float v) {
   return out & 0xFF;
 }
 
+// The same block quantiser for bf16-valued inputs with one division per
+// block: q = E2M1(x / s) by comparing |x| with the grid's midpoints times s.
+// Both are exact in fp32 (a midpoint has at most 3 significant bits, s at
+// most 4), and for x with 8 significant bits x / s is either exactly a
+// midpoint or at least 2^-8 (relative) away from one, so fp32(x / s) rounds
+// to the same code; ties go to the even code as in round-to-nearest-even.
+__device__ __forceinline__ void fp4_block16_bf16(const float (&v)[16], uint2& nib, uint32_t& s_code) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  s_code = e4m3_rn_sat(__fdiv_rn(amax, 6.0f));
+  const float s = e4m3_code_to_float(s_code);
+  // code >= 1 iff |x| > 0.25 s (tie to 0), >= 2 iff |x| >= 0.75 s (tie to 2), ...
+  const float t1 = 0.25f * s, t2 = 0.75f * s, t3 = 1.25f * s, t4 = 1.75f * s, t5 = 2.5f * s, t6 = 3.5f * s, t7 = 5.0f * s;
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = fabsf(v[i]);
+    uint32_t c = (a > t1) + (a >= t2) + (a > t3) + (a >= t4) + (a > t5) + (a >= t6) + (a > t7);
+    if (s == 0.0f) c = 0;
+    c |= (__float_as_uint(v[i]) >> 31) << 3;
+    packed[i >> 3] |= c << (4 * (i & 7));
+  }
+  nib = make_uint2(packed[0], packed[1]);
+}
+
 // One block of 16 channels (fp32 values) to its 8 nibble bytes and E4M3
 // scale code: sf = amax / 6, s = E4M3(sf), q = E2M1(x / s), sign kept.
 __device__ __forceinline__ void fp4_block16(const float (&v)[16], uint2& nib, uint32_t& s_code) {
@@ -78,7 +104,7 @@ quantize_kv_fp4_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int64_t l
   }
   uint2 nib;
   uint32_t s_code;
-  fp4_block16(v, nib, s_code);
+  fp4_block16_bf16(v, nib, s_code);                   // bf16 inputs: one division per block
   const int64_t dst = dst_rows ? dst_rows[row] : row_offset + row;
   uint8_t* out = kv + dst * 288;
   *reinterpret_cast<uint2*>(out + lane * 8) = nib;

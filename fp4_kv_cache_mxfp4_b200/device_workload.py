@@ -65,7 +65,10 @@ def make_device_workload(wl, csa2, seed_shift=0):
             for b in range(B):
                 csa2.csa2_quantize_window_fp8(swa[b], codes[b], swa_scale[b])
             swa = codes
-        layers.append(dict(mode=mode, qI=li["qI"].to(d), w=li["w"].to(d), q=li["q"].to(d), swa=swa,
+        q = li["q"].to(d)
+        q4 = torch.empty(B, Q, 64, 288, dtype=torch.uint8, device=d)      # the same q as FP4 rows
+        csa2.csa2_quantize_kv_fp4(q.reshape(-1, 512), q4.view(-1, 288))
+        layers.append(dict(mode=mode, qI=li["qI"].to(d), w=li["w"].to(d), q=q, q4=q4, swa=swa,
                            swa_scale=swa_scale, out=torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=d),
                            lse=torch.empty(B, Q, 64, device=d),
                            idx=torch.empty(B, Q, K, dtype=torch.int32, device=d) if mode != workloads.REUSE else None))
@@ -104,6 +107,19 @@ def set_flags(T, flags):
     else:
         for i in range(len(T["groups"])):
             T["stack"]._group_array[i].flags = flags
+
+
+def set_q_format(T, q_format, csa2):
+    """Attention Q of every layer of a staged step: bf16 rows (FMT_BF16) or
+    their FP4 rows (FMT_NVFP4, quantised Q)."""
+    for G in T["groups"]:
+        for j, L in enumerate(G["layers"]):
+            G["g"]._layer_array[j].q = (L["q4"] if q_format == csa2.FMT_NVFP4 else L["q"]).data_ptr()
+    if T["stack"] is None:
+        T["g"].q_format = q_format
+    else:
+        for i in range(len(T["groups"])):
+            T["stack"]._group_array[i].q_format = q_format
 
 
 def run_step(T, csa2, stream=None):

@@ -77,6 +77,7 @@ typedef enum csa2_status {
 #define CSA2_FMT_BF16     0     /* bf16 values                                  */
 #define CSA2_FMT_FP8      1     /* window rows: E4M3 codes + one f32 scale per row ([eogee] §3.4) */
 #define CSA2_FMT_MXFP4    2     /* index-K: 68-byte OCP MXFP4 entries ([eogee] §3.4) */
+#define CSA2_FMT_NVFP4    3     /* attention Q: quantised by the main-KV FP4 rule    */
 #define CSA2_INDEX_K_MXFP4_BYTES 68   /* 64 B of E2M1 nibbles + 4 E8M0 scales        */
 
 /* Static layer modes, [eogee] §3.2 and §3.3. */
@@ -295,6 +296,15 @@ size_t csa2_noalloc_scratch_bytes(void);
  * [0, swa_rows).  With swa_format CSA2_FMT_FP8 a window key is the
  * dequantised row E4M3(code) * s (csa2_quantize_window_fp8).
  *
+ * q_format CSA2_FMT_NVFP4 (quantised Q; [eogee] §3.4 notes the model itself
+ * avoids depending on native FP4 matmul): q holds u8 [B][Q][64][288], each
+ * head row in the main-KV entry format (E2M1 values, one E4M3 scale per 16
+ * channels; csa2_quantize_kv_fp4 writes it from bf16 rows), and the logits
+ * of every key use the dequantised Q.  The selected-entry logits then run
+ * on the block-scaled FP4 tensor cores straight from Q's and the cache's
+ * codes and scales (split mode; with 128 or more queries Q is expanded to
+ * bf16, exactly, and the bf16 path gives the same logits).
+ *
  * With fewer than 128 queries per call (B*Q) the keys of a query are split
  * into 128-key slices over several CTAs: up to 8 slices (K + W <= 1024)
  * they form one thread-block cluster and merge their results through
@@ -309,7 +319,8 @@ typedef struct csa2_attn_args {
     int32_t        K;           /* idx slots per query, 0..CSA2_MAX_K            */
     int32_t        W;           /* window rows per query, 0..CSA2_MAX_W          */
     int64_t        N;           /* cache rows per batch row                      */
-    const void*    q;           /* bf16 [B][Q][64][512]                          */
+    const void*    q;           /* bf16 [B][Q][64][512] (q_format CSA2_FMT_NVFP4:
+                                   u8 [B][Q][64][288] FP4 rows)                  */
     const void*    kv_fp4;      /* u8   [B][N][288]                              */
     const int32_t* idx;         /* int32 [B][Q][K]                               */
     const void*    swa;         /* bf16 [B][swa_rows][512]                       */
@@ -321,6 +332,7 @@ typedef struct csa2_attn_args {
     int32_t        swa_format;  /* CSA2_FMT_BF16 (swa is bf16) or CSA2_FMT_FP8   */
     const float*   swa_scale;   /* CSA2_FMT_FP8: f32 [B][swa_rows]; swa is then
                                    u8 [B][swa_rows][512] E4M3 codes              */
+    int32_t        q_format;    /* CSA2_FMT_BF16 or CSA2_FMT_NVFP4 (quantised Q)  */
 } csa2_attn_args;
 
 csa2_status csa2_sparse_attn(const csa2_attn_args* a, void* ws,
@@ -390,6 +402,8 @@ typedef struct csa2_group_args {
     int32_t          flags;     /* CSA2_GROUP_* bits                             */
     int32_t          swa_format;/* the layers' window rows: CSA2_FMT_BF16 or _FP8 */
     int32_t          index_k_format; /* kI: CSA2_FMT_BF16 or CSA2_FMT_MXFP4      */
+    int32_t          q_format;  /* every layer's q: CSA2_FMT_BF16, or _NVFP4 with
+                                   q as u8 [B][Q][64][288] FP4 rows               */
 } csa2_group_args;
 
 #define CSA2_GROUP_INPUTS_READY 1

@@ -20,9 +20,19 @@ slice is already rotated in the inputs, so it needs no separate treatment.
 float64 throughout.  Parity: pinned (tests/test_oracle_attention.py) against
 torch's scaled_dot_product_attention on the dense special case, softmax
 normalisation, uniform-score and single-key closed forms.
+
+Quantised Q ([eogee] §3.4 says the model deliberately does not rely on the
+tensor cores' native FP4 matmul, which would need Q in FP4 as well): the
+variant ``quantize_q`` puts every head row of Q through the main-KV rule
+(E2M1 values, one E4M3 scale per 16 channels, s = E4M3(amax / 6)), and the
+attention is then ``sparse_mqa`` on those values for every key, selected
+entries and window rows alike.  Pinned by: grid-valued Q is unchanged (the
+quantiser's idempotence) and the composition of pinned functions.
 """
 
 import numpy as np
+
+from . import fp4
 
 H = 64        # [nxbn] §3.1 num_attention_heads
 D = 512       # [nxbn] §3.1 head_dim
@@ -55,3 +65,11 @@ def sparse_mqa(q, kv_deq, idx, swa_rows, scale=None):
     o = p @ keys
     lse = (m + np.log(l))[:, 0]
     return o, lse
+
+
+def quantize_q(q):
+    """[..., 512] query rows through the main-KV FP4 rule and back
+    (float64, exact dequantised values)."""
+    q = np.asarray(q, dtype=np.float32)
+    rows = q.reshape(-1, q.shape[-1])
+    return fp4.dequantize_kv_fp4(fp4.quantize_kv_fp4(rows)).reshape(q.shape)

@@ -42,7 +42,7 @@ def test_every_declared_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert csa2.version() == 105
+    assert csa2.version() == 106
     assert csa2.status_string(0) == "ok"
     assert "workspace" in csa2.status_string(4)
     assert csa2.status_string(99) == "unknown status"
@@ -125,7 +125,8 @@ def test_index_validation_null_struct(L):
     (dict(q=None), 1), (dict(out=None), 1), (dict(idx=None), 1), (dict(swa=None), 1),
     (dict(B=0), 2), (dict(B=3, Q=30000), 2), (dict(K=-1), 2), (dict(K=0, W=0), 2), (dict(W=1025), 2),
     (dict(swa_rows=100), 2), (dict(Q=2, swa_step=1, swa_rows=128), 2),
-    (dict(out=FAKE + 8), 3), (dict(lse=FAKE + 4), 3),
+    (dict(out=FAKE + 8), 3), (dict(lse=FAKE + 4), 3), (dict(q_format=2), 1), (dict(q_format=4), 1),
+    (dict(q_format=3), 4),             # quantised Q: valid, zero-byte workspace
     (dict(), 4),                       # valid arguments, zero-byte workspace
 ])
 def test_attn_validation(L, kw, status):

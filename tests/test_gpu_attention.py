@@ -42,7 +42,7 @@ def _run(kv, q, swa, idx, W, swa_step, scale=0.0, want_lse=True):
     return out.float().cpu().numpy(), (lse.cpu().numpy() if want_lse else None)
 
 
-def _oracle(kv, q, swa, idx, W, swa_step, scale=None):
+def _oracle(kv, q, swa, idx, W, swa_step, scale=None, quantised_q=False):
     B, Q = q.shape[:2]
     o = np.zeros((B, Q, 64, 512))
     lse = np.zeros((B, Q, 64))
@@ -50,7 +50,8 @@ def _oracle(kv, q, swa, idx, W, swa_step, scale=None):
         deq = fp4.dequantize_kv_fp4(kv[b])
         for i in range(Q):
             rows = f32(swa[b])[i * swa_step: i * swa_step + W]
-            o[b, i], lse[b, i] = attention.sparse_mqa(f32(q[b, i]), deq, idx[b, i], rows, scale)
+            qi = attention.quantize_q(f32(q[b, i])) if quantised_q else f32(q[b, i])
+            o[b, i], lse[b, i] = attention.sparse_mqa(qi, deq, idx[b, i], rows, scale)
     return o, lse
 
 
@@ -102,3 +103,39 @@ def test_no_keys_at_all():
         out, lse = _run(kv, q, swa, idx, 0, 0)
         assert np.all(out == 0)
         assert np.all(np.isneginf(lse))
+
+
+def _q_rows_fp4(q):
+    """Oracle-made FP4 rows of Q (the main-KV entry format per head)."""
+    B, Q = q.shape[:2]
+    return torch.from_numpy(fp4.quantize_kv_fp4(f32(q).reshape(-1, 512)).reshape(B, Q, 64, 288))
+
+
+@pytest.mark.parametrize("B,Q,N,K,W,step,seed,m1", [
+    (2, 1, 1500, 512, 128, 0, 20, 0.0),    # 5 slices in a cluster: FP4 slices on the FP4 tensor path
+    (1, 2, 1500, 1024, 128, 0, 21, 0.05),  # 9 slices: partials and the merge kernel
+    (3, 1, 500, 130, 0, 0, 22, 0.0),       # selected entries only, a 2-key slice
+    (1, 1, 10, 0, 128, 0, 23, 0.0),        # window only (dequantised Q on the bf16 path)
+    (1, 130, 3000, 512, 128, 1, 24, 0.05), # one CTA per query: dequantised Q for every slice
+])
+def test_quantised_q_parity(B, Q, N, K, W, step, seed, m1):
+    """Quantised Q: Q given as FP4 rows; against the oracle's attention on
+    the dequantised Q (the logits of every key use those values)."""
+    kv, q, swa, idx = _case(B, Q, N, K, W, step, seed, minus_one=m1)
+    out, lse = _run(kv, _q_rows_fp4(q), swa, idx, W, step)
+    o_ref, lse_ref = _oracle(kv, q, swa, idx, W, step, quantised_q=True)
+    check_attention(out, o_ref, what="quantised q")
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-3, atol=1e-3)
+
+
+def test_quantised_q_exact_on_grid_values():
+    """Q already on the FP4 grid: the call on its FP4 rows equals the bf16
+    call (the rows hold exactly these values and every product is exact)."""
+    kv, q, swa, idx = _case(2, 1, 1500, 512, 128, 0, 25)
+    codes = np.random.default_rng(25).integers(0, 16, (2, 1, 64, 32, 16)).astype(np.uint8)
+    codes[..., 5] = 7
+    qg = torch.from_numpy((fp4.e2m1_value(codes) * 2.0 ** -6).reshape(2, 1, 64, 512).astype(np.float32)).to(torch.bfloat16)
+    a, la = _run(kv, qg, swa, idx, 128, 0)
+    b, lb = _run(kv, _q_rows_fp4(qg), swa, idx, 128, 0)
+    np.testing.assert_allclose(b, a, rtol=0, atol=2e-3 * np.abs(a).max())
+    np.testing.assert_allclose(lb, la, rtol=1e-5, atol=1e-5)

@@ -93,3 +93,43 @@ def test_skipped_slots_and_permutation():
     oa, _ = attention.sparse_mqa(qo, deq, idx, swa)
     ob, _ = attention.sparse_mqa(qo, deq + c, idx, swa + c)
     np.testing.assert_allclose(ob - oa, np.tile(c, (64, 1)), atol=1e-12)
+
+
+def test_quantize_q_keeps_grid_values_and_changes_others():
+    """Q rows already on the FP4 grid (E2M1 codes times an E4M3 scale per 16
+    channels, each block holding a 6 s element) come back unchanged; other
+    rows move by at most half an E2M1 step of their block's scale."""
+    rng = _rng(21)
+    codes = rng.integers(0, 16, (64, 32, 16)).astype(np.uint8)
+    codes[:, :, 3] = 7
+    scales = rng.integers(0x20, 0x50, (64, 32, 1)).astype(np.uint8)
+    grid = (fp4.e2m1_value(codes) * fp4.e4m3_value(scales)).reshape(64, 512)
+    np.testing.assert_array_equal(attention.quantize_q(grid.astype(np.float32)), grid)
+    q = torch.from_numpy((rng.normal(size=(64, 512)) / np.sqrt(512)).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    qh = attention.quantize_q(q)
+    amax = np.abs(q).reshape(64, 32, 16).max(axis=2, keepdims=True)
+    err = np.abs(qh - q).reshape(64, 32, 16)
+    # half the largest E2M1 gap (1 at the top, 2 between 4 and 6) times s <= amax/6 * (1 + 2^-3)
+    assert np.all(err <= amax / 6 * 1.125 + 1e-30)
+    assert np.any(qh != q)
+
+
+def test_quantised_q_attention_stays_close_to_bf16_q():
+    """Tolerance study for the quantised-Q variant on the workload's
+    distributions (q ~ N(0, 1/512), FP4 entries of N(0, 1) rows, 512
+    selected + 128 window rows): the output moves by a few percent of the
+    value scale, not more (the numbers are recorded in the design notes)."""
+    rng = _rng(22)
+    N = 4096
+    kv = fp4.dequantize_kv_fp4(fp4.quantize_kv_fp4(rng.normal(size=(N, 512)).astype(np.float32)))
+    worst_o, worst_lse = 0.0, 0.0
+    for t in range(4):
+        q = (rng.normal(size=(64, 512)) / np.sqrt(512)).astype(np.float32)
+        idx = rng.choice(N, 512, replace=False)
+        win = rng.normal(size=(128, 512))
+        o, lse = attention.sparse_mqa(q, kv, idx, win)
+        oq, lseq = attention.sparse_mqa(attention.quantize_q(q), kv, idx, win)
+        worst_o = max(worst_o, float(np.max(np.abs(oq - o))))
+        worst_lse = max(worst_lse, float(np.max(np.abs(lseq - lse))))
+    print("quantised-Q deviation: max |o| diff", worst_o, "max |lse| diff", worst_lse)
+    assert worst_o < 0.02 and worst_lse < 0.02
