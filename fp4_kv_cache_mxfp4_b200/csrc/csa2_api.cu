@@ -86,8 +86,8 @@ cudaError_t launch_scan_k(int QG, bool hsi, unsigned grid, size_t smem, cudaStre
     case 9: return launch_scan_t<4, true, KF4>(grid, smem, st, tk, tq, sp);
     default:
       if constexpr (KF4) return cudaErrorInvalidValue;   // plan_index caps MXFP4 groups at 4 queries
-      else return QG * 2 == 16 ? launch_scan_t<8, false, KF4>(grid, smem, st, tk, tq, sp)
-                               : launch_scan_t<8, true, KF4>(grid, smem, st, tk, tq, sp);
+      else return hsi ? launch_scan_t<8, true, KF4>(grid, smem, st, tk, tq, sp)
+                      : launch_scan_t<8, false, KF4>(grid, smem, st, tk, tq, sp);
   }
 }
 cudaError_t launch_scan(int QG, bool hsi, bool kf4, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,

@@ -165,6 +165,28 @@ def test_hsi_pool_and_pool_rescore():
         check_topk(r2["idx"][b, 0], ps, 512, positions=pos, what=f"pool b{b}")
 
 
+@pytest.mark.parametrize("Q", [2, 4, 5, 8])
+def test_hsi_pool_with_query_blocks(Q):
+    """Full scan with the HSI pool for several causal queries per MMA group
+    (2, 4 and 8-query kernels; 5 is a verify block in the 8-query kernel):
+    every query gets its own top-K and its own pool."""
+    B, N = 2, 8 * 900 + 3
+    qI, w, kI = _inputs(B, Q, N, 40 + Q)
+    n_vis = np.array([[N - Q + 1 + i for i in range(Q)], [N - 700 + i for i in range(Q)]])
+    nb = 300
+    r = _run(0, qI, w, kI, n_vis, 512, hsi_blocks=nb)
+    for b in range(B):
+        for q in range(Q):
+            s = _oracle_scores(qI, w, kI, b, q, int(n_vis[b, q]))
+            check_topk(r["idx"][b, q], s, 512, what=f"pos b{b} q{q}")
+            bs = indexer.block_scores(s, 8)
+            pool = r["pool"][b, q]
+            valid = pool[pool >= 0]
+            assert len(valid) == nb and np.all(np.diff(valid) > 0), f"pool b{b} q{q}"
+            check_topk(np.concatenate([valid[np.argsort(-bs[valid], kind="stable")], pool[pool < 0]]), bs, nb,
+                       what=f"blocks b{b} q{q}")
+
+
 def test_pool_with_padding_and_invisible_tail():
     B, Q, N = 1, 2, 4000
     qI, w, kI = _inputs(B, Q, N, 17)
