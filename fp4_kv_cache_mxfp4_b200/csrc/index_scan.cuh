@@ -63,10 +63,7 @@ constexpr int kRawStageBytes = kTileRows * 68;     // MXFP4 index-K: one raw til
 constexpr int kF4NibBytes = kTileRows * 64;        // MXFP4: repacked E2M1 tile, 128 rows x 64 B
 constexpr int kF4StageBytes = kF4NibBytes + 1024;  // + its 512-byte scale chunk, padded to the swizzle alignment
 constexpr int kF4MaxQG = 4;                        // MXFP4: queries per MMA group (TMEM room for scales)
-#ifndef CSA2_F4_RAW_STAGES
-#define CSA2_F4_RAW_STAGES 8
-#endif
-constexpr int kF4RawStages = CSA2_F4_RAW_STAGES;   // MXFP4: raw tiles in flight per CTA (at most)
+constexpr int kF4RawStages = 8;                    // MXFP4: raw tiles in flight per CTA (12-20 measured no faster)
 
 // accumulators in flight: as many as fit the 512 TMEM columns (less the
 // block-scale columns of the MXFP4 path), at most 4
