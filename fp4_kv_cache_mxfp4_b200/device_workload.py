@@ -49,6 +49,26 @@ def _stage_cache(cw, csa2, d):
     return dict(kv=kv, kI=kI, new=new, new_rows=new_rows)
 
 
+def _arena(tensors, d, copy=True):
+    """One device buffer holding every tensor of `tensors` (each at a
+    256-byte aligned offset): returns the buffer and the views, filled with
+    the tensors' values when `copy`.  A step's inputs (or outputs) then
+    move between host and device in one copy."""
+    offs, off = [], 0
+    for t in tensors:
+        off = (off + 255) & ~255
+        offs.append(off)
+        off += t.numel() * t.element_size()
+    buf = torch.empty(max(off, 1), dtype=torch.uint8, device=d)
+    views = []
+    for t, o in zip(tensors, offs):
+        v = buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+        if copy:
+            v.copy_(t)
+        views.append(v)
+    return buf, views
+
+
 def make_device_workload(wl, csa2, seed_shift=0):
     d = "cuda"
     wl = with_seed_shift(wl, seed_shift)
@@ -72,6 +92,18 @@ def make_device_workload(wl, csa2, seed_shift=0):
                            swa_scale=swa_scale, out=torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=d),
                            lse=torch.empty(B, Q, 64, device=d),
                            idx=torch.empty(B, Q, K, dtype=torch.int32, device=d) if mode != workloads.REUSE else None))
+    # the step's inputs (new entries, every layer's qI, w and q) in one
+    # device buffer and every layer's output in another
+    ins = [C["new"] for C in caches] + [L[k] for L in layers for k in ("qI", "w", "q")]
+    in_buf, in_views = _arena(ins, d)
+    for C in caches:
+        C["new"] = in_views.pop(0)
+    for L in layers:
+        for k in ("qI", "w", "q"):
+            L[k] = in_views.pop(0)
+    out_buf, out_views = _arena([L["out"] for L in layers], d, copy=False)
+    for L, v in zip(layers, out_views):
+        L["out"] = v
     n_vis = workloads.n_vis_tensor(wl).to(d)
     groups = []
     pool = None                      # the most recent pool built by a Full layer (handed to later groups)
@@ -97,7 +129,8 @@ def make_device_workload(wl, csa2, seed_shift=0):
     torch.cuda.synchronize()
     C0 = caches[0]
     return dict(wl=wl, g=groups[0]["g"], groups=groups, stack=stack, ws=ws, caches=caches, kv=C0["kv"], kI=C0["kI"],
-                new=C0["new"], new_rows=C0["new_rows"], layers=layers, pool=groups[0]["pool"], n_vis=n_vis)
+                new=C0["new"], new_rows=C0["new_rows"], layers=layers, pool=groups[0]["pool"], n_vis=n_vis,
+                inputs=in_buf, outputs=out_buf)
 
 
 def set_flags(T, flags):
