@@ -290,7 +290,7 @@ def step_algorithmic_bytes(wl):
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("common.cuh", "index_scan.cuh"):
+    for f in ("common.cuh", "index_scan.cuh", "index_scan_t.cuh"):
         h.update(open(os.path.join(ROOT, "fp4_kv_cache_mxfp4_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "quantize.cuh"
 #include "index_scan.cuh"
+#include "index_scan_t.cuh"
 #include "topk.cuh"
 #include "attention.cuh"
 #include "attention_tc.cuh"
@@ -64,7 +65,20 @@ cudaError_t set_scan_attrs_k() {
 }
 cudaError_t set_scan_attrs() {
   const cudaError_t a = set_scan_attrs_k<false>(), b = set_scan_attrs_k<true>();
+  const cudaError_t t[4] = {set_smem_attrs(index_scan_t_kernel<false, false>, kMaxDynSmem),
+                            set_smem_attrs(index_scan_t_kernel<true, false>, kMaxDynSmem),
+                            set_smem_attrs(index_scan_t_kernel<false, true>, kMaxDynSmem),
+                            set_smem_attrs(index_scan_t_kernel<true, true>, kMaxDynSmem)};
+  for (cudaError_t x : t) if (x != cudaSuccess) return x;
   return a != cudaSuccess ? a : b;
+}
+cudaError_t launch_scan_t1(bool hsi, bool kf4, unsigned grid, size_t smem, cudaStream_t st, const CUtensorMap& tk,
+                           const CUtensorMap& tq, const ScanParams& sp) {
+  const dim3 block(kf4 ? kScanThreadsF4 : kScanThreads);
+  if (kf4) return hsi ? launch_ex(index_scan_t_kernel<true, true>, dim3(grid), block, smem, st, 0, tk, tq, sp)
+                      : launch_ex(index_scan_t_kernel<false, true>, dim3(grid), block, smem, st, 0, tk, tq, sp);
+  return hsi ? launch_ex(index_scan_t_kernel<true, false>, dim3(grid), block, smem, st, 0, tk, tq, sp)
+             : launch_ex(index_scan_t_kernel<false, false>, dim3(grid), block, smem, st, 0, tk, tq, sp);
 }
 inline int scan_qg(int qg) { return qg <= 1 ? 1 : qg <= 2 ? 2 : qg <= 4 ? 4 : 8; }
 
@@ -261,12 +275,12 @@ cudaError_t launch_topk(const TopkParams& tp, int problems, const DeviceInfo& de
 // CTA per SM finish first, counting about four tiles of set-up per CTA.
 // Few groups (decode) get one wave over every SM; many groups (prefill) get
 // pieces that keep the last wave nearly full.
-int scan_ctas_per_group(int groups, int tiles, int sms) {
+int scan_ctas_per_group(int groups, int tiles, int sms, int setup_tiles = 4) {
   int best = 1;
   int64_t best_cost = INT64_MAX;
   for (int c = 1; c <= std::min(tiles, 4096); ++c) {
     const int64_t waves = (static_cast<int64_t>(groups) * c + sms - 1) / sms;
-    const int64_t cost = waves * ((tiles + c - 1) / c + 4);
+    const int64_t cost = waves * ((tiles + c - 1) / c + setup_tiles);
     if (cost < best_cost) { best_cost = cost; best = c; }
   }
   return best;
@@ -299,43 +313,76 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.hist_every = P.hist_every;
   sp.qblocks = P.pool ? 1 : (a->Q + P.qg - 1) / P.qg;
   sp.groups = P.pool ? P.BQ : a->B * sp.qblocks;
-  sp.tiles_per_group = static_cast<int>((P.n_elems + kTileRows - 1) / kTileRows);
-  sp.ctas_per_group = scan_ctas_per_group(sp.groups, sp.tiles_per_group, dev.sms);
-  const int QG = scan_qg(P.qg);
-  const uint32_t n_mma = 32u * QG;
-  sp.early_q = early_q ? 1 : 0;
   const bool kf4 = a->k_format == CSA2_FMT_MXFP4;
   const int smem_room = kMaxDynSmem - 1024;
-  int raw = 0;
-  if (kf4) {
-    // MXFP4 index-K: up to kF4RawStages raw tiles (8.5 KB each) in flight
-    // and 4 repacked stages (9 KB each) for the MMA
-    sp.k4 = static_cast<const uint8_t*>(a->kI);
-    sp.stages = 4;
-    raw = kF4RawStages;
-    while (raw > 2 && static_cast<int>(scan_smem_layout(sp.stages, QG, P.hb, P.hsi, raw).total) > smem_room) --raw;
+  sp.early_q = early_q ? 1 : 0;
+  if (P.qg == 1) {
+    // one query per group (decode, or the HSI pool re-score): the scan with
+    // the entries on the MMA's N side, 256 per instruction
+    const int tile_t = scan_t_tile(kf4);
+    sp.tiles_per_group = static_cast<int>((P.n_elems + tile_t - 1) / tile_t);
+    sp.ctas_per_group = scan_ctas_per_group(sp.groups, sp.tiles_per_group, dev.sms, 2);
+    int raw = 0;
+    if (kf4) {
+      // 6 raw tiles (13 KB each) in flight: 12 measured no faster, the
+      // tensor pipe (two block-scale copies and two MMAs per tile) sets the pace
+      sp.k4 = static_cast<const uint8_t*>(a->kI);
+      sp.stages = 4;
+      raw = 6;
+      while (raw > 2 && static_cast<int>(scan_t_smem_layout(sp.stages, P.hb, P.hsi, true, raw).total) > smem_room) --raw;
+    } else {
+      sp.stages = 2;                                // 2 x 64 KB in flight
+    }
+    sp.raw_stages = raw;
+    const ScanTSmem L = scan_t_smem_layout(sp.stages, P.hb, P.hsi, kf4, raw);
+    if (static_cast<int>(L.total) > smem_room) return CSA2_ERR_SHAPE;
+    sp.tmem_cols = scan_t_tmem_cols(kf4, sp.stages);
+    CUtensorMap tk, tq;
+    if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, 32)) return CSA2_ERR_CUDA;
+    if (kf4) tk = tq;                               // not read: index-K arrives by bulk copies
+    else if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : tile_t))
+      return CSA2_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(sp.groups * sp.ctas_per_group);
+    trace_pre(kKIndexScan, st);
+    const cudaError_t es = launch_scan_t1(P.hsi, kf4, grid, L.total + 1024, st, tk, tq, sp);
+    trace_post(st);
+    if (es != cudaSuccess) return CSA2_ERR_CUDA;
   } else {
-    // three 32 KB stages per SM measured fastest (fewer bytes in flight per
-    // stream keep DRAM pages open longer; 2, 4 and 6 stages were slower)
-    const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi, 0);
-    sp.stages = std::min(kScanStages, static_cast<int>((smem_room - L0.total) / (kStageBytes + 16)));
-    if (sp.stages < 2) return CSA2_ERR_SHAPE;
-  }
-  sp.raw_stages = raw;
-  const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi, raw);
-  if (static_cast<int>(L.total) > smem_room) return CSA2_ERR_SHAPE;
-  sp.tmem_cols = scan_tmem_cols(QG, kf4, sp.stages);
-  CUtensorMap tk, tq;
-  if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, n_mma)) return CSA2_ERR_CUDA;
-  if (kf4) tk = tq;                                 // not read: index-K arrives by bulk copies
-  else if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : kTileRows))
-    return CSA2_ERR_CUDA;
+    sp.tiles_per_group = static_cast<int>((P.n_elems + kTileRows - 1) / kTileRows);
+    sp.ctas_per_group = scan_ctas_per_group(sp.groups, sp.tiles_per_group, dev.sms);
+    const int QG = scan_qg(P.qg);
+    const uint32_t n_mma = 32u * QG;
+    int raw = 0;
+    if (kf4) {
+      // MXFP4 index-K: up to kF4RawStages raw tiles (8.5 KB each) in flight
+      // and 4 repacked stages (9 KB each) for the MMA
+      sp.k4 = static_cast<const uint8_t*>(a->kI);
+      sp.stages = 4;
+      raw = kF4RawStages;
+      while (raw > 2 && static_cast<int>(scan_smem_layout(sp.stages, QG, P.hb, P.hsi, raw).total) > smem_room) --raw;
+    } else {
+      // three 32 KB stages per SM measured fastest (fewer bytes in flight per
+      // stream keep DRAM pages open longer; 2, 4 and 6 stages were slower)
+      const ScanSmem L0 = scan_smem_layout(0, QG, P.hb, P.hsi, 0);
+      sp.stages = std::min(kScanStages, static_cast<int>((smem_room - L0.total) / (kStageBytes + 16)));
+      if (sp.stages < 2) return CSA2_ERR_SHAPE;
+    }
+    sp.raw_stages = raw;
+    const ScanSmem L = scan_smem_layout(sp.stages, QG, P.hb, P.hsi, raw);
+    if (static_cast<int>(L.total) > smem_room) return CSA2_ERR_SHAPE;
+    sp.tmem_cols = scan_tmem_cols(QG, kf4, sp.stages);
+    CUtensorMap tk, tq;
+    if (!make_map_bf16_128(&tq, a->qI, static_cast<uint64_t>(P.BQ) * 32, n_mma)) return CSA2_ERR_CUDA;
+    if (kf4) tk = tq;                                 // not read: index-K arrives by bulk copies
+    else if (!make_map_bf16_128(&tk, a->kI, static_cast<uint64_t>(a->B) * a->N, P.pool ? 8 : kTileRows))
+      return CSA2_ERR_CUDA;
 
-  const unsigned grid = static_cast<unsigned>(sp.groups * sp.ctas_per_group);
-  trace_pre(kKIndexScan, st);
-  const cudaError_t es = launch_scan(QG, P.hsi, kf4, grid, L.total + 1024, st, tk, tq, sp);
-  trace_post(st);
-  if (es != cudaSuccess) return CSA2_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(sp.groups * sp.ctas_per_group);
+    trace_pre(kKIndexScan, st);
+    const cudaError_t es = launch_scan(QG, P.hsi, kf4, grid, L.total + 1024, st, tk, tq, sp);
+    trace_post(st);
+    if (es != cudaSuccess) return CSA2_ERR_CUDA;
+  }
 
   TopkParams tp;
   memset(&tp, 0, sizeof(tp));
