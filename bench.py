@@ -44,10 +44,10 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
-# DRAM traffic (read + write) of one index_scan_kernel launch of the
-# default workload, from an ncu capture of that kernel (profiles/), valid
-# only while the scan's sources hash to the recorded value.
-SCAN_TRAFFIC = {"sha": "71042d82f35fc3a5", "bytes_per_launch": 138179584}
+# DRAM traffic (read + write) of one decode scan launch (index_scan_t_kernel)
+# of the default workload, from an ncu capture of that kernel (profiles/),
+# valid only while the scan's sources hash to the recorded value.
+SCAN_TRAFFIC = {"sha": "cdb8913912dfdac0", "bytes_per_launch": 137816832}
 
 
 def parse():
@@ -249,6 +249,16 @@ def label_launches(wl, names):
         else:
             labels.append(n)
     return labels
+
+
+def scan_kernel_name(wl, label):
+    """The scan kernel a launch label runs: one query per MMA group (a
+    decode row, or a pool re-score) takes the transposed kernel
+    index_scan_t_kernel; several queries per group index_scan_kernel.  The
+    launch trace names both index_scan_kernel."""
+    if label == "scan_pool" or (label == "scan" and wl.Q == 1):
+        return "index_scan_t_kernel"
+    return "index_scan_kernel"
 
 
 def label_work(wl, label):
@@ -569,6 +579,8 @@ def run_ours(args, world, rank, local):
         if labels is None:
             labels = label_launches(wl, [n for n, _ in recs])
         for i, (name, ms) in enumerate(recs):
+            if labels[i].startswith("scan"):
+                name = scan_kernel_name(wl, labels[i])
             c, t, _ = per_label.get(labels[i], (0, 0.0, name))
             per_label[labels[i]] = (c + 1, t + ms, name)
     barrier(world)

@@ -202,7 +202,7 @@ struct IndexPlan {
   int64_t ld, bld;     // score row strides (multiples of 4 for 16-byte loads)
   // counter region (histograms): zeroed at the start of every call; data
   // region (scores): no precondition
-  size_t off_hist, off_bhist, zero_bytes;
+  size_t off_hist, off_bhist, off_ctr, zero_bytes;
   size_t off_scores, off_bscores, data_bytes;
   size_t total;
 };
@@ -252,6 +252,8 @@ IndexPlan plan_index(const csa2_index_args* a) {
   size_t off = 0;
   P.off_hist = off;    off = up256(off + static_cast<size_t>(P.BQ) * nb * 4);
   P.off_bhist = off;   off = up256(off + (P.hsi ? static_cast<size_t>(P.BQ) * nb * 4 : 0));
+  // tile claims of the one-query-per-group scan, one counter per query
+  P.off_ctr = off;     off = up256(off + (P.qg == 1 ? static_cast<size_t>(P.BQ) * 4 : 0));
   P.zero_bytes = off;
   off = 0;
   P.off_scores = off;  off = up256(off + static_cast<size_t>(P.BQ) * P.ld * 4);
@@ -309,6 +311,7 @@ csa2_status run_index(const csa2_index_args* a, const DeviceInfo& dev, void* zer
   sp.nblk = P.nblk;
   sp.hist = reinterpret_cast<uint32_t*>(z + P.off_hist);
   sp.bhist = P.hsi ? reinterpret_cast<uint32_t*>(z + P.off_bhist) : nullptr;
+  sp.tile_ctr = reinterpret_cast<int*>(z + P.off_ctr);
   sp.hb = P.hb;
   sp.hist_every = P.hist_every;
   sp.qblocks = P.pool ? 1 : (a->Q + P.qg - 1) / P.qg;

@@ -109,6 +109,8 @@ struct ScanParams {
                           // the predecessor); 0: they may be the predecessor's results
   const uint8_t* k4;      // MXFP4 index-K: [B*N][68] entries (N a multiple of 4)
   int raw_stages;         // MXFP4 index-K: raw tiles in flight
+  int* tile_ctr;          // one query per group: [groups] tiles claimed past the first
+                          // ctas_per_group (zero at launch)
 };
 
 struct ScanSmem {

@@ -31,6 +31,15 @@
 //                  for the scales while the MMA of one tile overlaps the
 //                  epilogue of the other).
 //
+// Tiles are claimed, not assigned: CTA c of a query's group starts with
+// tile c and then takes the next unclaimed one from the query's counter
+// (one atomic per tile, claimed a tile ahead).  Under programmatic
+// dependent launch the CTAs whose SMs are still held by the previous
+// kernel start tens of microseconds late; with a fixed share of the tiles
+// they, not the bandwidth, set the end of the scan.  The producer passes
+// each tile's id beside its stage (a negative id ends the stream), the
+// MMA thread beside its accumulator.
+//
 // Warp roles as in index_scan.cuh.  HBM roofline: the same bytes per entry.
 #pragma once
 #include "index_scan.cuh"
@@ -48,7 +57,7 @@ constexpr int kTRawBytes = 192 * 68;                 // MXFP4: one raw tile of 6
 __host__ __device__ inline uint32_t scan_t_tmem_cols(bool, int) { return 512u; }
 
 struct ScanTSmem {
-  uint32_t stage0, raw0, qa0, qi0, sfa0, w0, hist0, bhist0, bar0, total;
+  uint32_t stage0, raw0, qa0, qi0, sfa0, w0, hist0, bhist0, bar0, tid0, total;
 };
 
 // stages / raw_stages: repacked (or bf16) stages and MXFP4 raw tiles
@@ -66,6 +75,7 @@ __host__ __device__ inline ScanTSmem scan_t_smem_layout(int stages, int hb, int 
   L.bhist0 = off; off += hsi ? (1u << hb) * 4 : 0;
   off = (off + 15) & ~15u;
   L.bar0 = off;   off += (2 * stages + 2 * 2 + 2 * raw_stages + 2) * 8 + 16 + 64;
+  L.tid0 = off;   off += (stages + raw_stages + 2) * 4;   // tile ids of the stages, raw tiles, accumulators
   L.total = off;
   return L;
 }
@@ -101,30 +111,96 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int cig = blockIdx.x % p.ctas_per_group;
   const int b = bq0 / p.Q;
   const int nbins = 1 << p.hb;
+  volatile int* stile = reinterpret_cast<volatile int*>(smem + L.tid0);   // tile of each stage
+  volatile int* rtile = stile + p.stages;                                 // MXFP4: tile of each raw slot
+  volatile int* acc_tile = rtile + R;                                     // tile of each accumulator
 
+  // tiles of this query: [0, tlim); CTA cig takes tile cig first and then
+  // claims tiles ctas_per_group, ctas_per_group + 1, ... from the query's
+  // counter, so that CTAs that start late (their SM still busy with the
+  // previous kernel) take fewer tiles
+  const int nv = p.n_vis[bq0];
+  const int tlim = p.pool_mode ? p.tiles_per_group : min(p.tiles_per_group, (nv + TILE - 1) / TILE);
+  const int first_tile = cig < tlim ? cig : -1;
+
+  uint64_t pol_stream = 0;
+  // producer step i: wait for the slot, record the tile (or the end marker,
+  // tile < 0), request its index-K
+  auto issue = [&](int i, int tile) -> bool {
+    if constexpr (KF4) {
+      const int r = i % R;
+      if (!mbar_wait(&rempty_bar[r], ((i / R) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag)) return false;
+      rtile[r] = tile;
+      if (tile < 0) { mbar_arrive(&rfull_bar[r]); return true; }
+      uint8_t* dst = smem + L.raw0 + r * kTRawBytes;
+      if (!p.pool_mode) {
+        const int64_t row0 = static_cast<int64_t>(tile) * TILE;
+        const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(TILE), p.N - row0));
+        mbar_arrive_expect_tx(&rfull_bar[r], rows * 68u);
+        bulk_load(dst, p.k4 + (static_cast<int64_t>(b) * p.N + row0) * 68, rows * 68u, &rfull_bar[r]);
+      } else {
+        const int32_t* pool = p.pool + static_cast<int64_t>(bq0) * p.pool_blocks;
+        mbar_arrive_expect_tx(&rfull_bar[r], (TILE / 8) * 544u);
+#pragma unroll 1
+        for (int j = 0; j < TILE / 8; ++j) {
+          const int slot = tile * (TILE / 8) + j;
+          int blk = (slot < p.pool_blocks) ? pool[slot] : -1;
+          if (blk < 0) blk = 0;                      // padding slot: load any block, scores masked
+          bulk_load(dst + j * 544, p.k4 + (static_cast<int64_t>(b) * p.N + static_cast<int64_t>(blk) * 8) * 68,
+                    544u, &rfull_bar[r]);
+        }
+      }
+    } else {
+      const int s = i % p.stages;
+      if (!mbar_wait(&empty_bar[s], ((i / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag)) return false;
+      stile[s] = tile;
+      if (tile < 0) { mbar_arrive(&full_bar[s]); return true; }
+      uint8_t* st = smem + L.stage0 + s * STAGE;
+      mbar_arrive_expect_tx(&full_bar[s], STAGE);
+      if (!p.pool_mode) {
+        const int32_t y = static_cast<int32_t>(static_cast<int64_t>(b) * p.N + static_cast<int64_t>(tile) * TILE);
+        tma_load_2d(st, &tmap_k, &full_bar[s], 0, y, pol_stream);
+        tma_load_2d(st + STAGE / 2, &tmap_k, &full_bar[s], 64, y, pol_stream);
+      } else {
+        const int32_t* pool = p.pool + static_cast<int64_t>(bq0) * p.pool_blocks;
+#pragma unroll 1
+        for (int j = 0; j < TILE / 8; ++j) {
+          const int slot = tile * (TILE / 8) + j;
+          int blk = (slot < p.pool_blocks) ? pool[slot] : -1;
+          if (blk < 0) blk = 0;
+          const int32_t y = static_cast<int32_t>(static_cast<int64_t>(b) * p.N + static_cast<int64_t>(blk) * 8);
+          tma_load_2d(st + j * 1024, &tmap_k, &full_bar[s], 0, y, pol_stream);
+          tma_load_2d(st + STAGE / 2 + j * 1024, &tmap_k, &full_bar[s], 64, y, pol_stream);
+        }
+      }
+    }
+    return true;
+  };
+
+  // the first tile of a full scan is requested before the block-wide set-up
+  // (it needs only the barriers); a pool re-score waits for its pool first
+  const bool early_first = !p.pool_mode && first_tile >= 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) { mbar_init(&full_bar[s], KF4 ? kScanCvtWarps : 1); mbar_init(&empty_bar[s], 1); }
     for (int r = 0; r < R; ++r) { mbar_init(&rfull_bar[r], 1); mbar_init(&rempty_bar[r], kScanCvtWarps); }
-    // one full/empty pair per epilogue set (tile parity), whether the two
-    // sets have an accumulator each (bf16) or share one (MXFP4)
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 1); mbar_init(&tempty_bar[a], 4); }
+    // tfull: the MMA commit and the MMA thread's arrival after it records
+    // the accumulator's tile; tempty: the four warps of the epilogue set
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull_bar[a], 2); mbar_init(&tempty_bar[a], 4); }
     mbar_init(q_bar, 1);
     mbar_init(q4_bar, kScanCvtWarps);
     *abort_flag = 0;
     fence_barrier_init();
+    if (!KF4) tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+    pol_stream = l2_policy_evict_first();
+    if (early_first) issue(0, first_tile);
   }
-  if (warp == 0 && lane == 0) { if (!KF4) tma_prefetch_desc(&tmap_k); tma_prefetch_desc(&tmap_q); }
   if (warp == 1) { tmem_alloc(tmem_slot, p.tmem_cols); tmem_relinquish(); }
   for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist_s[i] = 0;
   if (HSI) for (int i = threadIdx.x; i < nbins; i += blockDim.x) bhist_s[i] = 0;
   // what may start before the predecessor finishes: as in index_scan.cuh
   pdl_launch_dependents();
 
-  int tile_lo = static_cast<int>((static_cast<int64_t>(cig) * p.tiles_per_group) / p.ctas_per_group);
-  int tile_hi = static_cast<int>((static_cast<int64_t>(cig + 1) * p.tiles_per_group) / p.ctas_per_group);
-  const int nv = p.n_vis[bq0];
-  if (!p.pool_mode) tile_hi = min(tile_hi, (nv + TILE - 1) / TILE);
-  const int ntiles = max(0, tile_hi - tile_lo);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -132,9 +208,8 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0 && first_tile >= 0) {
       if (p.pool_mode) pdl_wait();
-      const uint64_t pol_stream = l2_policy_evict_first();
       const uint64_t pol_keep = l2_policy_evict_last();
       // bf16: the 32 head rows straight into the four replicas of each of
       // the A tile's two 128-byte-wide boxes; MXFP4: once, for quantising
@@ -154,77 +229,77 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
               tma_load_2d(qa + c * 16384 + rep * 4096, &tmap_q, q_bar, 64 * c, bq0 * 32, pol_keep);
         }
       };
-      const bool q_late = !p.early_q && !p.pool_mode;
-      if (!q_late) load_q();
+      bool q_loaded = false;
+      if (p.early_q || p.pool_mode) { load_q(); q_loaded = true; }
+      // the slots a late index-Q may trail: the consumers free none before it lands
       const int ring = KF4 ? R : p.stages;
-      for (int i = 0; i < ntiles; ++i) {
-        if (q_late && i == min(ring, ntiles)) { pdl_wait(); load_q(); }
-        const int tile = tile_lo + i;
-        if constexpr (KF4) {
-          const int r = i % R;
-          if (!mbar_wait(&rempty_bar[r], ((i / R) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag)) break;
-          uint8_t* dst = smem + L.raw0 + r * kTRawBytes;
-          if (!p.pool_mode) {
-            const int64_t row0 = static_cast<int64_t>(tile) * TILE;
-            const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(TILE), p.N - row0));
-            mbar_arrive_expect_tx(&rfull_bar[r], rows * 68u);
-            bulk_load(dst, p.k4 + (static_cast<int64_t>(b) * p.N + row0) * 68, rows * 68u, &rfull_bar[r]);
-          } else {
-            const int32_t* pool = p.pool + static_cast<int64_t>(bq0) * p.pool_blocks;
-            mbar_arrive_expect_tx(&rfull_bar[r], (TILE / 8) * 544u);
-#pragma unroll 1
-            for (int j = 0; j < TILE / 8; ++j) {
-              const int slot = tile * (TILE / 8) + j;
-              int blk = (slot < p.pool_blocks) ? pool[slot] : -1;
-              if (blk < 0) blk = 0;                  // padding slot: load any block, scores masked
-              bulk_load(dst + j * 544, p.k4 + (static_cast<int64_t>(b) * p.N + static_cast<int64_t>(blk) * 8) * 68,
-                        544u, &rfull_bar[r]);
-            }
-          }
-        } else {
-          const int s = i % p.stages;
-          if (!mbar_wait(&empty_bar[s], ((i / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag)) break;
-          uint8_t* st = smem + L.stage0 + s * STAGE;
-          mbar_arrive_expect_tx(&full_bar[s], STAGE);
-          if (!p.pool_mode) {
-            const int32_t y = static_cast<int32_t>(static_cast<int64_t>(b) * p.N + static_cast<int64_t>(tile) * TILE);
-            tma_load_2d(st, &tmap_k, &full_bar[s], 0, y, pol_stream);
-            tma_load_2d(st + STAGE / 2, &tmap_k, &full_bar[s], 64, y, pol_stream);
-          } else {
-            const int32_t* pool = p.pool + static_cast<int64_t>(bq0) * p.pool_blocks;
-#pragma unroll 1
-            for (int j = 0; j < TILE / 8; ++j) {
-              const int slot = tile * (TILE / 8) + j;
-              int blk = (slot < p.pool_blocks) ? pool[slot] : -1;
-              if (blk < 0) blk = 0;
-              const int32_t y = static_cast<int32_t>(static_cast<int64_t>(b) * p.N + static_cast<int64_t>(blk) * 8);
-              tma_load_2d(st + j * 1024, &tmap_k, &full_bar[s], 0, y, pol_stream);
-              tma_load_2d(st + STAGE / 2 + j * 1024, &tmap_k, &full_bar[s], 64, y, pol_stream);
-            }
-          }
-        }
+      auto claim = [&]() { return p.ctas_per_group + atomicAdd(p.tile_ctr + bq0, 1); };
+      int i = 0;
+      // producer step with the tile a claim returned: claim again in its
+      // place, issue; false once the stream has ended
+      auto step = [&](int& c) -> bool {
+        const int tile = c < tlim ? c : -1;
+        if (tile >= 0) c = claim();
+        if (!q_loaded && i == ring) { pdl_wait(); load_q(); q_loaded = true; }
+        const bool go = issue(i, tile) && tile >= 0;
+        ++i;
+        return go;
+      };
+      bool go = true;
+      if (early_first) {
+        i = 1;
+      } else {
+        if (!q_loaded && i == ring) { pdl_wait(); load_q(); q_loaded = true; }
+        go = issue(0, first_tile);
+        i = 1;
       }
-      if (q_late && ntiles <= ring) { pdl_wait(); load_q(); }
+      if constexpr (KF4) {
+        // four claims in flight (separate registers, oldest first), so that
+        // filling the six-tile raw ring does not wait on one atomic per tile
+        int c0 = claim(), c1 = claim(), c2 = claim(), c3 = claim();
+        while (go && step(c0) && step(c1) && step(c2) && step(c3)) {}
+      } else {
+        int c0 = claim();                           // one claim ahead
+        while (go && step(c0)) {}
+      }
+      if (!q_loaded) { pdl_wait(); load_q(); }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0 && first_tile >= 0) {
       const uint32_t qa_addr = smem_u32(smem + L.qa0);
-      if constexpr (KF4) {
-        const uint32_t sfa_col = tmem_base + 2 * TILE;
-        const uint32_t sfb_col = sfa_col + 4;
-        bool ok = mbar_wait(q4_bar, 0, kErrWaitOperand, abort_flag);
-        if (ok) {
-          tc_fence_after();
-          tmem_cp_sf_chunk(sfa_col, umma_desc_sf_chunk(smem_u32(smem + L.sfa0)));
+      const uint32_t sfa_col = tmem_base + 2 * TILE;      // MXFP4 scale columns
+      const uint32_t sfb_col = sfa_col + 4;
+      // local tile i is the end marker: it closes both epilogue sets
+      auto close_sets = [&](int i) {
+#pragma unroll 1
+        for (int k = 0; k < 2; ++k) {
+          const int ii = i + k, a = ii & 1;
+          if (k > 0 && !mbar_wait(&tempty_bar[a], ((ii >> 1) & 1) ^ 1, kErrWaitTmemEmpty, abort_flag)) return;
+          acc_tile[a] = -1;
+          mbar_arrive(&tfull_bar[a]);
+          mbar_arrive(&tfull_bar[a]);
         }
-        for (int i = 0; ok && i < ntiles; ++i) {
-          const int s = i % p.stages;
-          const int a = i & 1;
-          if (!mbar_wait(&tempty_bar[a], ((i >> 1) & 1) ^ 1, kErrWaitTmemEmpty, abort_flag)) break;
-          if (!mbar_wait(&full_bar[s], (i / p.stages) & 1, kErrWaitTmaFull, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t st_addr = smem_u32(smem + L.stage0 + s * STAGE);
+      };
+      bool have_q = false;
+      for (int i = 0;; ++i) {
+        const int s = i % p.stages;
+        const int a = i & 1;
+        if (!mbar_wait(&full_bar[s], (i / p.stages) & 1, kErrWaitTmaFull, abort_flag)) break;
+        const int tile = stile[s];
+        if (!mbar_wait(&tempty_bar[a], ((i >> 1) & 1) ^ 1, kErrWaitTmemEmpty, abort_flag)) break;
+        if (tile < 0) { close_sets(i); break; }
+        if (!have_q) {
+          if (!mbar_wait(KF4 ? q4_bar : q_bar, 0, kErrWaitOperand, abort_flag)) break;
+          have_q = true;
+          if constexpr (KF4) {
+            tc_fence_after();
+            tmem_cp_sf_chunk(sfa_col, umma_desc_sf_chunk(smem_u32(smem + L.sfa0)));
+          }
+        }
+        tc_fence_after();
+        const uint32_t st_addr = smem_u32(smem + L.stage0 + s * STAGE);
+        if constexpr (KF4) {
           tmem_cp_sf_chunk(sfb_col + 8 * s, umma_desc_sf_chunk(st_addr + TILE * 64));
           tmem_cp_sf_chunk(sfb_col + 8 * s + 4, umma_desc_sf_chunk(st_addr + TILE * 64 + 512));
 #pragma unroll
@@ -232,19 +307,8 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
             umma_mxf4(tmem_base + a * TILE, umma_desc_sw64_kmajor(qa_addr + 32 * ks),
                       umma_desc_sw64_kmajor(st_addr + 32 * ks), umma_idesc_mxf4(128, TILE, 2u * ks), sfa_col,
                       sfb_col + 8 * s, ks > 0 ? 1u : 0u);
-          umma_commit(&empty_bar[s]);
-          umma_commit(&tfull_bar[a]);
-        }
-      } else {
-        constexpr uint32_t idesc = umma_idesc_bf16_f32(128, TILE);
-        bool ok = mbar_wait(q_bar, 0, kErrWaitOperand, abort_flag);
-        for (int i = 0; ok && i < ntiles; ++i) {
-          const int s = i % p.stages;
-          const int a = i & 1;
-          if (!mbar_wait(&tempty_bar[a], ((i >> 1) & 1) ^ 1, kErrWaitTmemEmpty, abort_flag)) break;
-          if (!mbar_wait(&full_bar[s], (i / p.stages) & 1, kErrWaitTmaFull, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t st_addr = smem_u32(smem + L.stage0 + s * STAGE);
+        } else {
+          constexpr uint32_t idesc = umma_idesc_bf16_f32(128, TILE);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             // K step kk covers dims 16kk..16kk+15: box kk/4, 32-byte column (kk%4)
@@ -252,9 +316,11 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       umma_desc_sw128_kmajor(st_addr + (kk >> 2) * (STAGE / 2) + (kk & 3) * 32), idesc,
                       kk > 0 ? 1u : 0u);
           }
-          umma_commit(&empty_bar[s]);
-          umma_commit(&tfull_bar[a]);
         }
+        umma_commit(&empty_bar[s]);
+        acc_tile[a] = tile;
+        umma_commit(&tfull_bar[a]);
+        mbar_arrive(&tfull_bar[a]);
       }
     }
   } else if (KF4 && warp >= 2 + kScanEpiWarps) {
@@ -309,13 +375,23 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
       if (lane == 0) mbar_arrive(q4_bar);
     };
     bool q_done = false;
-    if (ntiles > 0 && (p.early_q || p.pool_mode)) { quantize_q(); q_done = true; }
-    for (int t = 0; t < ntiles; ++t) {
-      if (!q_done && t == min(p.stages, ntiles)) { quantize_q(); q_done = true; }
+    int t = 0;
+    for (; first_tile >= 0; ++t) {
+      // a late index-Q: once every stage holds a tile, the MMA needs it to go on
+      if (!q_done && t == p.stages) { quantize_q(); q_done = true; }
       const int r = t % Rc, st = t % p.stages;
       bool okc = mbar_wait(&rfull_bar[r], (t / Rc) & 1, kErrWaitTmaFull, abort_flag);
-      okc = okc && mbar_wait(&empty_bar[st], ((t / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag);
+      const int tile = okc ? rtile[r] : -1;
       if (!__all_sync(0xffffffffu, okc)) break;
+      if (!q_done && t == 0 && tile >= 0 && (p.early_q || p.pool_mode)) { quantize_q(); q_done = true; }
+      okc = mbar_wait(&empty_bar[st], ((t / p.stages) & 1) ^ 1, kErrWaitSmemEmpty, abort_flag);
+      if (!__all_sync(0xffffffffu, okc)) break;
+      if (tile < 0) {                             // end marker: pass it on to the MMA
+        if (crow == 0) stile[st] = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full_bar[st]);
+        break;
+      }
       uint8_t* stage = smem + L.stage0 + st * STAGE;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -331,6 +407,7 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
           *reinterpret_cast<uint32_t*>(stage + TILE * 64 + half * 512 + sf_chunk_off(crow, 0)) = wv[16];
         }
       }
+      if (crow == 0) stile[st] = tile;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
@@ -338,7 +415,7 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
         mbar_arrive(&rempty_bar[r]);
       }
     }
-    if (!q_done && ntiles > 0) quantize_q();
+    if (!q_done && t > 0) quantize_q();
   } else {
     // ------------------------------------------------------------ epilogue
     pdl_wait();                                   // before w and the first score store
@@ -408,10 +485,13 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
         warp_hist_add(bhist_s, okey(m) >> (32 - p.hb), writer && m != -INFINITY);
       }
     };
+    // local tile i: false at the end marker or a failed wait
     auto epi_tile = [&](int i) -> bool {
       const int a = i & 1;                          // accumulator (and its barriers)
       const bool ok = mbar_wait(&tfull_bar[a], (i >> 1) & 1, kErrWaitTmemFull, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) return false;
+      const int tile = acc_tile[a];
+      if (tile < 0) return false;
       tc_fence_after();
       // this warp's entries: columns CPQ quarter .. + CPQ - 1 of the accumulator
       const uint32_t col = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * TILE + CPQ * quarter;
@@ -429,7 +509,6 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[a]);
-      const int tile = tile_lo + i;
       const int64_t e0 = static_cast<int64_t>(tile) * TILE + CPQ * quarter;
       float x[32];
 #pragma unroll
@@ -440,7 +519,7 @@ index_scan_t_kernel(const __grid_constant__ CUtensorMap tmap_k,
       score_group(x, CPQ - 32, e0 + 32, tile);
       return true;
     };
-    for (int i = set; i < ntiles; i += 2)
+    for (int i = set; first_tile >= 0; i += 2)
       if (!epi_tile(i)) break;
     named_bar_sync(1, kScanEpiThreads);
     const int et = threadIdx.x - 64;

@@ -147,7 +147,8 @@ def test_quantize_validation(L):
 def test_workspace_sizes(L):
     a = _index(B=4, Q=1, K=512, N=131072)
     n = L.csa2_workspace_size(ctypes.byref(a), csa2.WS_INDEX)
-    # scores (4 B per entry per query) + one 4096-bin histogram per query
+    # scores (4 B per entry per query) + one 4096-bin histogram and one
+    # tile counter per query
     assert n >= 4 * 131072 * 4 + 4 * 4096 * 4
     assert n < 4 * 131072 * 4 + 4 * 4096 * 4 + 4096
     assert L.csa2_workspace_size(ctypes.byref(_index(Q=0)), csa2.WS_INDEX) == 0

@@ -71,3 +71,12 @@ def test_both_arms_print_the_same_config():
     c = bench.bench_config(wl, 1)
     assert c["workload"] == "group4_decode_ctx128k_b4" and c["N_entries"] == 131072 and c["r"] == 1
     assert c["layers"] == "full,reindex,reindex,reuse" and c["kv_cache"].startswith("FP4")
+
+
+def test_scan_kernel_names():
+    """One query per MMA group (decode rows, pool re-scores) runs the
+    transposed scan; several queries per group the other one."""
+    assert bench.scan_kernel_name(workloads.WORKLOADS[2], "scan") == "index_scan_t_kernel"
+    assert bench.scan_kernel_name(workloads.WORKLOADS[3], "scan_pool") == "index_scan_t_kernel"
+    assert bench.scan_kernel_name(workloads.WORKLOADS[4], "scan_prefill") == "index_scan_kernel"
+    assert workloads.WORKLOADS[4].Q > 1
