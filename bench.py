@@ -46,8 +46,8 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
 # DRAM traffic (read + write) of one decode scan launch (index_scan_t_kernel)
 # of the default workload, from an ncu capture of that kernel (profiles/),
-# valid only while the scan's sources hash to the recorded value.
-SCAN_TRAFFIC = {"sha": "cdb8913912dfdac0", "bytes_per_launch": 137816832}
+# valid only while the scan's code (comments aside) hashes to the recorded value.
+SCAN_TRAFFIC = {"sha": "6c4f3ac246280bd5", "bytes_per_launch": 137816832}
 
 
 def parse():
@@ -298,10 +298,39 @@ def step_algorithmic_bytes(wl):
     return total
 
 
+def code_tokens(text):
+    """C/C++ source without its comments, whitespace runs collapsed to one
+    space: what the compiler sees, so that editing a comment does not
+    change the digest.  String and character literals are kept whole."""
+    out = []
+    i, n = 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_sha():
+    """Digest of the decode scan's sources (comments and layout ignored)."""
     h = hashlib.sha256()
     for f in ("common.cuh", "index_scan.cuh", "index_scan_t.cuh"):
-        h.update(open(os.path.join(ROOT, "fp4_kv_cache_mxfp4_b200", "csrc", f), "rb").read())
+        with open(os.path.join(ROOT, "fp4_kv_cache_mxfp4_b200", "csrc", f)) as fh:
+            h.update(code_tokens(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

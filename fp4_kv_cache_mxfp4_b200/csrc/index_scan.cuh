@@ -10,6 +10,10 @@
 // epilogue thread then owns one entry: it reads its 32*QG head values from
 // TMEM and reduces them to QG scores (ReLU, weight, sum).
 //
+// This kernel serves rows with two or more queries (query blocks, prefill).
+// One query per group (decode rows, HSI pool re-scores) runs the transposed
+// kernel of index_scan_t.cuh, which shares these parameters and constants.
+//
 // Warp roles (320 threads; 448 with MXFP4 index-K):
 //   warp 0      TMA producer: streams index-K tiles into an S-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer

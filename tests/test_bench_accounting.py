@@ -80,3 +80,16 @@ def test_scan_kernel_names():
     assert bench.scan_kernel_name(workloads.WORKLOADS[3], "scan_pool") == "index_scan_t_kernel"
     assert bench.scan_kernel_name(workloads.WORKLOADS[4], "scan_prefill") == "index_scan_kernel"
     assert workloads.WORKLOADS[4].Q > 1
+
+
+def test_source_digest_ignores_comments_not_code():
+    """The recorded scan traffic stays valid across comment edits and is
+    dropped by any change of code."""
+    src = 'int f(int a) {  // the query\'s tile\n  /* two\n lines */ return a + 1; }\nconst char* s = "//x";\n'
+    base = bench.code_tokens(src)
+    assert base == 'int f(int a) { return a + 1; } const char* s = "//x";'
+    assert bench.code_tokens(src.replace("the query's tile", "another comment")) == base
+    assert bench.code_tokens(src.replace("  return", "\n\n    return")) == base
+    assert bench.code_tokens(src.replace("a + 1", "a + 2")) != base
+    assert bench.code_tokens(src.replace('"//x"', '"//y"')) != base
+    assert len(bench.kernel_source_sha()) == 16
