@@ -225,6 +225,9 @@ csa2_status validate_index(const csa2_index_args* a) {
   if (a->mode == CSA2_REINDEX_POOL && !a->pool_in) return CSA2_ERR_ARG;
   if (a->k_format != CSA2_FMT_BF16 && a->k_format != CSA2_FMT_MXFP4) return CSA2_ERR_ARG;
   if (a->k_format == CSA2_FMT_MXFP4 && (a->N & 3)) return CSA2_ERR_SHAPE;   // 16-byte aligned raw tiles
+  // a pool block of MXFP4 entries is fetched whole (8 x 68 B by one bulk
+  // copy, which has no bounds check): the blocks must tile each row
+  if (a->k_format == CSA2_FMT_MXFP4 && (hsi || a->mode == CSA2_REINDEX_POOL) && (a->N & 7)) return CSA2_ERR_SHAPE;
   if (!aligned16(a->qI) || !aligned16(a->w) || !aligned16(a->kI) || !aligned16(a->n_vis) || !aligned16(a->idx) ||
       (a->scores && !aligned16(a->scores)) || (hsi && !aligned16(a->pool_out)) ||
       (a->mode == CSA2_REINDEX_POOL && !aligned16(a->pool_in)))

@@ -213,7 +213,9 @@ csa2_status csa2_quantize_index_k_mxfp4(const void* x, int64_t n, int64_t ld_x,
  *   (ascending positions for an ascending pool).
  *
  * k_format CSA2_FMT_MXFP4: kI holds 68-byte MXFP4 entries [B][N][68]
- *   (csa2_quantize_index_k_mxfp4; N a multiple of 4).  The page has the
+ *   (csa2_quantize_index_k_mxfp4; N a multiple of 4, and of 8 when an HSI
+ *   pool is built or re-scored, since a pool block is fetched whole;
+ *   CSA2_ERR_SHAPE otherwise).  The page has the
  *   indexer's Q and K both in FP4, so index-Q (given in bf16) is quantised
  *   by the same rule inside the call (each head row of 128 dims, blocks of
  *   32: e = floor(log2 amax) - 2, q = E2M1(x / 2^e)) and the scores are

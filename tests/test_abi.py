@@ -111,6 +111,13 @@ def _call_attn(L, a, ws=FAKE, ws_bytes=0):
     (dict(N=2 ** 31), 2), (dict(hsi_blocks=-1), 2), (dict(hsi_blocks=2048, hsi_block=16, pool_out=FAKE), 2),
     (dict(hsi_blocks=2048, pool_out=None), 1), (dict(mode=2, hsi_blocks=2048, pool_in=None), 1),
     (dict(qI=FAKE + 8), 3), (dict(kI=FAKE + 4), 3), (dict(scores=FAKE + 2), 3),
+    # MXFP4 index-K: N a multiple of 4, and of 8 with an HSI pool (whole-block fetches)
+    (dict(k_format=2, N=4098), 2), (dict(k_format=2, N=4100), 4),
+    (dict(k_format=2, N=4100, hsi_blocks=512, pool_out=FAKE), 2),
+    (dict(k_format=2, N=4100, mode=2, hsi_blocks=512, pool_in=FAKE), 2),
+    (dict(k_format=2, N=4104, hsi_blocks=512, pool_out=FAKE), 4),
+    (dict(k_format=2, N=4104, mode=2, hsi_blocks=512, pool_in=FAKE), 4),
+    (dict(N=4100, hsi_blocks=512, pool_out=FAKE), 4),      # bf16 index-K: TMA bounds the blocks
     (dict(), 4),                       # valid arguments, zero-byte workspace
 ])
 def test_index_validation(L, kw, status):
