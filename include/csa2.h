@@ -107,7 +107,9 @@ typedef enum csa2_mode {
  *   dst_rows  optional int64 [n]: entry i goes to row dst_rows[i];
  *             NULL means row row_offset + i
  *   row_offset  first destination row when dst_rows is NULL, >= 0
- * Entries map to distinct rows (overlapping destinations race).
+ * Entries map to distinct rows (overlapping destinations race).  The call
+ * does not know the cache's size: every destination row must lie inside
+ * kv_fp4 (the caller's contract; nothing checks it).
  * Errors: ARG (x or kv_fp4 NULL with n > 0), SHAPE (n < 0, ld_x < 512,
  * row_offset < 0), ALIGN, CUDA.
  * ---------------------------------------------------------------------- */
