@@ -15,8 +15,9 @@ from test_gpu_stack import DECODER, ENCODER
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("per_layer", [True, False], ids=["per_layer", "coarse"])
 @pytest.mark.parametrize("wl", [workloads.WORKLOADS[0], DECODER, ENCODER], ids=lambda w: w.name)
-def test_io_call_matches_the_plain_call(wl):
+def test_io_call_matches_the_plain_call(wl, per_layer):
     csa2.load()
     T = make_device_workload(wl, csa2)
     run_step(T, csa2)
@@ -27,7 +28,7 @@ def test_io_call_matches_the_plain_call(wl):
 
     host_in = T["inputs"].cpu().pin_memory()
     host_out = torch.empty_like(T["outputs"], device="cpu").pin_memory()
-    io = csa2.io_args(*io_copies(T, host_in, host_out))
+    io = csa2.io_args(*io_copies(T, host_in, host_out, per_layer=per_layer))
 
     def scramble():
         T["inputs"].zero_()
