@@ -36,7 +36,8 @@ sys.path.insert(0, ROOT)
 
 from fp4_kv_cache_mxfp4_b200 import build as _build  # noqa: E402
 from fp4_kv_cache_mxfp4_b200 import workloads  # noqa: E402
-from fp4_kv_cache_mxfp4_b200.device_workload import make_device_workload, run_step, set_flags, set_q_format  # noqa: E402
+from fp4_kv_cache_mxfp4_b200.device_workload import (io_copies, make_device_workload, run_step, run_step_io,  # noqa: E402
+                                                     set_flags, set_q_format)
 
 METRIC = "CSA2 decode queries/s and HBM GB/s vs peak at 128K ctx, FP4 main KV"
 UNIT = "queries/s"
@@ -633,8 +634,22 @@ def run_ours(args, world, rank, local):
     def d2h_copies():
         host_out.copy_(T["outputs"], non_blocking=True)
 
-    e2e_ms = time_steps(call(0), args.steps, flush, st, world, h2d_copies, d2h_copies)
-    e2e_graph_ms = time_steps(graphs["model"].replay, args.steps, flush, st, world, h2d_copies, d2h_copies)
+    e2e_serial_ms = time_steps(call(0), args.steps, flush, st, world, h2d_copies, d2h_copies)
+    # the overlapped-copy call: each layer's inputs move in while earlier
+    # layers run, each layer's output moves out while later layers run
+    io = csa2.io_args(*io_copies(T, host_in, host_out))
+
+    def io_step():
+        set_flags(T, 0)
+        run_step_io(T, csa2, io)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        io_step()
+    e2e_ms = time_steps(io_step, args.steps, flush, st, world)
+    io_graph = capture(io_step)
+    e2e_graph_ms = time_steps(io_graph.replay, args.steps, flush, st, world)
+    del io_graph
     clk = clocks.stop()
     st_code = csa2.csa2_device_status()
     if st_code != (0, 0):
@@ -705,10 +720,15 @@ def run_ours(args, world, rank, local):
                        "(each kernel timed alone; mean over the timed replays)",
         "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "how": "eager library call per step through the C ABI, H2D of the step's inputs (one pinned "
-                       "buffer, one copy) and D2H of every layer's output (one copy) inside the events"},
+                "how": "eager csa2_group_decode_io / csa2_stack_decode_io call per step through the C ABI: "
+                       "every layer's inputs copied in from pinned host memory before that layer, every "
+                       "layer's output copied out after it, overlapped with the other layers, all inside "
+                       "the events"},
         "e2e_graph": {"value": queries / (e2e_graph_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_graph_ms,
-                      "how": "the same copies around a CUDA-graph replay of the call"},
+                      "how": "the same call captured as one CUDA graph (copies included) and replayed"},
+        "e2e_serial_copies": {"value": queries / (e2e_serial_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_serial_ms,
+                              "how": "eager csa2_group_decode / csa2_stack_decode call with one H2D copy of all "
+                                     "inputs before it and one D2H copy of all outputs after it"},
         "gpu_launches": len(labels) * args.steps,
         "clocks": clk,
     }

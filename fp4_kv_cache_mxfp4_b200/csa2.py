@@ -67,6 +67,14 @@ class StackArgs(ctypes.Structure):
     _fields_ = [("n_groups", _c_i32), ("groups", ctypes.POINTER(GroupArgs))]
 
 
+class Copy(ctypes.Structure):
+    _fields_ = [("dst", _c_p), ("src", _c_p), ("bytes", ctypes.c_size_t), ("layer", _c_i32)]
+
+
+class Io(ctypes.Structure):
+    _fields_ = [("in_", ctypes.POINTER(Copy)), ("n_in", _c_i32), ("out", ctypes.POINTER(Copy)), ("n_out", _c_i32)]
+
+
 _lib = None
 
 
@@ -88,6 +96,8 @@ def load(path=LIB_PATH):
     lib.csa2_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_group_decode.argtypes = [ctypes.POINTER(GroupArgs), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_stack_decode.argtypes = [ctypes.POINTER(StackArgs), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_group_decode_io.argtypes = [ctypes.POINTER(GroupArgs), ctypes.POINTER(Io), _c_p, ctypes.c_size_t, _c_p]
+    lib.csa2_stack_decode_io.argtypes = [ctypes.POINTER(StackArgs), ctypes.POINTER(Io), _c_p, ctypes.c_size_t, _c_p]
     lib.csa2_noalloc_scratch_bytes.argtypes = []
     lib.csa2_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.csa2_workspace_size.argtypes = [_c_p, _c_i32]
@@ -106,7 +116,8 @@ def load(path=LIB_PATH):
     for name in ("csa2_quantize_kv_fp4", "csa2_quantize_window_fp8", "csa2_quantize_index_k_mxfp4",
                  "csa2_compress_rope_quantize_kv_fp4",
                  "csa2_index_score_topk", "csa2_index_score_topk_noalloc", "csa2_sparse_attn",
-                 "csa2_group_decode", "csa2_stack_decode", "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
+                 "csa2_group_decode", "csa2_stack_decode", "csa2_group_decode_io", "csa2_stack_decode_io",
+                 "csa2_device_status", "csa2_trace_begin", "csa2_trace_stop",
                  "csa2_trace_end", "csa2_trace_get"):
         getattr(lib, name).restype = _c_i32
     _lib = lib
@@ -279,6 +290,32 @@ def csa2_stack_decode(args, ws, stream=None):
 def csa2_group_decode(args, ws, stream=None):
     _check(load().csa2_group_decode(ctypes.byref(args), _ptr(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)), "csa2_group_decode")
+
+
+def io_args(copies_in, copies_out):
+    """csa2_io over two lists of (dst, src, bytes, layer) tuples (addresses
+    as ints), each in non-decreasing layer order; the arrays are kept alive
+    by the returned struct."""
+    def arr(cs):
+        a = (Copy * max(len(cs), 1))()
+        for i, (dst, src, n, layer) in enumerate(cs):
+            a[i] = Copy(dst=dst, src=src, bytes=n, layer=layer)
+        return a
+    ai, ao = arr(copies_in), arr(copies_out)
+    io = Io(in_=ctypes.cast(ai, ctypes.POINTER(Copy)), n_in=len(copies_in),
+            out=ctypes.cast(ao, ctypes.POINTER(Copy)), n_out=len(copies_out))
+    io._arrays = (ai, ao)
+    return io
+
+
+def csa2_group_decode_io(args, io, ws, stream=None):
+    _check(load().csa2_group_decode_io(ctypes.byref(args), ctypes.byref(io), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)), "csa2_group_decode_io")
+
+
+def csa2_stack_decode_io(args, io, ws, stream=None):
+    _check(load().csa2_stack_decode_io(ctypes.byref(args), ctypes.byref(io), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)), "csa2_stack_decode_io")
 
 
 def csa2_workspace_size(args, which):

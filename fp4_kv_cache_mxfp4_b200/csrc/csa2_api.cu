@@ -7,6 +7,7 @@
 #include <math.h>
 #include <algorithm>
 #include <mutex>
+#include <vector>
 #include <string.h>
 
 #include "common.cuh"
@@ -628,12 +629,134 @@ csa2_status check_group(const csa2_group_args* g, size_t* iz, size_t* iw, size_t
   return CSA2_OK;
 }
 
+// ---------------------------------------------------------------- overlapped host copies
+// The copy streams and events of csa2_*_decode_io, one set per device,
+// created on first use and kept for the life of the process.
+struct IoDevice {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+IoDevice g_io[kMaxDevices];
+
+csa2_status validate_copies(const csa2_copy* c, int32_t n, int n_layers) {
+  if (n < 0 || (n > 0 && !c)) return CSA2_ERR_ARG;
+  int prev = 0;
+  for (int i = 0; i < n; ++i) {
+    if (!c[i].dst || !c[i].src || c[i].layer < 0 || c[i].layer >= n_layers || c[i].layer < prev) return CSA2_ERR_ARG;
+    prev = c[i].layer;
+  }
+  return CSA2_OK;
+}
+
+csa2_status validate_io(const csa2_io* io, int n_layers) {
+  if (!io) return CSA2_ERR_ARG;
+  const csa2_status s = validate_copies(io->in, io->n_in, n_layers);
+  return s != CSA2_OK ? s : validate_copies(io->out, io->n_out, n_layers);
+}
+
+// One io call: which layers have copies, their events, and the hooks the
+// group runner calls around each layer.  Event 0 marks the call's start on
+// the caller's stream, events 1 and 2 the ends of the two copy streams,
+// then one per layer with input copies and one per layer with outputs.
+struct IoRun {
+  const csa2_io* io = nullptr;
+  IoDevice* d = nullptr;
+  cudaStream_t st = nullptr;
+  std::vector<int> ev_in, ev_out;   // per layer: event index, -1 if none
+  std::vector<char> waited;
+};
+
+cudaError_t io_fail(cudaError_t e) {
+  if (e != cudaSuccess) g_last_cuda_error = e;
+  return e;
+}
+
+// Resources, then every input copy in order on the H2D stream (each layer's
+// last copy followed by that layer's event).
+csa2_status io_begin(IoRun* r, const csa2_io* io, int n_layers, cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
+  r->io = io;
+  r->st = st;
+  r->ev_in.assign(n_layers, -1);
+  r->ev_out.assign(n_layers, -1);
+  r->waited.assign(n_layers, 0);
+  int n_ev = 3;
+  for (int i = 0; i < io->n_in; ++i)
+    if (r->ev_in[io->in[i].layer] < 0) r->ev_in[io->in[i].layer] = n_ev++;
+  for (int i = 0; i < io->n_out; ++i)
+    if (r->ev_out[io->out[i].layer] < 0) r->ev_out[io->out[i].layer] = n_ev++;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    IoDevice& d = g_io[dev];
+    if (!d.h2d && io_fail(cudaStreamCreateWithFlags(&d.h2d, cudaStreamNonBlocking)) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (!d.d2h && io_fail(cudaStreamCreateWithFlags(&d.d2h, cudaStreamNonBlocking)) != cudaSuccess) return CSA2_ERR_CUDA;
+    while (static_cast<int>(d.ev.size()) < n_ev) {
+      cudaEvent_t e;
+      if (io_fail(cudaEventCreateWithFlags(&e, cudaEventDisableTiming)) != cudaSuccess) return CSA2_ERR_CUDA;
+      d.ev.push_back(e);
+    }
+    r->d = &d;
+  }
+  IoDevice& d = *r->d;
+  if (io_fail(cudaEventRecord(d.ev[0], st)) != cudaSuccess ||
+      io_fail(cudaStreamWaitEvent(d.h2d, d.ev[0], 0)) != cudaSuccess ||
+      io_fail(cudaStreamWaitEvent(d.d2h, d.ev[0], 0)) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  for (int i = 0; i < io->n_in; ++i) {
+    const csa2_copy& c = io->in[i];
+    if (c.bytes > 0 && io_fail(cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, d.h2d)) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+    if ((i + 1 == io->n_in || io->in[i + 1].layer != c.layer) &&
+        io_fail(cudaEventRecord(d.ev[r->ev_in[c.layer]], d.h2d)) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+  }
+  return CSA2_OK;
+}
+
+// Before layer l's first kernel: its input copies have landed.
+csa2_status io_before_layer(IoRun* r, int l) {
+  if (!r || r->ev_in[l] < 0 || r->waited[l]) return CSA2_OK;
+  r->waited[l] = 1;
+  return io_fail(cudaStreamWaitEvent(r->st, r->d->ev[r->ev_in[l]], 0)) == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
+// After layer l's attention: its output copies go out on the D2H stream.
+csa2_status io_after_layer(IoRun* r, int l) {
+  if (!r || r->ev_out[l] < 0) return CSA2_OK;
+  IoDevice& d = *r->d;
+  const cudaEvent_t e = d.ev[r->ev_out[l]];
+  if (io_fail(cudaEventRecord(e, r->st)) != cudaSuccess || io_fail(cudaStreamWaitEvent(d.d2h, e, 0)) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  for (int i = 0; i < r->io->n_out; ++i) {
+    const csa2_copy& c = r->io->out[i];
+    if (c.layer == l && c.bytes > 0 &&
+        io_fail(cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToHost, d.d2h)) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+  }
+  return CSA2_OK;
+}
+
+// Both copy streams join the caller's stream (also after a failure, so
+// that no copy stream is left forked from a capture).
+csa2_status io_end(IoRun* r) {
+  if (!r->d) return CSA2_OK;
+  IoDevice& d = *r->d;
+  const bool ok = io_fail(cudaEventRecord(d.ev[1], d.h2d)) == cudaSuccess &&
+                  io_fail(cudaEventRecord(d.ev[2], d.d2h)) == cudaSuccess &&
+                  io_fail(cudaStreamWaitEvent(r->st, d.ev[1], 0)) == cudaSuccess &&
+                  io_fail(cudaStreamWaitEvent(r->st, d.ev[2], 0)) == cudaSuccess;
+  return ok ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
 // Enqueue one validated group on `st` (workspace already large enough).
 // first_early: the first layer's inputs were complete before the call
 // (false for a group of a stack after the first: its first layer follows
 // the previous group's last layer in model order)
+// io / layer_base: the overlapped copies of an io call and the index of the
+// group's first layer among the call's layers (nullptr / 0 otherwise)
 csa2_status run_group(const csa2_group_args* g, size_t iz, size_t iw, const DeviceInfo& dev, void* ws,
-                      cudaStream_t st, bool first_early = true) {
+                      cudaStream_t st, bool first_early = true, IoRun* io = nullptr, int layer_base = 0) {
   struct SerialScope {                             // CSA2_GROUP_SERIAL: plain stream order for this call
     bool prev;
     explicit SerialScope(bool on) : prev(g_serial_launch) { if (on) g_serial_launch = true; }
@@ -644,6 +767,7 @@ csa2_status run_group(const csa2_group_args* g, size_t iz, size_t iw, const Devi
   uint8_t* dws = zws + iz;                         // data region shared by the layers in turn
   uint8_t* aws = zws + iw;
   if (cudaMemsetAsync(zws, 0, iz, st) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (io_before_layer(io, layer_base) != CSA2_OK) return CSA2_ERR_CUDA;    // the new entries
   if (g->n_new > 0) {
     if (launch_quantize(g->kv_new, g->n_new, 512, g->kv_fp4, g->new_rows, 0, st) != cudaSuccess) return CSA2_ERR_CUDA;
   }
@@ -654,6 +778,7 @@ csa2_status run_group(const csa2_group_args* g, size_t iz, size_t iw, const Devi
     // the first layer's inputs precede the call; a later layer's are, in a
     // model, the previous layer's results unless the caller says otherwise
     const bool early = inputs_ready || (i == 0 && first_early);
+    if (io_before_layer(io, layer_base + i) != CSA2_OK) return CSA2_ERR_CUDA;
     if (L.mode != CSA2_REUSE) {
       const csa2_index_args a = layer_index_args(g, L, cur_pool);
       const csa2_status s = run_index(&a, dev, zws, dws, st, g->kv_fp4, early);
@@ -665,6 +790,7 @@ csa2_status run_group(const csa2_group_args* g, size_t iz, size_t iw, const Devi
     const csa2_attn_args aa = layer_attn_args(g, L, last_idx);
     const csa2_status s = run_attn(&aa, aws, st, early);
     if (s != CSA2_OK) return s;
+    if (io_after_layer(io, layer_base + i) != CSA2_OK) return CSA2_ERR_CUDA;
   }
   return CSA2_OK;
 }
@@ -872,6 +998,50 @@ csa2_status csa2_stack_decode(const csa2_stack_args* sa, void* ws, size_t ws_byt
   return CSA2_OK;
 }
 
+csa2_status csa2_group_decode_io(const csa2_group_args* g, const csa2_io* io, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  size_t iz = 0, iw = 0, need = 0;
+  csa2_status s = check_group(g, &iz, &iw, &need);
+  if (s != CSA2_OK) return s;
+  s = validate_io(io, g->n_layers);
+  if (s != CSA2_OK) return s;
+  if (!ws || ws_bytes < need || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  IoRun r;
+  s = io_begin(&r, io, g->n_layers, st);
+  if (s == CSA2_OK) s = run_group(g, iz, iw, *dev, ws, st, true, &r, 0);
+  const csa2_status e = io_end(&r);
+  return s != CSA2_OK ? s : e;
+}
+
+csa2_status csa2_stack_decode_io(const csa2_stack_args* sa, const csa2_io* io, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  size_t need = 0;
+  csa2_status s = validate_stack(sa, &need);
+  if (s != CSA2_OK) return s;
+  int n_layers = 0;
+  for (int i = 0; i < sa->n_groups; ++i) n_layers += sa->groups[i].n_layers;
+  s = validate_io(io, n_layers);
+  if (s != CSA2_OK) return s;
+  if (!ws || ws_bytes < need || !aligned16(ws)) return CSA2_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  s = device_info(&dev);
+  if (s != CSA2_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  IoRun r;
+  s = io_begin(&r, io, n_layers, st);
+  for (int i = 0, base = 0; s == CSA2_OK && i < sa->n_groups; base += sa->groups[i].n_layers, ++i) {
+    size_t iz = 0, iw = 0, n = 0;
+    check_group(&sa->groups[i], &iz, &iw, &n);
+    s = run_group(&sa->groups[i], iz, iw, *dev, ws, st, i == 0, &r, base);
+  }
+  const csa2_status e = io_end(&r);
+  return s != CSA2_OK ? s : e;
+}
+
 size_t csa2_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 size_t csa2_workspace_size(const void* args, int32_t which) {
@@ -928,7 +1098,7 @@ const char* csa2_status_string(int32_t s) {
   }
 }
 
-int32_t csa2_version(void) { return 106; }
+int32_t csa2_version(void) { return 107; }
 
 csa2_status csa2_trace_begin(int32_t max_launches) {
   if (max_launches < 1 || max_launches > (1 << 20)) return CSA2_ERR_SHAPE;

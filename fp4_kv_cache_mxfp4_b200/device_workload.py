@@ -155,6 +155,63 @@ def set_q_format(T, q_format, csa2):
             T["stack"]._group_array[i].q_format = q_format
 
 
+def _span(views, base):
+    """(offset, bytes) of the arena range that holds `views`."""
+    lo = min(v.data_ptr() for v in views)
+    hi = max(v.data_ptr() + v.numel() * v.element_size() for v in views)
+    return lo - base, hi - lo
+
+
+def io_copies(T, host_in, host_out, per_layer=False):
+    """The host<->device copies of a staged step for the overlapped-copy
+    calls, through host mirrors of its input and output buffers (same
+    offsets): each cache's new entries before the first layer of the group
+    that quantises them, each layer's qI, w and q (one range) before that
+    layer, each layer's output after it.  Returns two lists of
+    (dst, src, bytes, layer) in layer order.
+
+    Every distinct layer named is a synchronisation point between the
+    caller's stream and a copy stream.  per_layer=False names as few as the
+    step allows: the inputs of layer 0 (and the new entries) before layer
+    0, all other inputs before layer 1 (an earlier layer than they need);
+    every output but the last layer's after the second-to-last layer (a
+    later one than they need), the last layer's after it."""
+    wl = T["wl"]
+    n = len(T["layers"])
+
+    def tag_in(l):
+        return l if per_layer else min(l, 1)
+
+    def tag_out(l):
+        return l if per_layer else max(l, n - 2)
+
+    din, dout = T["inputs"].data_ptr(), T["outputs"].data_ptr()
+    hin, hout = host_in.data_ptr(), host_out.data_ptr()
+    ins = []
+    for g in range(len(wl.groups)):
+        if g == 0 or wl.cache_per_group:
+            off, nb = _span([T["caches"][g if wl.cache_per_group else 0]["new"]], din)
+            ins.append((din + off, hin + off, nb, tag_in(wl.group_layers(g)[0])))
+    for l, L in enumerate(T["layers"]):
+        off, nb = _span([L["qI"], L["w"], L["q"]], din)
+        ins.append((din + off, hin + off, nb, tag_in(l)))
+    ins.sort(key=lambda c: c[3])
+    outs = []
+    for l, L in enumerate(T["layers"]):
+        off, nb = _span([L["out"]], dout)
+        outs.append((hout + off, dout + off, nb, tag_out(l)))
+    return ins, outs
+
+
+def run_step_io(T, csa2, io, stream=None):
+    """One step with its copies overlapped: csa2_group_decode_io or
+    csa2_stack_decode_io."""
+    if T["stack"] is None:
+        csa2.csa2_group_decode_io(T["g"], io, T["ws"], stream)
+    else:
+        csa2.csa2_stack_decode_io(T["stack"], io, T["ws"], stream)
+
+
 def run_step(T, csa2, stream=None):
     """One step through the library's public call: csa2_group_decode for one
     group, csa2_stack_decode for a stack."""

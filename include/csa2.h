@@ -442,6 +442,57 @@ typedef struct csa2_stack_args {
 csa2_status csa2_stack_decode(const csa2_stack_args* s, void* ws,
                               size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * csa2_group_decode_io / csa2_stack_decode_io -- the same step as
+ * csa2_group_decode / csa2_stack_decode, with the step's host<->device
+ * copies overlapped with its layers: a caller whose per-layer inputs (new
+ * entries, index-Q, w, q) sit in host memory and who wants the outputs
+ * back in host memory gets the copies hidden behind the layers that do
+ * not need them, instead of a copy in before the step and a copy out
+ * after it.
+ *
+ * Each copy names a layer, counted over the call's layers (a stack counts
+ * through its groups in order):
+ *   in[i]   host -> device; it has landed before the first kernel of layer
+ *           in[i].layer reads anything (a group's quantise step belongs to
+ *           its first layer, so the new entries name that layer);
+ *   out[i]  device -> host; it starts once layer out[i].layer's attention
+ *           has finished.
+ * Copies of each list are in non-decreasing layer order.  The input copies
+ * start after all work enqueued on `stream` before the call (a step may
+ * overwrite the device inputs the previous step read), all of them at
+ * once, in order, on a copy stream of the library's; the outputs go out on
+ * a second copy stream.  Both join `stream` before the call's last
+ * operation, so everything the call does, copies included, is ordered on
+ * `stream` (and a stream capture of the call records the copies as well).
+ * Host memory must be page-locked (cudaHostAlloc, cudaHostRegister) for
+ * copies to overlap and for capture.
+ *
+ * The copy streams and their events belong to the library, one set per
+ * device: io calls on one device must not overlap in time.
+ * Errors: those of csa2_group_decode / csa2_stack_decode; ARG when io is
+ * NULL, a count is negative, a list with copies is NULL, a copy has a NULL
+ * pointer or names a layer outside the call, or a list is out of order.
+ * ---------------------------------------------------------------------- */
+typedef struct csa2_copy {
+    void*       dst;
+    const void* src;
+    size_t      bytes;         /* 0: nothing to copy                             */
+    int32_t     layer;         /* see above                                      */
+} csa2_copy;
+
+typedef struct csa2_io {
+    const csa2_copy* in;       /* HOST array of n_in host->device copies         */
+    int32_t          n_in;
+    const csa2_copy* out;      /* HOST array of n_out device->host copies        */
+    int32_t          n_out;
+} csa2_io;
+
+csa2_status csa2_group_decode_io(const csa2_group_args* g, const csa2_io* io, void* ws,
+                                 size_t ws_bytes, void* stream);
+csa2_status csa2_stack_decode_io(const csa2_stack_args* s, const csa2_io* io, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* Workspace bytes needed by a call.  which = 1: csa2_index_args,
  * 2: csa2_attn_args, 3: csa2_group_args, 4: csa2_stack_args.  Returns 0
  * when the arguments are invalid for that call.

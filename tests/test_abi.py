@@ -42,10 +42,14 @@ def test_every_declared_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert csa2.version() == 106
+    assert csa2.version() == 107
     assert csa2.status_string(0) == "ok"
     assert "workspace" in csa2.status_string(4)
     assert csa2.status_string(99) == "unknown status"
+
+
+# Python field names that differ from the header's (`in` is a keyword)
+_C_NAME = {"in_": "in"}
 
 
 def _c_layout():
@@ -56,6 +60,8 @@ def _c_layout():
         "csa2_group_args": [f for f, _ in csa2.GroupArgs._fields_],
         "csa2_stack_args": [f for f, _ in csa2.StackArgs._fields_],
         "csa2_compress_args": [f for f, _ in csa2.CompressArgs._fields_],
+        "csa2_copy": [f for f, _ in csa2.Copy._fields_],
+        "csa2_io": [_C_NAME.get(f, f) for f, _ in csa2.Io._fields_],
     }
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "csa2.h"', "int main(void) {"]
     for s, fs in fields.items():
@@ -75,10 +81,11 @@ def test_struct_layouts_match_the_header():
     c = _c_layout()
     for cname, py in [("csa2_index_args", csa2.IndexArgs), ("csa2_attn_args", csa2.AttnArgs),
                       ("csa2_layer", csa2.Layer), ("csa2_group_args", csa2.GroupArgs),
-                      ("csa2_stack_args", csa2.StackArgs), ("csa2_compress_args", csa2.CompressArgs)]:
+                      ("csa2_stack_args", csa2.StackArgs), ("csa2_compress_args", csa2.CompressArgs),
+                      ("csa2_copy", csa2.Copy), ("csa2_io", csa2.Io)]:
         assert int(c[cname]) == ctypes.sizeof(py), cname
         for f, _ in py._fields_:
-            assert int(c[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
+            assert int(c[f"{cname}.{_C_NAME.get(f, f)}"]) == getattr(py, f).offset, (cname, f)
 
 
 def _index(**kw):
@@ -305,3 +312,43 @@ def test_compress_validation(L):
     assert args(x=FAKE + 8) == 3 and args(sin=FAKE + 2) == 3
     assert args(n_entries=0, x=None) == 0
 
+
+
+def test_io_validation(L):
+    """The overlapped-copy calls check their copy lists (layers inside the
+    call, non-decreasing, no NULL pointer) before anything is enqueued; a
+    valid list reaches the workspace check."""
+    first = (csa2.Layer * 2)()
+    first[0] = csa2.Layer(mode=0, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)
+    first[1] = csa2.Layer(mode=3, q=FAKE, swa=FAKE, out=FAKE)
+    later = (csa2.Layer * 2)()
+    later[0] = csa2.Layer(mode=2, qI=FAKE, w=FAKE, q=FAKE, swa=FAKE, out=FAKE, idx=FAKE)
+    later[1] = csa2.Layer(mode=3, q=FAKE, swa=FAKE, out=FAKE)
+    g1, g2 = _group(first), _group(later, pool_in=FAKE)
+    st = csa2.stack_args([g1, g2])
+
+    def group(io):
+        return L.csa2_group_decode_io(ctypes.byref(g1), io and ctypes.byref(io), ctypes.c_void_p(FAKE), 0, None)
+
+    def stack(io):
+        return L.csa2_stack_decode_io(ctypes.byref(st), ctypes.byref(io), ctypes.c_void_p(FAKE), 0, None)
+
+    ok_in = [(FAKE, FAKE, 64, 0), (FAKE, FAKE, 64, 0), (FAKE, FAKE, 0, 1)]
+    ok_out = [(FAKE, FAKE, 64, 0), (FAKE, FAKE, 64, 1)]
+    assert group(csa2.io_args(ok_in, ok_out)) == 4                          # valid: workspace next
+    assert group(csa2.io_args([], [])) == 4
+    assert group(None) == 1
+    assert group(csa2.io_args([(FAKE, FAKE, 64, 2)], [])) == 1              # layer outside the group
+    assert group(csa2.io_args([], [(FAKE, FAKE, 64, -1)])) == 1
+    assert group(csa2.io_args([(FAKE, FAKE, 64, 1), (FAKE, FAKE, 64, 0)], [])) == 1   # out of order
+    assert group(csa2.io_args([(None, FAKE, 64, 0)], [])) == 1
+    assert group(csa2.io_args([], [(FAKE, None, 64, 0)])) == 1
+    neg = csa2.io_args([], [])
+    neg.n_in = -1
+    assert group(neg) == 1
+    missing = csa2.io_args([], [])
+    missing.n_out, missing.out = 1, None
+    assert group(missing) == 1
+    # a stack counts its layers through the groups: 4 here
+    assert stack(csa2.io_args([(FAKE, FAKE, 64, 0), (FAKE, FAKE, 64, 2)], [(FAKE, FAKE, 64, 3)])) == 4
+    assert stack(csa2.io_args([(FAKE, FAKE, 64, 4)], [])) == 1
